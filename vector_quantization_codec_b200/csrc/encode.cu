@@ -1,0 +1,536 @@
+// encode.cu -- QAM-W encoder (paper section 3.1 steps 1-6, section 3.4, and the
+// activation-aware per-channel scaling).
+//
+// Kernels, in stream order:
+//   k_scales        s_j = binary16((a_j / mean a)^alpha)          (1 CTA)
+//   k_rownorm       r_i = ||w_i * s||_2 (fp32), r_hat = binary16(r) (warp/row)
+//   k_calib_select  the first min(1024, #non-zero) non-zero rows   (1 CTA)
+//   k_calib_accum   per-CTA sums of |z_k| over those rows           (128 CTAs)
+//   k_calib_finish  sigma_k = binary16(sum / (n sqrt(pi/2)))        (thread/pair)
+//   k_encode        rotate, normalise, nearest codeword, pack        (thread/chunk)
+// W is read twice from HBM-sized storage (norms, then encode); per matrix both
+// passes fit in L2 for the matrix sizes of LLM layers.
+#include "common.cuh"
+#include "launch.cuh"
+
+namespace qamw {
+namespace {
+
+// ------------------------------------------------------------------ scales
+
+__global__ void __launch_bounds__(1024) k_scales(const float* __restrict__ a, int d_in,
+                                                 float alpha, __half* __restrict__ s,
+                                                 int32_t* status) {
+  __shared__ double red[32];
+  int bad = 0;
+  double sum = 0.0;
+  for (int j = threadIdx.x; j < d_in; j += blockDim.x) {
+    const float v = a[j];
+    if (v > 0.f && isfinite(v))
+      sum += (double)v;
+    else
+      bad = 1;
+  }
+  // fixed-order tree reduction (deterministic)
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sum;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    double t = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (threadIdx.x == 0) red[0] = t;
+  }
+  __syncthreads();
+  const double mean = red[0] / (double)d_in;
+  int range = 0;
+  for (int j = threadIdx.x; j < d_in; j += blockDim.x) {
+    const float v = a[j];
+    __half h;
+    if (v > 0.f && isfinite(v)) {
+      h = __double2half(pow((double)v / mean, (double)alpha));
+      const float hf = __half2float(h);
+      if (isinf(hf) || hf == 0.f) range = 1;
+    } else {
+      h = __float2half(1.0f);
+    }
+    s[j] = h;
+  }
+  raise_flag(status, (bad ? QAMW_STATUS_BAD_STAT : 0) | (range ? QAMW_STATUS_RANGE : 0));
+}
+
+__global__ void k_fill_half(__half* p, int n, float v) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) p[i] = __float2half(v);
+}
+
+// --------------------------------------------------------------- row norms
+
+template <typename T>
+struct Vec8;  // 8 consecutive weights
+template <>
+struct Vec8<float> {
+  __device__ static void load(const float* p, float (&x)[8]) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+};
+template <>
+struct Vec8<__nv_bfloat16> {
+  __device__ static void load(const __nv_bfloat16* p, float (&x)[8]) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      x[2 * e] = __uint_as_float(u[e] << 16);
+      x[2 * e + 1] = __uint_as_float(u[e] & 0xffff0000u);
+    }
+  }
+};
+
+__device__ __forceinline__ void load_half8(const __half* p, float (&x)[8]) {
+  const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+  const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __half22float2(h[e]);
+    x[2 * e] = f.x;
+    x[2 * e + 1] = f.y;
+  }
+}
+
+// fp32 row norms of W*s, used to pick and normalise the calibration rows.
+template <typename T>
+__global__ void __launch_bounds__(256) k_rownorm(const T* __restrict__ W,
+                                                 const __half* __restrict__ s, int d_out,
+                                                 int d_in, float* __restrict__ r32,
+                                                 int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int warps = (gridDim.x * blockDim.x) >> 5;
+  int flags = 0;
+  for (int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < d_out; row += warps) {
+    const T* w = W + (int64_t)row * d_in;
+    float ss = 0.f;
+    int nonfinite = 0;
+    for (int j = lane * 8; j < d_in; j += 256) {
+      float x[8], sv[8];
+      Vec8<T>::load(w + j, x);
+      load_half8(s + j, sv);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (!isfinite(x[e])) nonfinite = 1;
+        const float t = x[e] * sv[e];
+        ss = fmaf(t, t, ss);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    nonfinite = __any_sync(0xffffffffu, nonfinite);
+    if (lane == 0) {
+      const float r = sqrtf(ss);
+      r32[row] = r;
+      if (nonfinite || !isfinite(r)) flags |= QAMW_STATUS_NONFINITE;
+    }
+  }
+  raise_flag(status, flags);
+}
+
+// ------------------------------------------------------------- calibration
+
+__global__ void __launch_bounds__(1024) k_calib_select(const float* __restrict__ r32, int d_out,
+                                                       int32_t* __restrict__ cal_rows,
+                                                       int32_t* __restrict__ n_cal) {
+  __shared__ int scan[1024];
+  const int t = threadIdx.x, T = blockDim.x;
+  const int per = (d_out + T - 1) / T;
+  const int lo = min(t * per, d_out), hi = min(lo + per, d_out);
+  int cnt = 0;
+  for (int i = lo; i < hi; ++i) cnt += (r32[i] > 0.f);
+  scan[t] = cnt;
+  __syncthreads();
+  for (int off = 1; off < T; off <<= 1) {  // inclusive Hillis-Steele scan
+    const int v = t >= off ? scan[t - off] : 0;
+    __syncthreads();
+    scan[t] += v;
+    __syncthreads();
+  }
+  int rank = scan[t] - cnt;
+  for (int i = lo; i < hi && rank < kCalRows; ++i)
+    if (r32[i] > 0.f) cal_rows[rank++] = i;
+  if (t == T - 1) *n_cal = min(scan[T - 1], kCalRows);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(1024) k_calib_accum(const T* __restrict__ W,
+                                                      const __half* __restrict__ s,
+                                                      const float* __restrict__ r32,
+                                                      const int32_t* __restrict__ cal_rows,
+                                                      const int32_t* __restrict__ n_cal_p,
+                                                      int d_in, int block, uint64_t seed,
+                                                      float* __restrict__ partial) {
+  extern __shared__ __align__(16) float f[];  // D_j * s_j
+  for (int j = threadIdx.x; j < d_in; j += blockDim.x) {
+    const float v = __half2float(s[j]);
+    f[j] = mask_negative(seed, (uint32_t)j) ? -v : v;
+  }
+  __syncthreads();
+  const int C = d_in / kE, P = d_in / 2;
+  const int c = threadIdx.x;
+  const bool active = c < C;
+  const int nb = min(block, kE), lanes = max(block / kE, 1);
+  const float inv_sqrt_b = 1.0f / sqrtf((float)block);
+  const int n_cal = *n_cal_p;
+  const int per = (kCalRows + gridDim.x - 1) / gridDim.x;
+  const int t0 = blockIdx.x * per, t1 = min(t0 + per, n_cal);
+  float acc[kQ];
+#pragma unroll
+  for (int q = 0; q < kQ; ++q) acc[q] = 0.f;
+  for (int t = t0; t < t1; ++t) {
+    const int row = cal_rows[t];
+    float x[kE];
+    if (active) {
+      load64(W + (int64_t)row * d_in + (int64_t)c * kE, x);
+#pragma unroll
+      for (int j = 0; j < kE; ++j) x[j] *= f[c * kE + j];
+    } else {
+#pragma unroll
+      for (int j = 0; j < kE; ++j) x[j] = 0.f;
+    }
+    fwht_reg<kE>(x, nb);
+    fwht_lanes<kE>(x, lanes);
+    const float inv = inv_sqrt_b / r32[row];
+#pragma unroll
+    for (int q = 0; q < kQ; ++q) {
+      const float zx = x[2 * q] * inv, zy = x[2 * q + 1] * inv;
+      acc[q] += sqrtf(fmaf(zx, zx, zy * zy));
+    }
+  }
+  if (active) {
+    float* dst = partial + (size_t)blockIdx.x * P + c * kQ;
+#pragma unroll
+    for (int q = 0; q < kQ; ++q) dst[q] = acc[q];
+  }
+}
+
+__global__ void k_calib_finish(const float* __restrict__ partial, int nparts,
+                               const int32_t* __restrict__ n_cal_p, int P,
+                               __half* __restrict__ sigma, int32_t* status) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= P) return;
+  double sum = 0.0;
+  for (int p = 0; p < nparts; ++p) sum += (double)partial[(size_t)p * P + k];
+  const int n = *n_cal_p;
+  const double rayleigh = 1.2533141373155002512;  // sqrt(pi/2)
+  __half h = __double2half(n > 0 ? sum / (double)n / rayleigh : 0.0);
+  const float hf = __half2float(h);
+  if (hf == 0.f) h = __float2half(1.0f);
+  if (isinf(hf)) raise_flag(status, QAMW_STATUS_RANGE);
+  sigma[k] = h;
+}
+
+// ---------------------------------------------------------------- encoder
+
+template <typename T>
+struct EncodeArgs {
+  const T* W;
+  const __half* scale;
+  const __half* sigma;
+  const float2* codebook;
+  const void* prefilter;  // nullable: exhaustive search
+  uint8_t* packed;
+  __half* rnorm;
+  int32_t* status;
+  unsigned long long* candidates;  // nullable: codewords scored, summed
+  int64_t row_bytes;
+  int d_out, d_in, block, K;
+  int rows_per_cta;  // R: whole rows per CTA iteration, R * C <= blockDim
+  uint64_t seed;
+};
+
+// One CTA iteration encodes R whole rows; thread (r, c) owns chunk c of row r.
+// Steps 1-6 of section 3.1 in one pass over W: scale by s, sum of squares
+// (reduced per row in a fixed order, so r is bitwise reproducible), Hadamard
+// butterflies, division by r sqrt(b) and sigma_k, nearest codeword, packing.
+template <int BITS, typename T>
+__global__ void __launch_bounds__(512) k_encode(const EncodeArgs<T> a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  float4* cbq = reinterpret_cast<float4*>(smem);
+  float* f = reinterpret_cast<float*>(cbq + a.K);  // D_j * s_j
+  const int P = a.d_in >> 1;
+  float* isg = f + a.d_in;                          // 1 / sigma_k
+  float* part = isg + P;                            // [blockDim] partial sums of squares
+  float* rsum = part + blockDim.x;                  // [R] row norms
+  for (int i = threadIdx.x; i < a.K; i += blockDim.x) cbq[i] = codeword_q(a.codebook[i]);
+  for (int j = threadIdx.x; j < a.d_in; j += blockDim.x) {
+    const float v = __half2float(a.scale[j]);
+    f[j] = mask_negative(a.seed, (uint32_t)j) ? -v : v;
+  }
+  for (int k = threadIdx.x; k < P; k += blockDim.x) isg[k] = 1.0f / __half2float(a.sigma[k]);
+  PrefilterView pf;
+  if (a.prefilter != nullptr) {
+    pf = prefilter_view(a.prefilter, a.K);
+  } else {
+    pf.G = 0;
+    pf.Gf = 0.f;
+  }
+  __syncthreads();
+
+  const int C = a.d_in / kE, R = a.rows_per_cta;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int rl = threadIdx.x / C, c = threadIdx.x - rl * C;
+  const int nb = min(a.block, kE), lanes = max(a.block / kE, 1);
+  const float sqrt_b = sqrtf((float)a.block);
+  int flags = 0;
+  unsigned scored = 0;
+  for (int64_t r0 = (int64_t)blockIdx.x * R; r0 < a.d_out; r0 += (int64_t)gridDim.x * R) {
+    const int64_t row = r0 + rl;
+    const bool active = rl < R && row < a.d_out;
+    float x[kE];
+    float ss = 0.f;
+    if (active) {
+      load64(a.W + row * a.d_in + (int64_t)c * kE, x);
+      const float* fc = f + c * kE;
+#pragma unroll
+      for (int j = 0; j < kE; ++j) {
+        x[j] *= fc[j];
+        ss = fmaf(x[j], x[j], ss);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < kE; ++j) x[j] = 0.f;
+    }
+    part[threadIdx.x] = ss;
+    fwht_reg<kE>(x, nb);
+    fwht_lanes<kE>(x, lanes);
+    __syncthreads();
+    for (int q = warp; q < R; q += nwarps) {
+      float t = 0.f;
+      for (int k = lane; k < C; k += 32) t += part[q * C + k];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      if (lane == 0) rsum[q] = sqrtf(t);
+    }
+    __syncthreads();
+    if (!active) continue;
+
+    const float r = rsum[rl];
+    if (c == 0) {
+      const __half h = __float2half_rn(r);
+      a.rnorm[row] = h;
+      if (!isfinite(r)) flags |= QAMW_STATUS_NONFINITE;
+      else if (isinf(__half2float(h))) flags |= QAMW_STATUS_RANGE;
+    }
+    const bool zero = !(r > 0.f);
+    const float inv = 1.0f / (r * sqrt_b);
+    const float* ic = isg + c * kQ;
+    uint32_t idx[kQ];
+#pragma unroll
+    for (int q = 0; q < kQ; ++q) {
+      const float px = (x[2 * q] * inv) * ic[q];
+      const float py = (x[2 * q + 1] * inv) * ic[q];
+      idx[q] = zero ? 0u : (uint32_t)nearest_pf(px, py, cbq, a.K, pf, scored);
+    }
+    uint32_t w[BITS];
+    pack32<BITS>(idx, w);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(a.packed + row * a.row_bytes) + (size_t)c * BITS;
+#pragma unroll
+    for (int t = 0; t < BITS; ++t) dst[t] = w[t];
+    if (c == C - 1) {  // zero the row's padding words
+      for (int64_t o = (int64_t)C * BITS * 4; o < a.row_bytes; o += 4)
+        *reinterpret_cast<uint32_t*>(a.packed + row * a.row_bytes + o) = 0u;
+    }
+  }
+  raise_flag(a.status, flags);
+  if (a.candidates != nullptr) {
+    unsigned long long v = scored;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) atomicAdd(a.candidates, v);
+  }
+}
+
+// Rows per CTA iteration and the CTA size: R whole rows of C chunk-threads,
+// R * C <= 512, chosen so that few threads idle and the CTA has 128-512 threads.
+void encode_shape(int C, int* R_out, int* threads_out) {
+  int bestR = 1, bestT = ((C + 31) / 32) * 32;
+  double bestScore = -1.0;
+  for (int R = 1; R * C <= 512; ++R) {
+    const int T = ((R * C + 31) / 32) * 32;
+    const double eff = (double)(R * C) / T;
+    const double score = eff - (T < 128 ? 0.5 : 0.0) - (T > 384 ? 0.01 : 0.0);
+    if (score > bestScore + 1e-9) {
+      bestScore = score;
+      bestR = R;
+      bestT = T;
+    }
+  }
+  *R_out = bestR;
+  *threads_out = bestT;
+}
+
+template <int BITS, typename T>
+cudaError_t run_encode(EncodeArgs<T> a, cudaStream_t stream) {
+  const int C = a.d_in / kE;
+  int R, threads;
+  encode_shape(C, &R, &threads);
+  a.rows_per_cta = R;
+  const size_t smem = (size_t)a.K * sizeof(float4) + (size_t)a.d_in * sizeof(float) +
+                      (size_t)(a.d_in / 2) * sizeof(float) + (size_t)threads * sizeof(float) +
+                      (size_t)R * sizeof(float);
+  const void* fn = reinterpret_cast<const void*>(&k_encode<BITS, T>);
+  cudaError_t err = allow_smem(fn, smem);
+  if (err != cudaSuccess) return err;
+  const int grid = persistent_grid(fn, threads, smem, (a.d_out + R - 1) / R);
+  k_encode<BITS, T><<<grid, threads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t encode_rows_typed(const T* W, const qamw_matrix& m, int32_t* st,
+                              unsigned long long* cand, cudaStream_t stream) {
+  EncodeArgs<T> a;
+  a.W = W;
+  a.scale = reinterpret_cast<const __half*>(m.chan_scale);
+  a.sigma = reinterpret_cast<const __half*>(m.sigma);
+  a.codebook = reinterpret_cast<const float2*>(m.codebook);
+  a.prefilter = m.prefilter;
+  a.packed = m.packed;
+  a.rnorm = reinterpret_cast<__half*>(m.row_norm);
+  a.status = st;
+  a.candidates = cand;
+  a.row_bytes = m.row_bytes;
+  a.d_out = m.d_out;
+  a.d_in = m.d_in;
+  a.block = m.block;
+  a.K = 1 << m.bits;
+  a.rows_per_cta = 1;
+  a.seed = m.mask_seed;
+  switch (m.bits) {
+    case 1: return run_encode<1, T>(a, stream);
+    case 2: return run_encode<2, T>(a, stream);
+    case 3: return run_encode<3, T>(a, stream);
+    case 4: return run_encode<4, T>(a, stream);
+    case 5: return run_encode<5, T>(a, stream);
+    case 6: return run_encode<6, T>(a, stream);
+    case 7: return run_encode<7, T>(a, stream);
+    case 8: return run_encode<8, T>(a, stream);
+    case 9: return run_encode<9, T>(a, stream);
+    case 10: return run_encode<10, T>(a, stream);
+    case 11: return run_encode<11, T>(a, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <typename T>
+cudaError_t calibrate_typed(const T* W, const qamw_matrix& m, const EncodeWorkspace& ws,
+                            int32_t* st, cudaStream_t stream) {
+  const int d_out = m.d_out, d_in = m.d_in, P = d_in / 2;
+  const __half* s = reinterpret_cast<const __half*>(m.chan_scale);
+  cudaError_t err;
+  {
+    const int threads = 256;
+    const void* fn = reinterpret_cast<const void*>(&k_rownorm<T>);
+    const int grid = persistent_grid(fn, threads, 0, ((int64_t)d_out * 32 + threads - 1) / threads);
+    k_rownorm<T><<<grid, threads, 0, stream>>>(W, s, d_out, d_in, ws.rnorm32, st);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  k_calib_select<<<1, 1024, 0, stream>>>(ws.rnorm32, d_out, ws.cal_rows, ws.n_cal);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  const int C = d_in / kE;
+  const int threads = ((C + 31) / 32) * 32;
+  const size_t smem = (size_t)d_in * sizeof(float);
+  const void* fn = reinterpret_cast<const void*>(&k_calib_accum<T>);
+  if ((err = allow_smem(fn, smem)) != cudaSuccess) return err;
+  k_calib_accum<T><<<kCalCtas, threads, smem, stream>>>(W, s, ws.rnorm32, ws.cal_rows, ws.n_cal,
+                                                        d_in, m.block, m.mask_seed,
+                                                        ws.cal_partial);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  k_calib_finish<<<(P + 255) / 256, 256, 0, stream>>>(ws.cal_partial, kCalCtas, ws.n_cal, P,
+                                                      reinterpret_cast<__half*>(m.sigma), st);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t calibrate_workspace_bytes(int d_out, int d_in, EncodeWorkspace* carve, void* base) {
+  const size_t P = (size_t)d_in / 2;
+  size_t off = 0;
+  const size_t o_r = off;
+  off += align256((size_t)d_out * sizeof(float));
+  const size_t o_rows = off;
+  off += align256(kCalRows * sizeof(int32_t));
+  const size_t o_n = off;
+  off += align256(sizeof(int32_t));
+  const size_t o_part = off;
+  off += align256((size_t)kCalCtas * P * sizeof(float));
+  if (carve) {
+    char* b = static_cast<char*>(base);
+    carve->rnorm32 = reinterpret_cast<float*>(b + o_r);
+    carve->cal_rows = reinterpret_cast<int32_t*>(b + o_rows);
+    carve->n_cal = reinterpret_cast<int32_t*>(b + o_n);
+    carve->cal_partial = reinterpret_cast<float*>(b + o_part);
+    carve->prefilter = nullptr;
+  }
+  return off;
+}
+
+size_t encode_workspace_bytes(int d_out, int d_in, int bits, EncodeWorkspace* carve, void* base) {
+  const size_t off = calibrate_workspace_bytes(d_out, d_in, carve, base);
+  if (carve) carve->prefilter = static_cast<char*>(base) + off;
+  return off + align256(prefilter_bytes_for(bits));
+}
+
+cudaError_t launch_channel_scales(const float* d_act_stat, int d_in, float alpha, uint16_t* d_scale,
+                                  int32_t* d_status, cudaStream_t stream) {
+  __half* s = reinterpret_cast<__half*>(d_scale);
+  if (d_act_stat != nullptr && alpha != 0.0f)
+    k_scales<<<1, 1024, 0, stream>>>(d_act_stat, d_in, alpha, s, d_status);
+  else
+    k_fill_half<<<(d_in + 255) / 256, 256, 0, stream>>>(s, d_in, 1.0f);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_calibrate(const void* d_W, int dtype, const qamw_matrix& m,
+                             const EncodeWorkspace& ws, int32_t* d_status, cudaStream_t stream) {
+  if (dtype == QAMW_DTYPE_F32)
+    return calibrate_typed<float>(static_cast<const float*>(d_W), m, ws, d_status, stream);
+  return calibrate_typed<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(d_W), m, ws, d_status,
+                                        stream);
+}
+
+cudaError_t launch_encode_rows(const void* d_W, int dtype, const qamw_matrix& m, int32_t* d_status,
+                               unsigned long long* d_candidates, cudaStream_t stream) {
+  if (dtype == QAMW_DTYPE_F32)
+    return encode_rows_typed<float>(static_cast<const float*>(d_W), m, d_status, d_candidates,
+                                    stream);
+  return encode_rows_typed<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(d_W), m, d_status,
+                                          d_candidates, stream);
+}
+
+cudaError_t launch_encode(const void* d_W, int dtype, const float* d_act_stat, float alpha,
+                          int flags, const qamw_matrix& m, const EncodeWorkspace& ws,
+                          int32_t* d_status, cudaStream_t stream) {
+  cudaError_t err;
+  if (!(flags & QAMW_SCALES_GIVEN)) {
+    err = launch_channel_scales(d_act_stat, m.d_in, alpha, m.chan_scale, d_status, stream);
+    if (err != cudaSuccess) return err;
+  }
+  if (!(flags & QAMW_SIGMA_GIVEN)) {
+    err = launch_calibrate(d_W, dtype, m, ws, d_status, stream);
+    if (err != cudaSuccess) return err;
+  }
+  qamw_matrix mm = m;
+  if (mm.prefilter == nullptr) {
+    err = launch_build_prefilter(m.codebook, m.bits, ws.prefilter, stream);
+    if (err != cudaSuccess) return err;
+    mm.prefilter = ws.prefilter;
+  }
+  return launch_encode_rows(d_W, dtype, mm, d_status, nullptr, stream);
+}
+
+}  // namespace qamw

@@ -1,0 +1,60 @@
+// launch.cuh -- host-side launchers of the QAM-W kernels (called by api.cu
+// after argument validation) and launch-shape helpers.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "qamw.h"
+
+namespace qamw {
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+// Grid for a grid-stride kernel: enough CTAs to cover `work_ctas`, at most the
+// number that can be resident at once (occupancy-limited), a multiple of the
+// SM count when the work allows.
+int persistent_grid(const void* kernel, int threads, size_t smem, int64_t work_ctas);
+
+// Opt a kernel into more than 48 KB of dynamic shared memory.
+cudaError_t allow_smem(const void* kernel, size_t smem);
+
+// Workspace carve-up of qamw_encode.
+struct EncodeWorkspace {
+  float* rnorm32;       // [d_out] fp32 row norms of W*s
+  int32_t* cal_rows;    // [1024] rows used by eq. (1)
+  int32_t* n_cal;       // [1]
+  float* cal_partial;   // [kCalCtas][P] partial sums of |z_k|
+  void* prefilter;      // prefilter table (when the matrix carries none)
+};
+constexpr int kCalRows = 1024;
+constexpr int kCalCtas = 128;
+size_t calibrate_workspace_bytes(int d_out, int d_in, EncodeWorkspace* carve, void* base);
+size_t encode_workspace_bytes(int d_out, int d_in, int bits, EncodeWorkspace* carve, void* base);
+
+size_t train_workspace_bytes(int bits);
+size_t gemv_workspace_bytes(int d_in, int batch);
+
+cudaError_t launch_decode(const qamw_matrix& m, uint16_t* d_out_bf16, int32_t* d_status,
+                          cudaStream_t stream);
+cudaError_t launch_channel_scales(const float* d_act_stat, int d_in, float alpha, uint16_t* d_scale,
+                                  int32_t* d_status, cudaStream_t stream);
+cudaError_t launch_calibrate(const void* d_W, int dtype, const qamw_matrix& m,
+                             const EncodeWorkspace& ws, int32_t* d_status, cudaStream_t stream);
+cudaError_t launch_encode_rows(const void* d_W, int dtype, const qamw_matrix& m, int32_t* d_status,
+                               unsigned long long* d_candidates, cudaStream_t stream);
+cudaError_t launch_encode(const void* d_W, int dtype, const float* d_act_stat, float alpha,
+                          int flags, const qamw_matrix& m, const EncodeWorkspace& ws,
+                          int32_t* d_status, cudaStream_t stream);
+cudaError_t launch_build_prefilter(const float* d_codebook, int bits, void* d_table,
+                                   cudaStream_t stream);
+cudaError_t launch_train(const float* d_samples, int64_t n, int bits, int iters,
+                         float* d_codebook, double* d_distortion, void* d_ws,
+                         int32_t* d_status, cudaStream_t stream);
+cudaError_t launch_decode_gemv(const qamw_matrix& m, const uint16_t* d_x, int batch,
+                               uint16_t* d_y, void* d_ws, int32_t* d_status,
+                               cudaStream_t stream);
+
+}  // namespace qamw
