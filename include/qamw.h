@@ -224,6 +224,29 @@ QAMW_API int qamw_decode(const qamw_matrix *m, uint16_t *d_W_out, int32_t *d_sta
 QAMW_API int qamw_decode_gemv(const qamw_matrix *m, const uint16_t *d_x, int batch, uint16_t *d_y,
                      void *d_workspace, size_t ws_bytes, int32_t *d_status, void *stream);
 
+/* Allocation-free variant of qamw_decode_gemv.  The paper has no counterpart:
+ * this entry point exists for callers that cannot allocate device memory,
+ * neither a workspace nor anything else -- plugins whose interface hands over
+ * only input and output pointers, engines that reserve all free device memory
+ * for their own pools up front, and latency-critical loops that must not call
+ * cudaMalloc/cudaFree because those synchronise the device.
+ *   Same arguments and result as qamw_decode_gemv minus the workspace: the
+ *   rotated activation lives in a fixed 1 MiB array in device memory that the
+ *   library reserves on every GPU that loads it, held until the process exits.
+ *   Limit: padded_batch * d_in/2 <= 131072, where padded_batch is batch rounded
+ *   up to 1, 4, 8 or 16 (e.g. batch 16 with d_in <= 16384, or batch 1 with any
+ *   d_in the library accepts); larger problems return QAMW_ERR_SHAPE and
+ *   enqueue nothing.
+ *   The first call on each device looks up that array's device address (with
+ *   the device current) and caches it; make that first call before any stream
+ *   capture.  The call allocates nothing and calls no allocating routine.
+ *   Every call on a device uses the same array, which keeps the previous
+ *   call's contents (each call overwrites everything it reads): calls whose
+ *   work overlaps on the GPU -- e.g. on two streams at once -- race on it, so
+ *   serialise them. */
+QAMW_API int qamw_decode_gemv_noalloc(const qamw_matrix *m, const uint16_t *d_x, int batch,
+                                      uint16_t *d_y, int32_t *d_status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

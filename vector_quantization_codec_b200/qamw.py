@@ -42,7 +42,8 @@ QAMW_OP_CALIBRATE = 3
 EXPORTS = ("qamw_row_bytes", "qamw_default_block", "qamw_bits_per_weight",
            "qamw_workspace_bytes", "qamw_prefilter_bytes", "qamw_status_string",
            "qamw_train_codebook", "qamw_build_prefilter", "qamw_encode", "qamw_channel_scales",
-           "qamw_calibrate_sigma", "qamw_encode_rows", "qamw_decode", "qamw_decode_gemv")
+           "qamw_calibrate_sigma", "qamw_encode_rows", "qamw_decode", "qamw_decode_gemv",
+           "qamw_decode_gemv_noalloc")
 
 
 class QamwError(RuntimeError):
@@ -79,6 +80,7 @@ def _load() -> C.CDLL:
         "qamw_encode_rows": (I, [V, I, C.POINTER(qamw_matrix), V, V, V]),
         "qamw_decode": (I, [C.POINTER(qamw_matrix), V, V, V]),
         "qamw_decode_gemv": (I, [C.POINTER(qamw_matrix), V, I, V, V, SZ, V, V]),
+        "qamw_decode_gemv_noalloc": (I, [C.POINTER(qamw_matrix), V, I, V, V, V]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -287,4 +289,19 @@ def qamw_decode_gemv(m: EncodedMatrix, x: torch.Tensor, y: torch.Tensor | None =
     rc = _lib.qamw_decode_gemv(C.byref(st), _p(x2), batch, _p(y), _p(workspace), workspace.numel(),
                                _p(status), _s(stream))
     _check("qamw_decode_gemv", rc)
+    return y
+
+
+def qamw_decode_gemv_noalloc(m: EncodedMatrix, x: torch.Tensor, y: torch.Tensor,
+                             status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """qamw_decode_gemv without a workspace, for callers that cannot allocate
+    device memory: the rotated activation lives in a fixed array inside the
+    library (limit: padded batch x d_in/2 <= 131072 pairs).  `y` must be given
+    (this wrapper allocates nothing either).  Calls that overlap on the GPU
+    share that array and must be serialised."""
+    x2 = x if x.dim() == 2 else x.view(1, -1)
+    st = m.struct()
+    rc = _lib.qamw_decode_gemv_noalloc(C.byref(st), _p(x2), x2.shape[0], _p(y), _p(status),
+                                       _s(stream))
+    _check("qamw_decode_gemv_noalloc", rc)
     return y
