@@ -479,6 +479,64 @@ def run_reference(args) -> dict | None:
     }
 
 
+def run_single_stage(args) -> dict:
+    """One stage alone on a d_out = args.rows x 4096 matrix (same distributions),
+    for kernel profiling and sweeps: `warmup` untimed then `steps` timed calls."""
+    import torch
+
+    from vector_quantization_codec_b200 import qamw, synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    rows = args.rows
+    K = 1 << BITS
+    samples = torch.from_numpy(synth.circular_gaussian_samples(TRAIN_N, seed=7)).to(dev)
+    codebook = torch.empty((K, 2), dtype=torch.float32, device=dev)
+    iters = TRAIN_ITERS if args.only != "train" else 1
+    if args.only != "train":
+        qamw.qamw_train_codebook(samples, BITS, iters, codebook)
+    prefilter = qamw.qamw_build_prefilter(codebook, BITS) if args.only != "train" else None
+    g = synth.rng(args.seed, 9)
+    W = torch.from_numpy((g.standard_t(5.0, size=(rows, D_IN)) * 0.02).astype("float32"))
+    W = W.to(torch.bfloat16).to(dev)
+    act = torch.from_numpy(synth.act_stat_lognormal(D_IN, args.seed)).to(dev)
+    x = torch.from_numpy(synth.gemv_x(args.batch, D_IN, args.seed)).to(torch.bfloat16).to(dev)
+    m = qamw.EncodedMatrix.empty(rows, D_IN, BLOCK, BITS, codebook, 0, prefilter)
+    if args.only != "train":
+        qamw.qamw_encode(W, m, act, ALPHA)
+    ws_cal = torch.empty(qamw.qamw_workspace_bytes(qamw.QAMW_OP_CALIBRATE, rows, D_IN, BITS),
+                         dtype=torch.uint8, device=dev)
+    ws_g = torch.empty(qamw.qamw_workspace_bytes(qamw.QAMW_OP_GEMV, rows, D_IN, BITS, args.batch),
+                       dtype=torch.uint8, device=dev)
+    W_hat = torch.empty((rows, D_IN), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((args.batch, rows), dtype=torch.bfloat16, device=dev)
+    fns = {
+        "encode": lambda: qamw.qamw_encode_rows(W, m),
+        "calibrate": lambda: qamw.qamw_calibrate_sigma(W, m, workspace=ws_cal),
+        "decode": lambda: qamw.qamw_decode(m, W_hat),
+        "gemv": lambda: qamw.qamw_decode_gemv(m, x, y, workspace=ws_g),
+        "train": lambda: qamw.qamw_train_codebook(samples, BITS, 1, codebook),
+    }
+    fn = fns[args.only]
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    ab = algorithmic_bytes(rows, D_IN, BITS, args.batch)
+    key = {"encode": "encode", "calibrate": "encode", "decode": "decode", "gemv": "gemv"}.get(args.only)
+    out = dict(stage=args.only, rows=rows, d_in=D_IN, batch=args.batch, ms=ms,
+               Mweights_per_s=rows * D_IN / (ms * 1e-3) / 1e6)
+    if key:
+        out["GB_per_s"] = ab[key] / (ms * 1e-3) / 1e9
+    return out
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -487,9 +545,17 @@ def main(argv=None) -> int:
     ap.add_argument("--impl", default="qamw", choices=["qamw", "reference"])
     ap.add_argument("--cpu-rows", type=int, default=64, help="rows of the CPU oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["encode", "calibrate", "decode", "gemv", "train"],
+                    help="profiling mode: time one stage alone (no step, no JSON contract)")
+    ap.add_argument("--rows", type=int, default=16384, help="--only: rows of the d_in=4096 matrix")
+    ap.add_argument("--batch", type=int, default=1, help="--only gemv: batch columns")
+    ap.add_argument("--seed", type=int, default=0)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.only:
+        print(json.dumps(run_single_stage(args)), flush=True)
+        return 0
     out = run_reference(args) if args.impl == "reference" else run_gpu(args)
     if out is not None:
         print(json.dumps(out), flush=True)

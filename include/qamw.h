@@ -68,6 +68,9 @@ extern "C" {
                                   /* underflowing to 0; |sample| >= 2^10        */
 #define QAMW_STATUS_BAD_STAT 0x4  /* activation statistic <= 0 or non-finite;  */
                                   /* the scale of that channel is set to 1      */
+#define QAMW_STATUS_TIMEOUT 0x8   /* a bounded wait for an asynchronous copy    */
+                                  /* gave up; the outputs of that call are not  */
+                                  /* valid                                       */
 
 /* ------------------------------------------------------------------ enums */
 #define QAMW_DTYPE_F32 0  /* W as IEEE binary32                              */
@@ -130,10 +133,11 @@ QAMW_API const char *qamw_status_string(int code);
 
 /* Section 3.6 eq. (2): Lloyd iterations for the joint 2D codebook.
  *   d_samples   [n][2] fp32 draws of the unit circular Gaussian (the caller
- *               draws them; n >= 2^bits).
+ *               draws them; n >= 2^bits), 8-byte aligned.
  *   bits        K = 2^bits codewords, 1..11.
  *   iters       number of Lloyd iterations (>= 0).
- *   d_codebook  [K][2] fp32 output; initialised to the first K samples, then
+ *   d_codebook  [K][2] fp32 output (16-byte aligned); initialised to the first
+ *               K samples, then
  *               each iteration assigns every sample to its nearest codeword
  *               (lowest index on ties) and moves each codeword to the mean of
  *               its cell; an empty cell keeps its codeword.  Cell sums are
@@ -141,7 +145,10 @@ QAMW_API const char *qamw_status_string(int code);
  *               reproducible.
  *   d_distortion [iters] fp64 mean squared distance of each iteration's
  *               assignment (nullable).
- *   d_workspace qamw_workspace_bytes(QAMW_OP_TRAIN, 0, 0, bits, 0) bytes.
+ *   d_workspace qamw_workspace_bytes(QAMW_OP_TRAIN, 0, 0, bits, 0) bytes,
+ *               16-byte aligned (cell sums and the per-iteration prefilter
+ *               table that makes the assignment exact at a few codewords per
+ *               sample).
  * Samples are skipped (and flagged) when non-finite (NONFINITE) or when a
  * coordinate has |x| >= 2^10 (RANGE); n <= 2^25 keeps the fixed-point sums exact. */
 QAMW_API int qamw_train_codebook(const float *d_samples, int64_t n, int bits, int iters,

@@ -69,6 +69,7 @@ CASES = [
     (19, 1024, 256, 10, "bf16", 0.5),
     (12, 256, 32, 2, "f32", 0.5),
     (9, 320, 64, 4, "bf16", 0.5),
+    (16, 20480, 128, 11, "bf16", 0.5),
 ]
 
 
@@ -128,7 +129,7 @@ def test_decode_matches_oracle(case):
 
 GEMV_CASES = [(256, 512, 64, 8, 1), (300, 1024, 128, 11, 4), (97, 4096, 1024, 7, 16),
               (64, 192, 64, 3, 3), (24, 11008, 128, 11, 13), (33, 640, 128, 9, 8),
-              (17, 128, 1, 1, 1)]
+              (17, 128, 1, 1, 1), (16, 20480, 128, 11, 1), (10, 20480, 256, 8, 5)]
 
 
 @pytest.mark.parametrize("case", GEMV_CASES, ids=lambda c: f"{c[0]}x{c[1]}_b{c[2]}_B{c[3]}_n{c[4]}")
@@ -328,3 +329,27 @@ def test_encode_is_deterministic():
     b, _ = gpu_encode(Wt, d_in, block, bits, cb, act, 0.5)
     for x, y in [(a.packed, b.packed), (a.row_norm, b.row_norm), (a.sigma, b.sigma)]:
         assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
+
+
+@pytest.mark.parametrize("bits", [7, 11])
+def test_far_points_use_exact_sector_lists(bits):
+    # sigma given 20x too small pushes normalised pairs to |p| ~ 20-60, far off
+    # the prefilter grid: the angular-sector lists must give the oracle's
+    # indices, and score few codewords (no exhaustive fallback).
+    d_out, d_in, block = 64, 1024, 128
+    cb = codebook(bits)
+    Wt, W = weights(d_out, d_in, 21, "bf16")
+    m, _ = gpu_encode(Wt, d_in, block, bits, cb)
+    sig = (m.sigma.float() / 20).half()
+    m2 = qamw.EncodedMatrix(d_out, d_in, block, bits, 0, torch.empty_like(m.packed),
+                            torch.empty_like(m.row_norm), sig, m.chan_scale, m.codebook, m.prefilter)
+    cand = torch.zeros(1, dtype=torch.int64, device=DEV)
+    qamw.qamw_encode_rows(Wt, m2, candidates=cand)
+    torch.cuda.synchronize()
+    enc = oracle.encode(W, bits, block, cb, s_half=halves(m.chan_scale), sigma_half=halves(sig),
+                        want_points=True)
+    assert np.median(np.linalg.norm(enc["points"], axis=-1)) > 15
+    check_indices(oracle.unpack(m2.packed.cpu().numpy(), d_in // 2, bits), enc["idx"],
+                  enc["points"], cb)
+    pairs = d_out * d_in // 2
+    assert cand.item() < 40 * pairs

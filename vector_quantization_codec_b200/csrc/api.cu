@@ -128,6 +128,7 @@ const char* qamw_status_string(int code) {
     case QAMW_STATUS_NONFINITE: return "non-finite input";
     case QAMW_STATUS_RANGE: return "binary16 range exceeded";
     case QAMW_STATUS_BAD_STAT: return "activation statistic not positive and finite";
+    case QAMW_STATUS_TIMEOUT: return "a bounded wait for an asynchronous copy gave up";
     default: return code > 0 ? "several status flags" : "unknown error";
   }
 }
@@ -137,11 +138,10 @@ int qamw_train_codebook(const float* d_samples, int64_t n, int bits, int iters, 
                         int32_t* d_status, void* stream) {
   if (bits < 1 || bits > 11 || iters < 0 || !d_samples || !d_codebook) return QAMW_ERR_INVALID;
   if (n < ((int64_t)1 << bits)) return QAMW_ERR_SHAPE;
-  if (!aligned16(d_samples) && ((reinterpret_cast<uintptr_t>(d_samples) & 7u) != 0))
-    return QAMW_ERR_ALIGN;
-  if ((reinterpret_cast<uintptr_t>(d_codebook) & 7u) != 0) return QAMW_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(d_samples) & 7u) != 0) return QAMW_ERR_ALIGN;
+  if (!aligned16(d_codebook)) return QAMW_ERR_ALIGN;
   if (!d_workspace || ws_bytes < train_workspace_bytes(bits)) return QAMW_ERR_WORKSPACE;
-  if ((reinterpret_cast<uintptr_t>(d_workspace) & 7u) != 0) return QAMW_ERR_ALIGN;
+  if (!aligned16(d_workspace)) return QAMW_ERR_ALIGN;
   return cuda_rc(launch_train(d_samples, n, bits, iters, d_codebook, d_distortion, d_workspace,
                               d_status, static_cast<cudaStream_t>(stream)));
 }

@@ -41,24 +41,29 @@ __device__ __forceinline__ void raise_flag(int32_t* status, int flag) {
   if (flag && status) atomicOr(status, flag);
 }
 
+// One butterfly stage of span H over N values held in registers.
+template <int N, int H>
+__device__ __forceinline__ void fwht_stage(float (&v)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; i += 2 * H) {
+#pragma unroll
+    for (int j = i; j < i + H; ++j) {
+      const float a = v[j], b = v[j + H];
+      v[j] = a + b;
+      v[j + H] = a - b;
+    }
+  }
+}
+
 // Sylvester Hadamard butterflies of span < nb over the N values a thread holds
 // (N and nb powers of two).  With nb >= N this is v <- H_N v in natural order;
-// with nb < N it is H_nb on each group of nb consecutive values.
-template <int N>
+// with nb < N it is H_nb on each group of nb consecutive values.  The stages
+// are expanded at compile time so that v stays in registers.
+template <int N, int H = 1>
 __device__ __forceinline__ void fwht_reg(float (&v)[N], int nb) {
-#pragma unroll
-  for (int h = 1; h < N; h <<= 1) {
-    if (h < nb) {
-#pragma unroll
-      for (int i = 0; i < N; i += 2 * h) {
-#pragma unroll
-        for (int j = i; j < i + h; ++j) {
-          const float a = v[j], b = v[j + h];
-          v[j] = a + b;
-          v[j + h] = a - b;
-        }
-      }
-    }
+  if constexpr (H < N) {
+    if (H < nb) fwht_stage<N, H>(v);
+    fwht_reg<N, 2 * H>(v, nb);
   }
 }
 
@@ -91,6 +96,17 @@ __device__ __forceinline__ void unpack32(const uint32_t (&w)[BITS], uint32_t (&i
       v = __funnelshift_r(w[wi], w[wi + 1], sh);
     idx[q] = v & mask;
   }
+}
+
+// Index q (compile-time) of the 32 packed in w.
+template <int BITS, int Q>
+__device__ __forceinline__ uint32_t extract_idx(const uint32_t (&w)[BITS]) {
+  constexpr int bit = Q * BITS, wi = bit >> 5, sh = bit & 31;
+  constexpr uint32_t mask = (1u << BITS) - 1u;
+  if constexpr (sh + BITS <= 32)
+    return (w[wi] >> sh) & mask;
+  else
+    return __funnelshift_r(w[wi], w[wi + 1], sh) & mask;
 }
 
 template <int BITS>
@@ -137,6 +153,57 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// ------------------------------------------------------- async bulk copies
+// cp.async.bulk global -> shared with mbarrier completion (TMA, no tensor map,
+// never multicast).  Every wait is bounded: kSpinLimit tries with a short sleep
+// between them (well under a second in total) before the caller gives up.
+constexpr unsigned kSpinLimit = 1u << 20;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// src and dst 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}" : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity) {
+  for (unsigned i = 0; i < kSpinLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    __nanosleep(256);
+  }
+  return false;
+}
+
 // ---------------------------------------------------------------- prefilter
 // Table written by the prefilter kernels and read by the encoder / trainer.
 struct PrefilterHeader {
@@ -147,32 +214,44 @@ struct PrefilterHeader {
   int32_t G;     // cells per side (0: no grid, always exhaustive)
   int32_t cap;   // list capacity per cell
   int32_t K;
-  int32_t pad;
+  int32_t NS;    // angular sectors for points off the grid (|p| >= R)
 };
 
-constexpr int kPfCap = 32;        // candidates per cell
-constexpr uint8_t kPfOverflow = 255;  // count value of a cell searched exhaustively
+// Each cell's list is 32 uint16: entry 0 is the count (kPfOverflow: search
+// exhaustively), entries 1..count the candidate indices in ascending order.
+// One 16-byte load fetches the count and the first 7 candidates.
+constexpr int kPfSlots = 32;
+constexpr int kPfCap = kPfSlots - 1;         // candidates per cell
+constexpr uint32_t kPfOverflow = 0xffffu;
 
 __host__ __device__ inline int prefilter_grid(int bits) {
-  return bits <= 5 ? 0 : (bits <= 7 ? 32 : (bits <= 9 ? 64 : 128));
+  return bits <= 5 ? 0 : (bits <= 7 ? 64 : (bits <= 9 ? 128 : 256));
 }
 
-__host__ __device__ inline size_t prefilter_counts_offset() { return sizeof(PrefilterHeader); }
+__host__ __device__ inline size_t prefilter_lists_offset() {
+  return (sizeof(PrefilterHeader) + 15) / 16 * 16;
+}
 
-__host__ __device__ inline size_t prefilter_lists_offset(int G) {
-  return sizeof(PrefilterHeader) + (((size_t)G * G + 15) / 16) * 16;
+// Points off the grid are looked up by angle in kPfSectors equal sectors of
+// the region |p| >= R (list of every codeword that can win there).
+constexpr int kPfSectors = 256;
+
+__host__ __device__ inline int prefilter_sectors(int bits) {
+  return prefilter_grid(bits) > 0 ? kPfSectors : 0;
 }
 
 __host__ __device__ inline size_t prefilter_bytes_for(int bits) {
   const int G = prefilter_grid(bits);
-  return prefilter_lists_offset(G) + (size_t)G * G * kPfCap * sizeof(uint16_t);
+  return prefilter_lists_offset() +
+         ((size_t)G * G + prefilter_sectors(bits)) * kPfSlots * sizeof(uint16_t);
 }
 
 struct PrefilterView {
   float R, inv_h, Gf;
   int G;  // 0: exhaustive search only
-  const uint8_t* counts;
-  const uint16_t* lists;
+  int NS;
+  const uint4* lists;    // [G*G][4] (32 uint16 per cell)
+  const uint4* sectors;  // [NS][4]
 };
 
 // A table built for another codebook size is ignored (exhaustive search), so a
@@ -182,11 +261,12 @@ __device__ __forceinline__ PrefilterView prefilter_view(const void* table, int K
   PrefilterView v;
   v.R = h->R;
   v.inv_h = h->inv_h;
-  v.G = (h->K == K && h->cap == kPfCap) ? h->G : 0;
+  v.G = (h->K == K && h->cap == kPfCap && h->NS == kPfSectors) ? h->G : 0;
+  v.NS = h->NS;
   v.Gf = (float)v.G;
-  v.counts = reinterpret_cast<const uint8_t*>(table) + prefilter_counts_offset();
-  v.lists = reinterpret_cast<const uint16_t*>(reinterpret_cast<const uint8_t*>(table) +
-                                              prefilter_lists_offset(h->G));
+  v.lists = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(table) +
+                                           prefilter_lists_offset());
+  v.sectors = v.lists + (size_t)v.G * v.G * (kPfSlots / 8);
   return v;
 }
 
@@ -214,36 +294,89 @@ __device__ __forceinline__ int nearest_all(float m2x, float m2y, const float4* c
   return bi;
 }
 
-// Same result as nearest_all: the cell's list holds every codeword that can win
-// for a point of the cell, in ascending index order.
-__device__ __forceinline__ int nearest_pf(float px, float py, const float4* cbq, int K,
-                                          const PrefilterView& pf, unsigned& scored) {
-  const float m2x = -2.f * px, m2y = -2.f * py;
-  if (pf.G > 0) {
+__device__ __forceinline__ void score(float m2x, float m2y, const float4* cbq, uint32_t j,
+                                      float& be, int& bi) {
+  const float4 c = cbq[j];
+  const float e = fmaf(m2x, c.x, fmaf(m2y, c.y, c.z));
+  if (e < be) {
+    be = e;
+    bi = (int)j;
+  }
+}
+
+// Split form of nearest_pf, so that a caller can fetch the next point's list
+// head while it scores the current point.
+struct PfCursor {
+  const uint4* L;  // nullptr: exhaustive search
+  uint4 head;
+};
+
+__device__ __forceinline__ PfCursor pf_locate(float px, float py, const PrefilterView& pf) {
+  PfCursor cur;
+  cur.L = nullptr;
+  cur.head = make_uint4(0u, 0u, 0u, 0u);
+  if (pf.G > 0 && isfinite(px) && isfinite(py)) {
     const float gx = (px + pf.R) * pf.inv_h;
     const float gy = (py + pf.R) * pf.inv_h;
     if (gx >= 0.f && gx < pf.Gf && gy >= 0.f && gy < pf.Gf) {
-      const int cell = (int)gy * pf.G + (int)gx;
-      const int cnt = __ldg(pf.counts + cell);
-      if (cnt != kPfOverflow) {
-        scored += (unsigned)cnt;
-        const uint16_t* L = pf.lists + (size_t)cell * kPfCap;
-        float be = INFINITY;
-        int bi = 0;
-        for (int t = 0; t < cnt; ++t) {
-          const int j = __ldg(L + t);
-          const float4 c = cbq[j];
-          const float e = fmaf(m2x, c.x, fmaf(m2y, c.y, c.z));
-          if (e < be) {
-            be = e;
-            bi = j;
-          }
-        }
-        return bi;
-      }
+      cur.L = pf.lists + ((size_t)((int)gy * pf.G + (int)gx)) * (kPfSlots / 8);
+    } else {
+      const float t = (atan2f(py, px) + 3.14159265f) * ((float)pf.NS * 0.159154943f);
+      const int sct = min(max((int)t, 0), pf.NS - 1);
+      cur.L = pf.sectors + (size_t)sct * (kPfSlots / 8);
+    }
+    cur.head = __ldg(cur.L);
+  }
+  return cur;
+}
+
+// Rare paths of pf_finish: lists longer than 7 (slots 8..count), overflowed
+// lists and points that are not finite (exhaustive search).  Kept out of line
+// so that the common path stays small.
+static __device__ __noinline__ int pf_finish_slow(const uint4* L, uint32_t cnt, float m2x, float m2y,
+                                           const float4* cbq, int K, float be, int bi,
+                                           unsigned* scored) {
+  if (L == nullptr || cnt == kPfOverflow) return nearest_all(m2x, m2y, cbq, K, *scored);
+  for (uint32_t g = 1; g * 8 <= cnt; ++g) {
+    const uint4 q = __ldg(L + g);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if (g * 8 + e > cnt) break;
+      const uint32_t w = e < 2 ? q.x : (e < 4 ? q.y : (e < 6 ? q.z : q.w));
+      score(m2x, m2y, cbq, (e & 1) ? (w >> 16) : (w & 0xffffu), be, bi);
     }
   }
-  return nearest_all(m2x, m2y, cbq, K, scored);
+  return bi;
+}
+
+// Slots 1..7 of every list are filled (unused ones repeat the first
+// candidate, which cannot change a strict-'<' argmin taken in ascending slot
+// order), so the common case scores 7 codewords without branching.
+__device__ __forceinline__ int pf_finish(const PfCursor& cur, float px, float py,
+                                         const float4* cbq, int K, unsigned& scored) {
+  const float m2x = -2.f * px, m2y = -2.f * py;
+  const uint4 q = cur.head;
+  const uint32_t cnt = q.x & 0xffffu;
+  float be = INFINITY;
+  int bi = 0;
+  if (cur.L != nullptr && cnt != kPfOverflow) {
+    scored += cnt;
+    score(m2x, m2y, cbq, q.x >> 16, be, bi);
+    score(m2x, m2y, cbq, q.y & 0xffffu, be, bi);
+    score(m2x, m2y, cbq, q.y >> 16, be, bi);
+    score(m2x, m2y, cbq, q.z & 0xffffu, be, bi);
+    score(m2x, m2y, cbq, q.z >> 16, be, bi);
+    score(m2x, m2y, cbq, q.w & 0xffffu, be, bi);
+    score(m2x, m2y, cbq, q.w >> 16, be, bi);
+    if (cnt < 8) return bi;
+  }
+  return pf_finish_slow(cur.L, cnt, m2x, m2y, cbq, K, be, bi, &scored);
+}
+
+// Nearest codeword through the prefilter (same result as nearest_all).
+__device__ __forceinline__ int nearest_pf(float px, float py, const float4* cbq, int K,
+                                          const PrefilterView& pf, unsigned& scored) {
+  return pf_finish(pf_locate(px, py, pf), px, py, cbq, K, scored);
 }
 
 }  // namespace qamw

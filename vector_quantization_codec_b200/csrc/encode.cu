@@ -163,23 +163,30 @@ __global__ void __launch_bounds__(1024) k_calib_select(const float* __restrict__
   if (t == T - 1) *n_cal = min(scan[T - 1], kCalRows);
 }
 
-template <typename T>
-__global__ void __launch_bounds__(1024) k_calib_accum(const T* __restrict__ W,
+// CTA b owns calibration ranks [8b, 8b + 8) and processes RPC of those rows at
+// once (thread (g, c): chunk c of row g of the batch), accumulating |z_k| in
+// registers; the RPC row groups are then summed in a fixed order through a
+// transposed shared buffer into partial[b][k].
+template <typename T, int MAXT>
+__global__ void __launch_bounds__(MAXT) k_calib_accum(const T* __restrict__ W,
                                                       const __half* __restrict__ s,
                                                       const float* __restrict__ r32,
                                                       const int32_t* __restrict__ cal_rows,
                                                       const int32_t* __restrict__ n_cal_p,
-                                                      int d_in, int block, uint64_t seed,
+                                                      int d_in, int block, uint64_t seed, int RPC,
                                                       float* __restrict__ partial) {
-  extern __shared__ __align__(16) float f[];  // D_j * s_j
+  extern __shared__ __align__(16) float sm[];
+  const int C = d_in / kE, P = d_in / 2;
+  float* fT = sm;            // [j][c]: D * s of column 64c + j
+  float* red = sm + d_in;    // [g][q][c]
+#pragma unroll 4
   for (int j = threadIdx.x; j < d_in; j += blockDim.x) {
     const float v = __half2float(s[j]);
-    f[j] = mask_negative(seed, (uint32_t)j) ? -v : v;
+    fT[(j % kE) * C + j / kE] = mask_negative(seed, (uint32_t)j) ? -v : v;
   }
   __syncthreads();
-  const int C = d_in / kE, P = d_in / 2;
-  const int c = threadIdx.x;
-  const bool active = c < C;
+  const int g = threadIdx.x / C, c = threadIdx.x - g * C;
+  const bool lane_ok = g < RPC;
   const int nb = min(block, kE), lanes = max(block / kE, 1);
   const float inv_sqrt_b = 1.0f / sqrtf((float)block);
   const int n_cal = *n_cal_p;
@@ -188,30 +195,39 @@ __global__ void __launch_bounds__(1024) k_calib_accum(const T* __restrict__ W,
   float acc[kQ];
 #pragma unroll
   for (int q = 0; q < kQ; ++q) acc[q] = 0.f;
-  for (int t = t0; t < t1; ++t) {
-    const int row = cal_rows[t];
+  for (int base = t0; base < t1; base += RPC) {
+    const int t = base + g;
+    const bool active = lane_ok && t < t1;
+    const int row = active ? cal_rows[t] : 0;
     float x[kE];
     if (active) {
       load64(W + (int64_t)row * d_in + (int64_t)c * kE, x);
 #pragma unroll
-      for (int j = 0; j < kE; ++j) x[j] *= f[c * kE + j];
+      for (int j = 0; j < kE; ++j) x[j] *= fT[j * C + c];
     } else {
 #pragma unroll
       for (int j = 0; j < kE; ++j) x[j] = 0.f;
     }
     fwht_reg<kE>(x, nb);
     fwht_lanes<kE>(x, lanes);
-    const float inv = inv_sqrt_b / r32[row];
+    if (active) {
+      const float inv = inv_sqrt_b / r32[row];
 #pragma unroll
-    for (int q = 0; q < kQ; ++q) {
-      const float zx = x[2 * q] * inv, zy = x[2 * q + 1] * inv;
-      acc[q] += sqrtf(fmaf(zx, zx, zy * zy));
+      for (int q = 0; q < kQ; ++q) {
+        const float zx = x[2 * q] * inv, zy = x[2 * q + 1] * inv;
+        acc[q] += sqrtf(fmaf(zx, zx, zy * zy));
+      }
     }
   }
-  if (active) {
-    float* dst = partial + (size_t)blockIdx.x * P + c * kQ;
+  if (lane_ok) {
 #pragma unroll
-    for (int q = 0; q < kQ; ++q) dst[q] = acc[q];
+    for (int q = 0; q < kQ; ++q) red[(size_t)g * P + q * C + c] = acc[q];
+  }
+  __syncthreads();
+  for (int k = threadIdx.x; k < P; k += blockDim.x) {
+    float v = 0.f;
+    for (int gg = 0; gg < RPC; ++gg) v += red[(size_t)gg * P + (k % kQ) * C + k / kQ];
+    partial[(size_t)blockIdx.x * P + k] = v;
   }
 }
 
@@ -255,20 +271,27 @@ struct EncodeArgs {
 // (reduced per row in a fixed order, so r is bitwise reproducible), Hadamard
 // butterflies, division by r sqrt(b) and sigma_k, nearest codeword, packing.
 template <int BITS, typename T>
-__global__ void __launch_bounds__(512) k_encode(const EncodeArgs<T> a) {
+__global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
   extern __shared__ __align__(16) unsigned char smem[];
   float4* cbq = reinterpret_cast<float4*>(smem);
-  float* f = reinterpret_cast<float*>(cbq + a.K);  // D_j * s_j
-  const int P = a.d_in >> 1;
-  float* isg = f + a.d_in;                          // 1 / sigma_k
-  float* part = isg + P;                            // [blockDim] partial sums of squares
+  // per-column tables transposed, [position in chunk][chunk], so that the lanes
+  // of a warp (consecutive chunks) read consecutive words
+  const int P = a.d_in >> 1, C = a.d_in / kE;
+  float* fT = reinterpret_cast<float*>(cbq + a.K);  // [j][c]: D * s of column 64c + j
+  float* isgT = fT + a.d_in;                        // [q][c]: 1 / sigma of pair 32c + q
+  float* part = isgT + P;                           // [blockDim] partial sums of squares
   float* rsum = part + blockDim.x;                  // [R] row norms
+  // table fills: unrolled so that each thread's loads are in flight together
+#pragma unroll 4
   for (int i = threadIdx.x; i < a.K; i += blockDim.x) cbq[i] = codeword_q(a.codebook[i]);
+#pragma unroll 4
   for (int j = threadIdx.x; j < a.d_in; j += blockDim.x) {
     const float v = __half2float(a.scale[j]);
-    f[j] = mask_negative(a.seed, (uint32_t)j) ? -v : v;
+    fT[(j % kE) * C + j / kE] = mask_negative(a.seed, (uint32_t)j) ? -v : v;
   }
-  for (int k = threadIdx.x; k < P; k += blockDim.x) isg[k] = 1.0f / __half2float(a.sigma[k]);
+#pragma unroll 4
+  for (int k = threadIdx.x; k < P; k += blockDim.x)
+    isgT[(k % kQ) * C + k / kQ] = 1.0f / __half2float(a.sigma[k]);
   PrefilterView pf;
   if (a.prefilter != nullptr) {
     pf = prefilter_view(a.prefilter, a.K);
@@ -278,7 +301,7 @@ __global__ void __launch_bounds__(512) k_encode(const EncodeArgs<T> a) {
   }
   __syncthreads();
 
-  const int C = a.d_in / kE, R = a.rows_per_cta;
+  const int R = a.rows_per_cta;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int rl = threadIdx.x / C, c = threadIdx.x - rl * C;
   const int nb = min(a.block, kE), lanes = max(a.block / kE, 1);
@@ -292,10 +315,9 @@ __global__ void __launch_bounds__(512) k_encode(const EncodeArgs<T> a) {
     float ss = 0.f;
     if (active) {
       load64(a.W + row * a.d_in + (int64_t)c * kE, x);
-      const float* fc = f + c * kE;
 #pragma unroll
       for (int j = 0; j < kE; ++j) {
-        x[j] *= fc[j];
+        x[j] *= fT[j * C + c];
         ss = fmaf(x[j], x[j], ss);
       }
     } else {
@@ -325,16 +347,32 @@ __global__ void __launch_bounds__(512) k_encode(const EncodeArgs<T> a) {
     }
     const bool zero = !(r > 0.f);
     const float inv = 1.0f / (r * sqrt_b);
-    const float* ic = isg + c * kQ;
-    uint32_t idx[kQ];
+    // nearest codeword of each pair, packing as we go; the list head of pair
+    // q+1 is fetched while pair q is scored
+    uint32_t w[BITS];
+#pragma unroll
+    for (int t = 0; t < BITS; ++t) w[t] = 0u;
+    float is = isgT[c];
+    float px = (x[0] * inv) * is, py = (x[1] * inv) * is;
+    PfCursor cur = pf_locate(px, py, pf);
 #pragma unroll
     for (int q = 0; q < kQ; ++q) {
-      const float px = (x[2 * q] * inv) * ic[q];
-      const float py = (x[2 * q + 1] * inv) * ic[q];
-      idx[q] = zero ? 0u : (uint32_t)nearest_pf(px, py, cbq, a.K, pf, scored);
+      float nx = 0.f, ny = 0.f;
+      PfCursor nxt = cur;
+      if (q + 1 < kQ) {
+        const float is1 = isgT[(q + 1) * C + c];
+        nx = (x[2 * q + 2] * inv) * is1;
+        ny = (x[2 * q + 3] * inv) * is1;
+        nxt = pf_locate(nx, ny, pf);
+      }
+      const uint32_t id = zero ? 0u : (uint32_t)pf_finish(cur, px, py, cbq, a.K, scored);
+      const int bit = q * BITS, wi = bit >> 5, sh = bit & 31;
+      w[wi] |= id << sh;
+      if (sh + BITS > 32) w[wi + 1] |= id >> (32 - sh);
+      cur = nxt;
+      px = nx;
+      py = ny;
     }
-    uint32_t w[BITS];
-    pack32<BITS>(idx, w);
     uint32_t* dst = reinterpret_cast<uint32_t*>(a.packed + row * a.row_bytes) + (size_t)c * BITS;
 #pragma unroll
     for (int t = 0; t < BITS; ++t) dst[t] = w[t];
@@ -360,7 +398,8 @@ void encode_shape(int C, int* R_out, int* threads_out) {
   for (int R = 1; R * C <= 512; ++R) {
     const int T = ((R * C + 31) / 32) * 32;
     const double eff = (double)(R * C) / T;
-    const double score = eff - (T < 128 ? 0.5 : 0.0) - (T > 384 ? 0.01 : 0.0);
+    // prefer 256-thread CTAs: two per SM at <= 128 registers
+    const double score = eff - (T < 256 ? 0.05 * (256 - T) / 128.0 : 0.0) - (T > 256 ? 0.02 : 0.0);
     if (score > bestScore + 1e-9) {
       bestScore = score;
       bestR = R;
@@ -440,13 +479,25 @@ cudaError_t calibrate_typed(const T* W, const qamw_matrix& m, const EncodeWorksp
   k_calib_select<<<1, 1024, 0, stream>>>(ws.rnorm32, d_out, ws.cal_rows, ws.n_cal);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   const int C = d_in / kE;
-  const int threads = ((C + 31) / 32) * 32;
-  const size_t smem = (size_t)d_in * sizeof(float);
-  const void* fn = reinterpret_cast<const void*>(&k_calib_accum<T>);
+  // rows per batch: at most the 8 rows a CTA owns, 256 threads, ~200 KB of shared memory
+  // rows per batch: at most the 8 rows a CTA owns, 256 threads (512 when one
+  // row has more than 256 chunks), ~200 KB of shared memory
+  const int maxt = C > 256 ? 512 : 256;
+  int RPC = 8;
+  if (RPC * C > maxt) RPC = maxt / C;
+  while (RPC > 1 && (size_t)d_in * 4 * (1 + RPC / 2) > 200 * 1024) --RPC;
+  if (RPC < 1) RPC = 1;
+  const int threads = ((RPC * C + 31) / 32) * 32;
+  const size_t smem = (size_t)d_in * sizeof(float) + (size_t)RPC * P * sizeof(float);
+  const void* fn = maxt == 256 ? reinterpret_cast<const void*>(&k_calib_accum<T, 256>)
+                               : reinterpret_cast<const void*>(&k_calib_accum<T, 512>);
   if ((err = allow_smem(fn, smem)) != cudaSuccess) return err;
-  k_calib_accum<T><<<kCalCtas, threads, smem, stream>>>(W, s, ws.rnorm32, ws.cal_rows, ws.n_cal,
-                                                        d_in, m.block, m.mask_seed,
-                                                        ws.cal_partial);
+  if (maxt == 256)
+    k_calib_accum<T, 256><<<kCalCtas, threads, smem, stream>>>(
+        W, s, ws.rnorm32, ws.cal_rows, ws.n_cal, d_in, m.block, m.mask_seed, RPC, ws.cal_partial);
+  else
+    k_calib_accum<T, 512><<<kCalCtas, threads, smem, stream>>>(
+        W, s, ws.rnorm32, ws.cal_rows, ws.n_cal, d_in, m.block, m.mask_seed, RPC, ws.cal_partial);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   k_calib_finish<<<(P + 255) / 256, 256, 0, stream>>>(ws.cal_partial, kCalCtas, ws.n_cal, P,
                                                       reinterpret_cast<__half*>(m.sigma), st);

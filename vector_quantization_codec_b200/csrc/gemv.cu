@@ -3,21 +3,262 @@
 // W_hat row i = r_i * diag(1/s) R_inv yhat_i with yhat_i pair k = sigma_k c[idx_ik]
 // (paper section 3.2).  R_inv = R_fwd^T, so
 //   y[t][i] = r_i * sum_k < xbar_t[k], c[idx_ik] >,  xbar_t = sigma (.) R_fwd(x_t / s)
-// (pair k = coordinates 2k, 2k+1).  k_rotate computes xbar once per call into
-// the workspace; k_gemv streams the packed indices and gathers codewords.
+// (pair k = coordinates 2k, 2k+1): the activation is rotated once and the
+// weights are never decoded to BF16.
+//
+// batch 1 (k_gemv1): one persistent CTA per SM.  Each warp owns a fixed slice of
+//   32 chunks (1024 pairs) and computes xbar for it straight into registers.
+//   Tiles of R whole rows of packed indices stream into a 3-stage shared ring
+//   through cp.async.bulk (TMA, mbarrier completion, bounded waits); codewords
+//   come from an fp16x2 copy of the codebook replicated so that a warp's 32
+//   random lookups hit at most 2 lanes per bank.  Per-slice partial dot
+//   products are summed in a fixed order (bitwise reproducible).
+// batch 2..16 (k_rotate + k_gemv): xbar for all columns is written once to the
+//   workspace (chunk-interleaved so that lanes read consecutive words), then
+//   one warp per row accumulates all batch columns.
+#include <utility>
+
 #include "common.cuh"
 #include "launch.cuh"
 
 namespace qamw {
 namespace {
 
-// xbar[t][k] (float2) for t < batch, zeros for batch <= t < bpad; one thread
-// per (t, chunk of 64 columns).
+// ------------------------------------------------------------------ batch 1
+
+constexpr int kGemvStages = 3;
+
+struct Gemv1Args {
+  const uint8_t* packed;
+  const __half* rnorm;
+  const __half* sigma;
+  const __half* scale;
+  const __nv_bfloat16* x;
+  const float2* codebook;
+  __nv_bfloat16* y;
+  int32_t* status;
+  int64_t row_bytes;
+  int d_out, d_in, block, K;
+  uint64_t seed;
+  int S;            // slices of 32 chunks per row
+  int k;            // warps per slice
+  int R;            // rows per tile (multiple of k)
+  int ntiles;
+  int copies_log2;  // codebook replicas (power of two)
+  unsigned stage_bytes;
+};
+
+__host__ __device__ inline size_t align16(size_t v) { return (v + 15) & ~(size_t)15; }
+
+// acc += <xr pair q, fp16x2 codeword of index q> for the 32 indices packed in w
+// (every index a compile-time constant, so xr stays in registers).
+template <int BITS, int... Q>
+__device__ __forceinline__ void dot_pairs(const uint32_t (&w)[BITS], const uint32_t* tab, int cl,
+                                          uint32_t copy, const float (&xr)[kE], float& acc0,
+                                          float& acc1, std::integer_sequence<int, Q...>) {
+  (
+      [&] {
+        const uint32_t h = tab[(extract_idx<BITS, Q>(w) << cl) | copy];
+        const float2 cw = __half22float2(*reinterpret_cast<const __half2*>(&h));
+        acc0 = fmaf(xr[2 * Q], cw.x, acc0);
+        acc1 = fmaf(xr[2 * Q + 1], cw.y, acc1);
+      }(),
+      ...);
+}
+
+template <int BITS, int MAXT>
+__global__ void __launch_bounds__(MAXT, 1) k_gemv1(const Gemv1Args a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int copies = 1 << a.copies_log2;
+  uint32_t* tab = reinterpret_cast<uint32_t*>(smem);  // [K][copies] fp16x2
+  unsigned char* stage = smem + (size_t)a.K * copies * 4;
+  float* partial = reinterpret_cast<float*>(stage + (size_t)kGemvStages * a.stage_bytes);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(partial) +
+                                              align16((size_t)a.R * a.S * 4));
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int C = a.d_in / kE;
+
+  if (tid == 0) {
+    for (int s = 0; s < kGemvStages; ++s) mbar_init(&bar[s], 1);
+    fence_mbar_init();
+  }
+  // fp16x2 codebook, `copies` replicas of each entry side by side; each thread
+  // loads its codewords together, then writes their replicas
+#pragma unroll 4
+  for (int j = tid; j < a.K; j += blockDim.x) {
+    const float2 c = a.codebook[j];
+    const __half2 h = __floats2half2_rn(c.x, c.y);
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(&h);
+    for (int r = 0; r < copies; ++r) tab[(j << a.copies_log2) + r] = u;
+  }
+  __syncthreads();
+  // first tiles in flight while xbar is computed
+  if (tid == 0) {
+    for (int s = 0; s < kGemvStages; ++s) {
+      const int tile = blockIdx.x + s * gridDim.x;
+      if (tile >= a.ntiles) break;
+      const int r0 = tile * a.R, nr = min(a.R, a.d_out - r0);
+      const unsigned bytes = (unsigned)(nr * a.row_bytes);
+      mbar_expect_tx(&bar[s], bytes);
+      bulk_g2s(stage + (size_t)s * a.stage_bytes, a.packed + (int64_t)r0 * a.row_bytes, bytes,
+               &bar[s]);
+    }
+  }
+
+  // xbar of this lane's chunk c: sigma (.) R_fwd(x / s), in registers
+  const int sl = warp % a.S, kk = warp / a.S;
+  const int c = sl * 32 + lane;
+  const bool active = c < C;
+  float xr[kE];
+  int flags = 0;
+  if (active) {
+    load64(a.x + (int64_t)c * kE, xr);
+#pragma unroll
+    for (int j = 0; j < kE; ++j) {
+      const int col = c * kE + j;
+      if (!isfinite(xr[j])) flags = QAMW_STATUS_NONFINITE;
+      const float q = __fdiv_rn(xr[j], __half2float(a.scale[col]));
+      xr[j] = mask_negative(a.seed, (uint32_t)col) ? -q : q;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < kE; ++j) xr[j] = 0.f;
+  }
+  fwht_reg<kE>(xr, min(a.block, kE));
+  fwht_lanes<kE>(xr, max(a.block / kE, 1));
+  if (active) {
+    const float inv_sqrt_b = 1.0f / sqrtf((float)a.block);
+#pragma unroll
+    for (int q = 0; q < kQ; ++q) {
+      const float sg = __half2float(a.sigma[c * kQ + q]) * inv_sqrt_b;
+      xr[2 * q] *= sg;
+      xr[2 * q + 1] *= sg;
+    }
+  }
+
+  const uint32_t cmask = (uint32_t)(copies - 1);
+  int it = 0;
+  bool timed_out = false;
+  for (int tile = blockIdx.x; tile < a.ntiles; tile += gridDim.x, ++it) {
+    const int st = it % kGemvStages;
+    const unsigned parity = (unsigned)(it / kGemvStages) & 1u;
+    const bool ok = mbar_wait_bounded(&bar[st], parity);
+    if (__syncthreads_or(!ok)) {
+      timed_out = true;
+      break;
+    }
+    const int r0 = tile * a.R, nr = min(a.R, a.d_out - r0);
+    const unsigned char* buf = stage + (size_t)st * a.stage_bytes;
+    for (int rl = kk; rl < nr; rl += a.k) {
+      float acc0 = 0.f, acc1 = 0.f;
+      if (active) {
+        const uint32_t* src =
+            reinterpret_cast<const uint32_t*>(buf + (size_t)rl * a.row_bytes) + (size_t)c * BITS;
+        uint32_t w[BITS];
+#pragma unroll
+        for (int t = 0; t < BITS; ++t) w[t] = src[t];
+        dot_pairs<BITS>(w, tab, a.copies_log2, (uint32_t)lane & cmask, xr, acc0, acc1,
+                        std::make_integer_sequence<int, kQ>{});
+      }
+      float acc = acc0 + acc1;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) partial[rl * a.S + sl] = acc;
+    }
+    __syncthreads();
+    for (int r = tid; r < nr; r += blockDim.x) {
+      float sum = 0.f;
+      for (int s = 0; s < a.S; ++s) sum += partial[r * a.S + s];
+      a.y[r0 + r] = __float2bfloat16_rn(sum * __half2float(a.rnorm[r0 + r]));
+    }
+    if (tid == 0) {
+      const int next = tile + kGemvStages * gridDim.x;
+      if (next < a.ntiles) {
+        const int n0 = next * a.R, nn = min(a.R, a.d_out - n0);
+        const unsigned bytes = (unsigned)(nn * a.row_bytes);
+        mbar_expect_tx(&bar[st], bytes);
+        bulk_g2s(stage + (size_t)st * a.stage_bytes, a.packed + (int64_t)n0 * a.row_bytes, bytes,
+                 &bar[st]);
+      }
+    }
+    __syncthreads();
+  }
+  if (timed_out) {
+    // let this CTA's copies still in flight land before its shared memory goes away
+    if (tid == 0) {
+      for (int s = 0; s < kGemvStages; ++s) {
+        const int t2 = it + s;
+        const int tile = blockIdx.x + t2 * gridDim.x;
+        if (tile >= a.ntiles) break;
+        mbar_wait_bounded(&bar[t2 % kGemvStages], (unsigned)(t2 / kGemvStages) & 1u);
+      }
+    }
+    flags |= QAMW_STATUS_TIMEOUT;
+  }
+  raise_flag(a.status, flags);
+}
+
+// Shared memory of k_gemv1 for given replicas and tile rows.
+size_t gemv1_smem(int K, int copies_log2, unsigned stage_bytes, int R, int S) {
+  return (size_t)K * ((size_t)1 << copies_log2) * 4 + (size_t)kGemvStages * stage_bytes +
+         align16((size_t)R * S * 4) + kGemvStages * sizeof(uint64_t);
+}
+
+template <int BITS>
+cudaError_t run_gemv1(const qamw_matrix& m, const uint16_t* d_x, uint16_t* d_y,
+                      int32_t* d_status, cudaStream_t stream) {
+  Gemv1Args a;
+  a.packed = m.packed;
+  a.rnorm = reinterpret_cast<const __half*>(m.row_norm);
+  a.sigma = reinterpret_cast<const __half*>(m.sigma);
+  a.scale = reinterpret_cast<const __half*>(m.chan_scale);
+  a.x = reinterpret_cast<const __nv_bfloat16*>(d_x);
+  a.codebook = reinterpret_cast<const float2*>(m.codebook);
+  a.y = reinterpret_cast<__nv_bfloat16*>(d_y);
+  a.status = d_status;
+  a.row_bytes = m.row_bytes;
+  a.d_out = m.d_out;
+  a.d_in = m.d_in;
+  a.block = m.block;
+  a.K = 1 << m.bits;
+  a.seed = m.mask_seed;
+  const int C = m.d_in / kE;
+  a.S = (C + 31) / 32;
+  a.k = a.S <= 8 ? 8 / a.S : 1;
+  // ~24 KB of indices per stage, whole rows, a multiple of k rows
+  int R = (int)(24576 / m.row_bytes);
+  R = R < a.k ? a.k : (R / a.k) * a.k;
+  a.R = R;
+  a.stage_bytes = (unsigned)(R * m.row_bytes);
+  a.ntiles = (m.d_out + R - 1) / R;
+  int cl = a.K <= 1024 ? 5 : 4;
+  while (cl > 0 && gemv1_smem(a.K, cl, a.stage_bytes, R, a.S) > 227 * 1024) --cl;
+  a.copies_log2 = cl;
+  const size_t smem = gemv1_smem(a.K, cl, a.stage_bytes, R, a.S);
+  if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
+  const int threads = 32 * a.S * a.k;
+  // 256-thread bound (up to 255 registers) unless a row needs more than 8 slices
+  const void* fn = threads <= 256 ? reinterpret_cast<const void*>(&k_gemv1<BITS, 256>)
+                                  : reinterpret_cast<const void*>(&k_gemv1<BITS, 512>);
+  cudaError_t err = allow_smem(fn, smem);
+  if (err != cudaSuccess) return err;
+  const int grid = a.ntiles < sm_count() ? a.ntiles : sm_count();
+  if (threads <= 256)
+    k_gemv1<BITS, 256><<<grid, threads, smem, stream>>>(a);
+  else
+    k_gemv1<BITS, 512><<<grid, threads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------- batch 2..16
+
+// xbarT[t][q][c] (float2) = pair 32c+q of xbar_t, for t < batch; zeros for
+// batch <= t < bpad; one thread per (t, chunk c).
 __global__ void __launch_bounds__(256) k_rotate(const __nv_bfloat16* __restrict__ x, int batch,
                                                 int bpad, int d_in, int block, uint64_t seed,
                                                 const __half* __restrict__ s,
                                                 const __half* __restrict__ sigma,
-                                                float2* __restrict__ xbar, int32_t* status) {
+                                                float2* __restrict__ xbarT, int32_t* status) {
   const int C = d_in / kE, P = d_in / 2;
   const int64_t V = (int64_t)bpad * C;
   const int nb = min(block, kE), lanes = max(block / kE, 1);
@@ -47,11 +288,11 @@ __global__ void __launch_bounds__(256) k_rotate(const __nv_bfloat16* __restrict_
     fwht_reg<kE>(xv, nb);
     fwht_lanes<kE>(xv, lanes);
     if (active) {
-      float2* dst = xbar + t * P + (int64_t)c * kQ;
+      float2* dst = xbarT + t * P + c;
 #pragma unroll
       for (int q = 0; q < kQ; ++q) {
         const float sg = __half2float(sigma[c * kQ + q]) * inv_sqrt_b;
-        dst[q] = make_float2(xv[2 * q] * sg, xv[2 * q + 1] * sg);
+        dst[(size_t)q * C] = make_float2(xv[2 * q] * sg, xv[2 * q + 1] * sg);
       }
     }
   }
@@ -63,7 +304,7 @@ template <int BITS, int B>
 __global__ void __launch_bounds__(256) k_gemv(const uint8_t* __restrict__ packed, int64_t row_bytes,
                                               const __half* __restrict__ rnorm,
                                               const float2* __restrict__ codebook, int K,
-                                              const float2* __restrict__ xbar, int d_out, int d_in,
+                                              const float2* __restrict__ xbarT, int d_out, int d_in,
                                               int batch, __nv_bfloat16* __restrict__ y) {
   extern __shared__ __align__(16) unsigned char smem[];
   float2* cb = reinterpret_cast<float2*>(smem);
@@ -84,12 +325,12 @@ __global__ void __launch_bounds__(256) k_gemv(const uint8_t* __restrict__ packed
       uint32_t idx[kQ];
       unpack32<BITS>(w, idx);
 #pragma unroll
-      for (int q = 0; q < kQ; q += 2) {
-        const float2 c0 = cb[idx[q]], c1 = cb[idx[q + 1]];
+      for (int q = 0; q < kQ; ++q) {
+        const float2 cw = cb[idx[q]];
 #pragma unroll
         for (int t = 0; t < B; ++t) {
-          const float4 xb = __ldg(reinterpret_cast<const float4*>(xbar + (int64_t)t * P + c * kQ + q));
-          acc[t] = fmaf(xb.x, c0.x, fmaf(xb.y, c0.y, fmaf(xb.z, c1.x, fmaf(xb.w, c1.y, acc[t]))));
+          const float2 xb = __ldg(xbarT + (int64_t)t * P + (int64_t)q * C + c);
+          acc[t] = fmaf(xb.x, cw.x, fmaf(xb.y, cw.y, acc[t]));
         }
       }
     }
@@ -124,9 +365,9 @@ cudaError_t run_gemv(const qamw_matrix& m, int batch, const float2* xbar, uint16
 }
 
 template <int BITS>
-cudaError_t gemv_bits(const qamw_matrix& m, int batch, const float2* xbar, uint16_t* d_y,
-                      cudaStream_t stream) {
-  if (batch == 1) return run_gemv<BITS, 1>(m, batch, xbar, d_y, stream);
+cudaError_t gemv_bits(const qamw_matrix& m, const uint16_t* d_x, int batch, const float2* xbar,
+                      uint16_t* d_y, int32_t* d_status, cudaStream_t stream) {
+  if (batch == 1) return run_gemv1<BITS>(m, d_x, d_y, d_status, stream);
   if (batch <= 4) return run_gemv<BITS, 4>(m, batch, xbar, d_y, stream);
   if (batch <= 8) return run_gemv<BITS, 8>(m, batch, xbar, d_y, stream);
   return run_gemv<BITS, 16>(m, batch, xbar, d_y, stream);
@@ -144,8 +385,8 @@ cudaError_t launch_decode_gemv(const qamw_matrix& m, const uint16_t* d_x, int ba
                                uint16_t* d_y, void* d_ws, int32_t* d_status,
                                cudaStream_t stream) {
   float2* xbar = static_cast<float2*>(d_ws);
-  const int bpad = batch == 1 ? 1 : (batch <= 4 ? 4 : (batch <= 8 ? 8 : 16));
-  {
+  if (batch > 1) {
+    const int bpad = batch <= 4 ? 4 : (batch <= 8 ? 8 : 16);
     const int threads = 256;
     const int64_t V = (int64_t)bpad * (m.d_in / kE);
     const void* fn = reinterpret_cast<const void*>(&k_rotate);
@@ -158,20 +399,20 @@ cudaError_t launch_decode_gemv(const qamw_matrix& m, const uint16_t* d_x, int ba
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
-  // The kernel runs B = 1/4/8/16 columns; columns batch..B-1 read the zeroed
-  // xbar padding and are not written to y.
+  // The batch 2..16 kernels run B = 4/8/16 columns; columns batch..B-1 read
+  // the zeroed xbar padding and are not written to y.
   switch (m.bits) {
-    case 1: return gemv_bits<1>(m, batch, xbar, d_y, stream);
-    case 2: return gemv_bits<2>(m, batch, xbar, d_y, stream);
-    case 3: return gemv_bits<3>(m, batch, xbar, d_y, stream);
-    case 4: return gemv_bits<4>(m, batch, xbar, d_y, stream);
-    case 5: return gemv_bits<5>(m, batch, xbar, d_y, stream);
-    case 6: return gemv_bits<6>(m, batch, xbar, d_y, stream);
-    case 7: return gemv_bits<7>(m, batch, xbar, d_y, stream);
-    case 8: return gemv_bits<8>(m, batch, xbar, d_y, stream);
-    case 9: return gemv_bits<9>(m, batch, xbar, d_y, stream);
-    case 10: return gemv_bits<10>(m, batch, xbar, d_y, stream);
-    case 11: return gemv_bits<11>(m, batch, xbar, d_y, stream);
+    case 1: return gemv_bits<1>(m, d_x, batch, xbar, d_y, d_status, stream);
+    case 2: return gemv_bits<2>(m, d_x, batch, xbar, d_y, d_status, stream);
+    case 3: return gemv_bits<3>(m, d_x, batch, xbar, d_y, d_status, stream);
+    case 4: return gemv_bits<4>(m, d_x, batch, xbar, d_y, d_status, stream);
+    case 5: return gemv_bits<5>(m, d_x, batch, xbar, d_y, d_status, stream);
+    case 6: return gemv_bits<6>(m, d_x, batch, xbar, d_y, d_status, stream);
+    case 7: return gemv_bits<7>(m, d_x, batch, xbar, d_y, d_status, stream);
+    case 8: return gemv_bits<8>(m, d_x, batch, xbar, d_y, d_status, stream);
+    case 9: return gemv_bits<9>(m, d_x, batch, xbar, d_y, d_status, stream);
+    case 10: return gemv_bits<10>(m, d_x, batch, xbar, d_y, d_status, stream);
+    case 11: return gemv_bits<11>(m, d_x, batch, xbar, d_y, d_status, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -13,8 +13,11 @@
 //      four corners decides it.
 // M bounds the fp32 rounding of the encoder's |c|^2 - 2 p.c scores with a wide
 // margin, and cells are grown by eps to cover rounding of the cell index, so a
-// list search returns exactly what the exhaustive fp32 search would.  Cells
-// whose list exceeds kPfCap, and points off the grid, take the exhaustive path.
+// list search returns exactly what the exhaustive fp32 search would.  Points
+// off the grid (|p| >= R) use the list of their angular sector, built by the
+// same dominance test over the unbounded sector region.  Lists that exceed
+// kPfCap (none for the codebooks trained here) and non-finite points take the
+// exhaustive path.
 #include "common.cuh"
 #include "launch.cuh"
 
@@ -55,7 +58,7 @@ __global__ void __launch_bounds__(1024) k_pf_header(const float2* __restrict__ c
     h.G = G;
     h.cap = kPfCap;
     h.K = K;
-    h.pad = 0;
+    h.NS = G > 0 ? kPfSectors : 0;
     *hdr = h;
   }
 }
@@ -73,9 +76,8 @@ __global__ void __launch_bounds__(kBuildWarps * 32) k_pf_build(const float2* __r
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int cell = blockIdx.x * kBuildWarps + wib;
   if (cell >= G * G) return;
-  uint8_t* counts = reinterpret_cast<uint8_t*>(table) + prefilter_counts_offset();
   uint16_t* lists = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(table) +
-                                                prefilter_lists_offset(G));
+                                                prefilter_lists_offset());
   const int gx = cell % G, gy = cell / G;
   const double R = hdr.R, h = hdr.h, M = hdr.margin;
   const double eps = ldexp(R, -16);
@@ -143,13 +145,148 @@ __global__ void __launch_bounds__(kBuildWarps * 32) k_pf_build(const float2* __r
     }
   }
   __syncwarp();
+  uint16_t* L = lists + (size_t)cell * kPfSlots;
   if (overflow || m > kPfCap) {
-    if (lane == 0) counts[cell] = kPfOverflow;
+    if (lane == 0) L[0] = (uint16_t)kPfOverflow;
     return;
   }
-  uint16_t* L = lists + (size_t)cell * kPfCap;
-  for (int t = lane; t < kPfCap; t += 32) L[t] = t < m ? keep[wib][t] : (uint16_t)0;
-  if (lane == 0) counts[cell] = (uint8_t)m;
+  // slot 0: count; slots 1..m: candidates; slots up to 7 repeat the first
+  // candidate (scored without a branch by the encoder); the rest zero
+  if (lane == 0) L[0] = (uint16_t)m;
+  for (int t = lane; t < kPfCap; t += 32)
+    L[1 + t] = t < m ? keep[wib][t] : (t < 7 ? keep[wib][0] : (uint16_t)0);
+}
+
+// Warp-wide argmin_j |q - c_j|^2 (any minimiser will do: it only seeds the
+// dominance test below).
+__device__ int warp_nearest(const float2* cb, int K, double qx, double qy) {
+  const int lane = threadIdx.x & 31;
+  double bd = INFINITY;
+  int bj = 0;
+  for (int j = lane; j < K; j += 32) {
+    const float2 c = cb[j];
+    const double d = (qx - c.x) * (qx - c.x) + (qy - c.y) * (qy - c.y);
+    if (d < bd) {
+      bd = d;
+      bj = j;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const double od = __shfl_xor_sync(0xffffffffu, bd, o);
+    const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+    if (od < bd || (od == bd && oj < bj)) {
+      bd = od;
+      bj = oj;
+    }
+  }
+  return bj;
+}
+
+// Off-grid sector s: the points p = r e(theta), theta in the sector's angle
+// range (grown by eps), r >= R_in, lie in the region beyond the chord P0-P1
+// between the rays e0 and e1: conv{P0, P1} + cone{e0, e1}.  Codeword j is
+// dominated by k over that region when the affine gap
+// |q - c_j|^2 - |q - c_k|^2 exceeds M at P0 and P1 and grows along e0 and e1
+// (slope at least min_slope, which also covers the fp32 rounding of scores of
+// very distant points).
+struct SectorGeom {
+  double p0x, p0y, p1x, p1y, e0x, e0y, e1x, e1y, M, min_slope;
+};
+
+__device__ bool dominated(const SectorGeom& g, float2 cj, float2 ck) {
+  const double dx = (double)ck.x - cj.x, dy = (double)ck.y - cj.y;
+  if (g.e0x * dx + g.e0y * dy < g.min_slope) return false;
+  if (g.e1x * dx + g.e1y * dy < g.min_slope) return false;
+  const double cj2 = (double)cj.x * cj.x + (double)cj.y * cj.y;
+  const double ck2 = (double)ck.x * ck.x + (double)ck.y * ck.y;
+  // |q-c_j|^2 - |q-c_k|^2 = 2 q.(c_k - c_j) + |c_j|^2 - |c_k|^2
+  const double f0 = 2.0 * (g.p0x * dx + g.p0y * dy) + cj2 - ck2;
+  const double f1 = 2.0 * (g.p1x * dx + g.p1y * dy) + cj2 - ck2;
+  return f0 > g.M && f1 > g.M;
+}
+
+constexpr int kRefs = 15;
+
+__global__ void __launch_bounds__(kBuildWarps * 32) k_pf_sectors(const float2* __restrict__ cb,
+                                                                 void* __restrict__ table) {
+  __shared__ uint16_t cand[kBuildWarps][kMaxCand];
+  __shared__ uint16_t keep[kBuildWarps][kMaxCand];
+  const PrefilterHeader hdr = *reinterpret_cast<const PrefilterHeader*>(table);
+  const int G = hdr.G, K = hdr.K, NS = hdr.NS;
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int sct = blockIdx.x * kBuildWarps + wib;
+  if (sct >= NS) return;
+  uint16_t* L = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(table) +
+                                            prefilter_lists_offset()) +
+                ((size_t)G * G + sct) * kPfSlots;
+  const double pi = 3.14159265358979323846, eps = 1e-4;
+  const double t0 = -pi + 2.0 * pi * sct / NS - eps, t1 = -pi + 2.0 * pi * (sct + 1) / NS + eps;
+  const double Rin = (double)hdr.R * (1.0 - 1.0 / 1024);
+  SectorGeom g;
+  g.e0x = cos(t0);
+  g.e0y = sin(t0);
+  g.e1x = cos(t1);
+  g.e1y = sin(t1);
+  g.p0x = Rin * g.e0x;
+  g.p0y = Rin * g.e0y;
+  g.p1x = Rin * g.e1x;
+  g.p1y = Rin * g.e1y;
+  g.M = hdr.margin;
+  g.min_slope = ldexp(1.0 + (double)hdr.R, -16);
+
+  // reference codewords: nearest ones at several radii along e0, e1 and the middle
+  int refs[kRefs];
+  const double tm = 0.5 * (t0 + t1);
+  const double dirs[3][2] = {{g.e0x, g.e0y}, {g.e1x, g.e1y}, {cos(tm), sin(tm)}};
+  const double radii[5] = {1.0, 2.0, 4.0, 16.0, 256.0};
+  for (int d = 0; d < 3; ++d)
+    for (int r = 0; r < 5; ++r)
+      refs[d * 5 + r] = warp_nearest(cb, K, Rin * radii[r] * dirs[d][0], Rin * radii[r] * dirs[d][1]);
+
+  // 1. codewords not dominated by any reference, ascending j
+  int n = 0;
+  for (int j0 = 0; j0 < K; j0 += 32) {
+    const int j = j0 + lane;
+    bool ok = j < K;
+    if (ok) {
+      const float2 cj = cb[j];
+      for (int r = 0; r < kRefs && ok; ++r)
+        if (refs[r] != j && dominated(g, cj, cb[refs[r]])) ok = false;
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, ok);
+    const int pos = n + __popc(bal & ((1u << lane) - 1u));
+    if (ok && pos < kMaxCand) cand[wib][pos] = (uint16_t)j;
+    n += __popc(bal);
+  }
+  __syncwarp();
+  if (n > kMaxCand) {
+    if (lane == 0) L[0] = (uint16_t)kPfOverflow;
+    return;
+  }
+  // 2. candidates not dominated by another candidate
+  int m = 0;
+  for (int u0 = 0; u0 < n; u0 += 32) {
+    const int u = u0 + lane;
+    bool alive = u < n;
+    if (alive) {
+      const float2 cj = cb[cand[wib][u]];
+      for (int v = 0; v < n && alive; ++v)
+        if (v != u && dominated(g, cj, cb[cand[wib][v]])) alive = false;
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, alive);
+    const int pos = m + __popc(bal & ((1u << lane) - 1u));
+    if (alive) keep[wib][pos] = cand[wib][u];
+    m += __popc(bal);
+  }
+  __syncwarp();
+  if (m > kPfCap) {
+    if (lane == 0) L[0] = (uint16_t)kPfOverflow;
+    return;
+  }
+  if (lane == 0) L[0] = (uint16_t)m;
+  for (int t = lane; t < kPfCap; t += 32)
+    L[1 + t] = t < m ? keep[wib][t] : (t < 7 ? keep[wib][0] : (uint16_t)0);
 }
 
 }  // namespace
@@ -165,6 +302,9 @@ cudaError_t launch_build_prefilter(const float* d_codebook, int bits, void* d_ta
   if (err != cudaSuccess || G == 0) return err;
   const int cells = G * G;
   k_pf_build<<<(cells + kBuildWarps - 1) / kBuildWarps, kBuildWarps * 32, 0, stream>>>(cb, d_table);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  const int NS = prefilter_sectors(bits);
+  k_pf_sectors<<<(NS + kBuildWarps - 1) / kBuildWarps, kBuildWarps * 32, 0, stream>>>(cb, d_table);
   return cudaGetLastError();
 }
 

@@ -2,6 +2,9 @@
 // circular Gaussian (paper section 3.6 eq. 2).
 //
 // Per iteration:
+//   prefilter: the exact nearest-codeword table of the current codebook
+//              (prefilter.cu), so that each sample scores a few codewords
+//              instead of K; the assignment equals the exhaustive fp32 search;
 //   k_assign : every sample -> nearest codeword (fp32, lowest index on ties);
 //              cell sums of x, y and of the squared distance are accumulated
 //              as 64-bit integers in units of 2^-28, first in shared memory
@@ -39,7 +42,8 @@ __global__ void k_init(const float2* __restrict__ samples, int K, float2* __rest
 
 __global__ void __launch_bounds__(512) k_assign(const float2* __restrict__ samples, int64_t n,
                                                 const float2* __restrict__ cb, int K,
-                                                TrainAccum acc, int32_t* status) {
+                                                const void* __restrict__ table, TrainAccum acc,
+                                                int32_t* status) {
   extern __shared__ __align__(16) unsigned char smem[];
   float4* cbq = reinterpret_cast<float4*>(smem);
   unsigned long long* ssx = reinterpret_cast<unsigned long long*>(cbq + K);
@@ -56,6 +60,13 @@ __global__ void __launch_bounds__(512) k_assign(const float2* __restrict__ sampl
     sd = 0ull;
     sn = 0ull;
   }
+  PrefilterView pf;
+  if (table != nullptr) {
+    pf = prefilter_view(table, K);
+  } else {
+    pf.G = 0;
+    pf.Gf = 0.f;
+  }
   __syncthreads();
   int flags = 0;
   unsigned long long my_d = 0ull, my_n = 0ull;
@@ -71,7 +82,7 @@ __global__ void __launch_bounds__(512) k_assign(const float2* __restrict__ sampl
       continue;
     }
     unsigned scored = 0;
-    const int j = nearest_all(-2.f * p.x, -2.f * p.y, cbq, K, scored);
+    const int j = nearest_pf(p.x, p.y, cbq, K, pf, scored);
     const float dx = p.x - cbq[j].x, dy = p.y - cbq[j].y;
     const float d = fmaf(dx, dx, dy * dy);
     atomicAdd(&ssx[j], (unsigned long long)__float2ll_rn(p.x * kFix));
@@ -128,7 +139,8 @@ __global__ void k_zero_u64(unsigned long long* p, int n) {
 
 size_t train_workspace_bytes(int bits) {
   const size_t K = (size_t)1 << bits;
-  return (3 * K + 2) * sizeof(unsigned long long);
+  const size_t acc = ((3 * K + 2) * sizeof(unsigned long long) + 255) & ~(size_t)255;
+  return acc + prefilter_bytes_for(bits);
 }
 
 cudaError_t launch_train(const float* d_samples, int64_t n, int bits, int iters, float* d_codebook,
@@ -139,6 +151,8 @@ cudaError_t launch_train(const float* d_samples, int64_t n, int bits, int iters,
   float2* cb = reinterpret_cast<float2*>(d_codebook);
   unsigned long long* w = static_cast<unsigned long long*>(d_ws);
   TrainAccum acc{w, w + K, w + 2 * K, w + 3 * K, w + 3 * K + 1};
+  const size_t acc_bytes = ((3 * (size_t)K + 2) * sizeof(unsigned long long) + 255) & ~(size_t)255;
+  void* table = prefilter_grid(bits) > 0 ? static_cast<char*>(d_ws) + acc_bytes : nullptr;
   const int nz = 3 * K + 2;
   k_zero_u64<<<(nz + 255) / 256, 256, 0, stream>>>(w, nz);
   k_init<<<(K + 255) / 256, 256, 0, stream>>>(samples, K, cb);
@@ -150,7 +164,10 @@ cudaError_t launch_train(const float* d_samples, int64_t n, int bits, int iters,
   if ((err = allow_smem(fn, smem)) != cudaSuccess) return err;
   const int grid = persistent_grid(fn, threads, smem, (n + threads - 1) / threads);
   for (int it = 0; it < iters; ++it) {
-    k_assign<<<grid, threads, smem, stream>>>(samples, n, cb, K, acc, d_status);
+    if (table != nullptr) {
+      if ((err = launch_build_prefilter(d_codebook, bits, table, stream)) != cudaSuccess) return err;
+    }
+    k_assign<<<grid, threads, smem, stream>>>(samples, n, cb, K, table, acc, d_status);
     k_update<<<(K + 255) / 256, 256, 0, stream>>>(cb, K, acc, d_distortion, it);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }

@@ -29,6 +29,7 @@ QAMW_ERR_CUDA = -5
 QAMW_STATUS_NONFINITE = 0x1
 QAMW_STATUS_RANGE = 0x2
 QAMW_STATUS_BAD_STAT = 0x4
+QAMW_STATUS_TIMEOUT = 0x8
 QAMW_DTYPE_F32 = 0
 QAMW_DTYPE_BF16 = 1
 QAMW_SIGMA_GIVEN = 0x1
