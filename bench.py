@@ -522,15 +522,30 @@ def run_single_stage(args) -> dict:
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        fn()
-    e1.record()
+    if args.eager:
+        e0.record()
+        for _ in range(args.steps):
+            fn()
+        e1.record()
+    else:
+        # `steps` back-to-back calls captured in one CUDA graph: device time only,
+        # no host launch overhead between calls (the warm-up filled the library's
+        # launch-shape caches, so capture sees launches only)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(args.steps):
+                fn()
+        graph.replay()
+        torch.cuda.synchronize()
+        e0.record()
+        graph.replay()
+        e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
     ab = algorithmic_bytes(rows, D_IN, BITS, args.batch)
     key = {"encode": "encode", "calibrate": "encode", "decode": "decode", "gemv": "gemv"}.get(args.only)
     out = dict(stage=args.only, rows=rows, d_in=D_IN, batch=args.batch, ms=ms,
+               timing="eager" if args.eager else "cuda graph of back-to-back calls",
                Mweights_per_s=rows * D_IN / (ms * 1e-3) / 1e6)
     if key:
         out["GB_per_s"] = ab[key] / (ms * 1e-3) / 1e9
@@ -550,6 +565,7 @@ def main(argv=None) -> int:
     ap.add_argument("--rows", type=int, default=16384, help="--only: rows of the d_in=4096 matrix")
     ap.add_argument("--batch", type=int, default=1, help="--only gemv: batch columns")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--eager", action="store_true", help="--only: time eager calls, not a graph")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

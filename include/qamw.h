@@ -96,8 +96,8 @@ typedef struct qamw_matrix {
     int64_t row_bytes;      /* must equal qamw_row_bytes(d_in, bits)         */
     uint8_t *packed;        /* [d_out][row_bytes] bit-packed indices, 16B-aligned */
     uint16_t *row_norm;     /* [d_out] binary16 row norms r                   */
-    uint16_t *sigma;        /* [d_in/2] binary16 pair scales sigma_k          */
-    uint16_t *chan_scale;   /* [d_in] binary16 channel scales s_j             */
+    uint16_t *sigma;        /* [d_in/2] binary16 pair scales sigma_k, 16B-aligned */
+    uint16_t *chan_scale;   /* [d_in] binary16 channel scales s_j, 16B-aligned */
     const float *codebook;  /* [K][2] fp32 codewords (x, y), 16B-aligned      */
     const void *prefilter;  /* table from qamw_build_prefilter() for this
                                codebook, or NULL (then qamw_encode builds one

@@ -100,10 +100,14 @@ def _encode(m, W=FAKE, dtype=qamw.QAMW_DTYPE_BF16, flags=0, ws=FAKE, ws_bytes=1 
     (dict(codebook=None), qamw.QAMW_ERR_INVALID),
     (dict(packed=FAKE + 8), qamw.QAMW_ERR_ALIGN),
     (dict(codebook=FAKE + 4), qamw.QAMW_ERR_ALIGN),
+    (dict(sigma=FAKE + 2), qamw.QAMW_ERR_ALIGN),
+    (dict(chan_scale=FAKE + 8), qamw.QAMW_ERR_ALIGN),
 ])
 def test_matrix_argument_errors(kw, rc):
     m = _matrix(**kw)
     assert _encode(m) == rc
+    assert qamw.lib().qamw_decode_gemv_noalloc(C.byref(m), C.c_void_p(FAKE), 1, C.c_void_p(FAKE),
+                                               None, None) == rc
     assert qamw.lib().qamw_decode(C.byref(m), C.c_void_p(FAKE), None, None) == rc
     assert qamw.lib().qamw_decode_gemv(C.byref(m), C.c_void_p(FAKE), 1, C.c_void_p(FAKE),
                                        C.c_void_p(FAKE), 1 << 40, None, None) == rc

@@ -21,12 +21,64 @@ int sm_count() {
   return cached[dev];
 }
 
+// Occupancy and shared-memory opt-in are per (device, kernel, shape) facts:
+// computed once and cached, so that a call costs the launches and little else.
+namespace {
+struct LaunchKey {
+  int dev;
+  const void* fn;
+  int threads;
+  size_t smem;
+  bool operator==(const LaunchKey& o) const {
+    return dev == o.dev && fn == o.fn && threads == o.threads && smem == o.smem;
+  }
+};
+struct LaunchCache {
+  std::mutex mu;
+  LaunchKey key[256];
+  int value[256];
+  int n = 0;
+};
+LaunchCache g_occupancy, g_smem_optin;
+
+bool cache_get(LaunchCache& c, const LaunchKey& k, int* v) {
+  std::lock_guard<std::mutex> lock(c.mu);
+  for (int i = 0; i < c.n; ++i)
+    if (c.key[i] == k) {
+      *v = c.value[i];
+      return true;
+    }
+  return false;
+}
+
+void cache_put(LaunchCache& c, const LaunchKey& k, int v) {
+  std::lock_guard<std::mutex> lock(c.mu);
+  for (int i = 0; i < c.n; ++i)
+    if (c.key[i] == k) return;
+  if (c.n < 256) {
+    c.key[c.n] = k;
+    c.value[c.n] = v;
+    ++c.n;
+  }
+}
+
+int current_device() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return dev;
+}
+}  // namespace
+
 int persistent_grid(const void* kernel, int threads, size_t smem, int64_t work_ctas) {
+  const LaunchKey k{current_device(), kernel, threads, smem};
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) !=
-          cudaSuccess ||
-      per_sm < 1)
-    per_sm = 1;
+  if (!cache_get(g_occupancy, k, &per_sm)) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) !=
+            cudaSuccess ||
+        per_sm < 1)
+      per_sm = 1;
+    cache_put(g_occupancy, k, per_sm);
+  }
   const int64_t resident = (int64_t)per_sm * sm_count();
   int64_t g = work_ctas < resident ? work_ctas : resident;
   return (int)(g < 1 ? 1 : g);
@@ -34,7 +86,27 @@ int persistent_grid(const void* kernel, int threads, size_t smem, int64_t work_c
 
 cudaError_t allow_smem(const void* kernel, size_t smem) {
   if (smem <= 48 * 1024) return cudaSuccess;
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // the attribute is a maximum: one call with the largest size seen so far
+  const LaunchKey k{current_device(), kernel, 0, 0};
+  int have = 0;
+  if (cache_get(g_smem_optin, k, &have) && (size_t)have >= smem) return cudaSuccess;
+  const cudaError_t err =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err == cudaSuccess) {
+    std::lock_guard<std::mutex> lock(g_smem_optin.mu);
+    bool found = false;
+    for (int i = 0; i < g_smem_optin.n; ++i)
+      if (g_smem_optin.key[i] == k) {
+        if (g_smem_optin.value[i] < (int)smem) g_smem_optin.value[i] = (int)smem;
+        found = true;
+      }
+    if (!found && g_smem_optin.n < 256) {
+      g_smem_optin.key[g_smem_optin.n] = k;
+      g_smem_optin.value[g_smem_optin.n] = (int)smem;
+      ++g_smem_optin.n;
+    }
+  }
+  return err;
 }
 
 }  // namespace qamw
@@ -64,6 +136,7 @@ int check_matrix(const qamw_matrix* m, bool need_outputs) {
   if (!m->packed || !m->row_norm || !m->sigma || !m->chan_scale || !m->codebook)
     return QAMW_ERR_INVALID;
   if (!aligned16(m->packed) || !aligned16(m->codebook)) return QAMW_ERR_ALIGN;
+  if (!aligned16(m->sigma) || !aligned16(m->chan_scale)) return QAMW_ERR_ALIGN;
   if (m->prefilter && !aligned16(m->prefilter)) return QAMW_ERR_ALIGN;
   (void)need_outputs;
   return QAMW_OK;

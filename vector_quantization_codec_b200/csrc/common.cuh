@@ -148,6 +148,46 @@ __device__ __forceinline__ void load64(const __nv_bfloat16* p, float (&x)[kE]) {
   }
 }
 
+// n consecutive binary16 values (n a multiple of 8, 16-byte aligned) as fp32,
+// with all loads issued before any use.
+template <int N>
+__device__ __forceinline__ void load_halves(const __half* p, float (&x)[N]) {
+  uint4 v[N / 8];
+  const uint4* s = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int t = 0; t < N / 8; ++t) v[t] = __ldg(s + t);
+#pragma unroll
+  for (int t = 0; t < N / 8; ++t) {
+    const __half2* h = reinterpret_cast<const __half2*>(&v[t]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(h[e]);
+      x[8 * t + 2 * e] = f.x;
+      x[8 * t + 2 * e + 1] = f.y;
+    }
+  }
+}
+
+// Cooperative fill of a chunk-interleaved table: dst[(j % PERIOD) * C + j / PERIOD]
+// = f(j, src[j]) for j < n, src binary16 (16-byte aligned, n a multiple of 8),
+// 8 values per 16-byte load, every thread's loads issued together.
+template <int PERIOD, typename F>
+__device__ __forceinline__ void fill_interleaved(float* dst, const __half* src, int n, int C,
+                                                 F f) {
+#pragma unroll 2
+  for (int j8 = threadIdx.x * 8; j8 < n; j8 += blockDim.x * 8) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + j8));
+    const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f2 = __half22float2(h[e]);
+      const int j = j8 + 2 * e;
+      dst[(j % PERIOD) * C + j / PERIOD] = f(j, f2.x);
+      dst[((j + 1) % PERIOD) * C + (j + 1) / PERIOD] = f(j + 1, f2.y);
+    }
+  }
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -217,9 +257,12 @@ struct PrefilterHeader {
   int32_t NS;    // angular sectors for points off the grid (|p| >= R)
 };
 
-// Each cell's list is 32 uint16: entry 0 is the count (kPfOverflow: search
-// exhaustively), entries 1..count the candidate indices in ascending order.
-// One 16-byte load fetches the count and the first 7 candidates.
+// Each cell's list is 32 uint16 slots: slot 0 is the count (kPfOverflow:
+// search exhaustively), slots 1..count the candidate indices in ascending
+// order.  Slots 0-7 of every list (the "head") are stored together in one
+// array of 16-byte entries -- one load fetches the count and the first 7
+// candidates, and a 128-byte line holds 8 neighbouring heads -- and slots
+// 8-31 (the "tail", rarely needed) in a second array.
 constexpr int kPfSlots = 32;
 constexpr int kPfCap = kPfSlots - 1;         // candidates per cell
 constexpr uint32_t kPfOverflow = 0xffffu;
@@ -246,12 +289,25 @@ __host__ __device__ inline size_t prefilter_bytes_for(int bits) {
          ((size_t)G * G + prefilter_sectors(bits)) * kPfSlots * sizeof(uint16_t);
 }
 
+// List n (cells 0..G*G-1, then sectors): head at heads[n], tail at tails[3n..3n+2].
+__host__ __device__ inline size_t prefilter_tails_offset(int bits) {
+  const int G = prefilter_grid(bits);
+  return prefilter_lists_offset() + ((size_t)G * G + prefilter_sectors(bits)) * 16;
+}
+
+__device__ __forceinline__ uint16_t* prefilter_slot(void* table, int G, int NS, size_t n, int t) {
+  uint8_t* base = reinterpret_cast<uint8_t*>(table) + prefilter_lists_offset();
+  if (t < 8) return reinterpret_cast<uint16_t*>(base + n * 16) + t;
+  const size_t nlists = (size_t)G * G + NS;
+  return reinterpret_cast<uint16_t*>(base + nlists * 16 + n * 48) + (t - 8);
+}
+
 struct PrefilterView {
   float R, inv_h, Gf;
   int G;  // 0: exhaustive search only
   int NS;
-  const uint4* lists;    // [G*G][4] (32 uint16 per cell)
-  const uint4* sectors;  // [NS][4]
+  const uint4* heads;  // [G*G + NS]
+  const uint4* tails;  // [G*G + NS][3]
 };
 
 // A table built for another codebook size is ignored (exhaustive search), so a
@@ -264,9 +320,9 @@ __device__ __forceinline__ PrefilterView prefilter_view(const void* table, int K
   v.G = (h->K == K && h->cap == kPfCap && h->NS == kPfSectors) ? h->G : 0;
   v.NS = h->NS;
   v.Gf = (float)v.G;
-  v.lists = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(table) +
+  v.heads = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(table) +
                                            prefilter_lists_offset());
-  v.sectors = v.lists + (size_t)v.G * v.G * (kPfSlots / 8);
+  v.tails = v.heads + ((size_t)h->G * h->G + h->NS);
   return v;
 }
 
@@ -307,38 +363,39 @@ __device__ __forceinline__ void score(float m2x, float m2y, const float4* cbq, u
 // Split form of nearest_pf, so that a caller can fetch the next point's list
 // head while it scores the current point.
 struct PfCursor {
-  const uint4* L;  // nullptr: exhaustive search
+  const uint4* tail;  // nullptr: exhaustive search
   uint4 head;
 };
 
 __device__ __forceinline__ PfCursor pf_locate(float px, float py, const PrefilterView& pf) {
   PfCursor cur;
-  cur.L = nullptr;
+  cur.tail = nullptr;
   cur.head = make_uint4(0u, 0u, 0u, 0u);
   if (pf.G > 0 && isfinite(px) && isfinite(py)) {
     const float gx = (px + pf.R) * pf.inv_h;
     const float gy = (py + pf.R) * pf.inv_h;
+    size_t n;
     if (gx >= 0.f && gx < pf.Gf && gy >= 0.f && gy < pf.Gf) {
-      cur.L = pf.lists + ((size_t)((int)gy * pf.G + (int)gx)) * (kPfSlots / 8);
+      n = (size_t)((int)gy * pf.G + (int)gx);
     } else {
       const float t = (atan2f(py, px) + 3.14159265f) * ((float)pf.NS * 0.159154943f);
-      const int sct = min(max((int)t, 0), pf.NS - 1);
-      cur.L = pf.sectors + (size_t)sct * (kPfSlots / 8);
+      n = (size_t)pf.G * pf.G + min(max((int)t, 0), pf.NS - 1);
     }
-    cur.head = __ldg(cur.L);
+    cur.head = __ldg(pf.heads + n);
+    cur.tail = pf.tails + 3 * n;
   }
   return cur;
 }
 
-// Rare paths of pf_finish: lists longer than 7 (slots 8..count), overflowed
-// lists and points that are not finite (exhaustive search).  Kept out of line
-// so that the common path stays small.
-static __device__ __noinline__ int pf_finish_slow(const uint4* L, uint32_t cnt, float m2x, float m2y,
-                                           const float4* cbq, int K, float be, int bi,
-                                           unsigned* scored) {
-  if (L == nullptr || cnt == kPfOverflow) return nearest_all(m2x, m2y, cbq, K, *scored);
+// Rare paths of pf_finish: lists longer than 7 (tail slots 8..count),
+// overflowed lists and points that are not finite (exhaustive search).  Kept
+// out of line so that the common path stays small.
+static __device__ __noinline__ int pf_finish_slow(const uint4* tail, uint32_t cnt, float m2x,
+                                                  float m2y, const float4* cbq, int K, float be,
+                                                  int bi, unsigned* scored) {
+  if (tail == nullptr || cnt == kPfOverflow) return nearest_all(m2x, m2y, cbq, K, *scored);
   for (uint32_t g = 1; g * 8 <= cnt; ++g) {
-    const uint4 q = __ldg(L + g);
+    const uint4 q = __ldg(tail + (g - 1));
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       if (g * 8 + e > cnt) break;
@@ -359,7 +416,7 @@ __device__ __forceinline__ int pf_finish(const PfCursor& cur, float px, float py
   const uint32_t cnt = q.x & 0xffffu;
   float be = INFINITY;
   int bi = 0;
-  if (cur.L != nullptr && cnt != kPfOverflow) {
+  if (cur.tail != nullptr && cnt != kPfOverflow) {
     scored += cnt;
     score(m2x, m2y, cbq, q.x >> 16, be, bi);
     score(m2x, m2y, cbq, q.y & 0xffffu, be, bi);
@@ -370,7 +427,7 @@ __device__ __forceinline__ int pf_finish(const PfCursor& cur, float px, float py
     score(m2x, m2y, cbq, q.w >> 16, be, bi);
     if (cnt < 8) return bi;
   }
-  return pf_finish_slow(cur.L, cnt, m2x, m2y, cbq, K, be, bi, &scored);
+  return pf_finish_slow(cur.tail, cnt, m2x, m2y, cbq, K, be, bi, &scored);
 }
 
 // Nearest codeword through the prefilter (same result as nearest_all).

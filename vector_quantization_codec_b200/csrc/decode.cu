@@ -24,6 +24,7 @@ struct DecodeArgs {
   const __half* scale;
   const float2* codebook;
   __nv_bfloat16* out;
+  int32_t* status;
   int64_t row_bytes;
   int d_out, d_in, block, K;
   uint64_t seed;
@@ -46,53 +47,120 @@ __device__ __forceinline__ void gather_pairs(const uint32_t (&w)[BITS], const fl
       ...);
 }
 
+constexpr int kDecStages = 2;
+
+// Bytes of the input stage of one CTA iteration: its T chunks' words, the row
+// padding between them, and 16-byte alignment at both ends.
+__host__ __device__ inline unsigned decode_stage_bytes(int threads, int bits) {
+  return (unsigned)(((size_t)threads * (bits * 4 + 16) + 32 + 15) & ~(size_t)15);
+}
+
+// First byte and length (16-byte aligned) of the packed words of virtual
+// threads [v0, v1).
+__device__ __forceinline__ void chunk_span(const DecodeArgs& a, int C, int BITS, int64_t v0,
+                                           int64_t v1, int64_t& start16, unsigned& bytes) {
+  const int64_t r0 = v0 / C, r1 = (v1 - 1) / C;
+  const int64_t s = r0 * a.row_bytes + (v0 - r0 * C) * BITS * 4;
+  const int64_t e = r1 * a.row_bytes + (v1 - 1 - r1 * C + 1) * BITS * 4;
+  start16 = s & ~(int64_t)15;
+  bytes = (unsigned)(((e + 15) & ~(int64_t)15) - start16);
+}
+
 // Per-column factors live transposed in shared memory, [position in chunk][chunk],
 // so that the 32 lanes of a warp (32 consecutive chunks) read 32 consecutive
-// words.  Each warp's output -- 32 chunks of 64 BF16 = 4 KB, contiguous in W_hat
-// because virtual thread v owns bytes [128 v, 128 v + 128) -- is staged in a
-// swizzled shared tile (16-byte unit t of lane l at slot t ^ (l & 7), no bank
-// conflicts on either side) and written back with 512-byte coalesced stores.
+// words.  The packed words of each grid-stride iteration -- one contiguous byte
+// range, since consecutive virtual threads own consecutive chunks -- arrive by
+// cp.async.bulk into a 2-stage ring ahead of use (two CTAs fit on an SM).  Each warp's output -- 32
+// chunks of 64 BF16 = 4 KB, contiguous in W_hat because virtual thread v owns
+// bytes [128 v, 128 v + 128) -- is staged in a swizzled shared tile (16-byte
+// unit t of lane l at slot t ^ (l & 7), no bank conflicts on either side) and
+// written back with 512-byte coalesced stores.
 template <int BITS>
 __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  uint4* stage = reinterpret_cast<uint4*>(smem);                  // [warps][32 lanes][8]
-  float2* cb = reinterpret_cast<float2*>(stage + blockDim.x * 8);
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint4* stage = reinterpret_cast<uint4*>(smem);  // [warps][32 lanes][8] output tile
+  const unsigned in_bytes = decode_stage_bytes(blockDim.x, BITS);
+  unsigned char* in = smem + (size_t)blockDim.x * 128;  // [kDecStages][in_bytes]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(in + (size_t)kDecStages * in_bytes);
+  int* issued = reinterpret_cast<int*>(bar + kDecStages);
+  float2* cb = reinterpret_cast<float2*>(bar + kDecStages + 2);
   const int P = a.d_in >> 1, C = a.d_in / kE;
   float* sgT = reinterpret_cast<float*>(cb + a.K);  // [q][c] = sigma_{32c+q}
   float* gT = sgT + P;                               // [j][c] = D/(sqrt(b) s) of column 64c+j
+  const int64_t V = (int64_t)a.d_out * C;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
 
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(&bar[s], 1);
+      issued[s] = 0;
+    }
+    fence_mbar_init();
+    for (int s = 0; s < kDecStages; ++s) {
+      const int64_t b0 = (int64_t)blockIdx.x * blockDim.x + s * stride;
+      if (b0 >= V) break;
+      int64_t st16;
+      unsigned nb;
+      chunk_span(a, C, BITS, b0, min(b0 + (int64_t)blockDim.x, V), st16, nb);
+      mbar_expect_tx(&bar[s], nb);
+      bulk_g2s(in + (size_t)s * in_bytes, a.packed + st16, nb, &bar[s]);
+      issued[s] = 1;
+    }
+  }
   // table fills: unrolled so that each thread's loads are in flight together
 #pragma unroll 4
   for (int i = threadIdx.x; i < a.K; i += blockDim.x) cb[i] = a.codebook[i];
-#pragma unroll 4
-  for (int k = threadIdx.x; k < P; k += blockDim.x)
-    sgT[(k % kQ) * C + k / kQ] = __half2float(a.sigma[k]);
+  fill_interleaved<kQ>(sgT, a.sigma, P, C, [](int, float v) { return v; });
   const float inv_sqrt_b = 1.0f / sqrtf((float)a.block);
-#pragma unroll 4
-  for (int j = threadIdx.x; j < a.d_in; j += blockDim.x) {
-    const float v = inv_sqrt_b / __half2float(a.scale[j]);
-    gT[(j % kE) * C + j / kE] = mask_negative(a.seed, (uint32_t)j) ? -v : v;
-  }
+  const uint64_t seed = a.seed;
+  fill_interleaved<kE>(gT, a.scale, a.d_in, C, [=](int j, float sv) {
+    const float v = inv_sqrt_b / sv;
+    return mask_negative(seed, (uint32_t)j) ? -v : v;
+  });
   __syncthreads();
 
   const int lane = threadIdx.x & 31;
   uint4* wstage = stage + (threadIdx.x >> 5) * 256;
-  const int64_t V = (int64_t)a.d_out * C;
   const int nb = min(a.block, kE);
   const int lanes = max(a.block / kE, 1);
   uint4* out16 = reinterpret_cast<uint4*>(a.out);
-  for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < V;
-       base += (int64_t)gridDim.x * blockDim.x) {
+  int flags = 0;
+  int it = 0;
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < V; base += stride, ++it) {
+    const int stg = it % kDecStages;
+    const bool ok = mbar_wait_bounded(&bar[stg], (unsigned)(it / kDecStages) & 1u);
+    if (__syncthreads_or(!ok)) {
+      flags |= QAMW_STATUS_TIMEOUT;
+      break;
+    }
     const int64_t v = base + threadIdx.x;
     const bool active = v < V;
     const int64_t row = active ? v / C : 0;
     const int c = active ? (int)(v - row * C) : 0;
 
     uint32_t w[BITS];
-    const uint32_t* src =
-        reinterpret_cast<const uint32_t*>(a.packed + row * a.row_bytes) + (size_t)c * BITS;
+    {
+      int64_t st16;
+      unsigned nbytes;
+      chunk_span(a, C, BITS, base, min(base + (int64_t)blockDim.x, V), st16, nbytes);
+      const int64_t off = active ? row * a.row_bytes + (int64_t)c * BITS * 4 - st16 : 0;
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(in + (size_t)stg * in_bytes + off);
 #pragma unroll
-    for (int t = 0; t < BITS; ++t) w[t] = active ? __ldg(src + t) : 0u;
+      for (int t = 0; t < BITS; ++t) w[t] = active ? src[t] : 0u;
+    }
+    __syncthreads();  // every thread has its words: the stage can be refilled
+    if (threadIdx.x == 0) {
+      const int64_t b2 = base + (int64_t)kDecStages * stride;
+      if (b2 < V) {
+        int64_t st16;
+        unsigned nbytes;
+        chunk_span(a, C, BITS, b2, min(b2 + (int64_t)blockDim.x, V), st16, nbytes);
+        mbar_expect_tx(&bar[stg], nbytes);
+        bulk_g2s(in + (size_t)stg * in_bytes, a.packed + st16, nbytes, &bar[stg]);
+        issued[stg] += 1;
+      }
+    }
+
     float x[kE];
     gather_pairs<BITS>(w, cb, sgT + c, C, x, std::make_integer_sequence<int, kQ>{});
     fwht_reg<kE>(x, nb);
@@ -119,10 +187,19 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
     }
     __syncwarp();
   }
+  // after a timeout: let the copies still in flight land before this CTA's
+  // shared memory goes away
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDecStages; ++s)
+      if (issued[s] > 0) mbar_wait_bounded(&bar[s], (unsigned)(issued[s] - 1) & 1u);
+  }
+  raise_flag(a.status, flags);
 }
 
-size_t decode_smem(int threads, const DecodeArgs& a) {
-  return (size_t)threads * 128 + (size_t)a.K * sizeof(float2) +
+size_t decode_smem(int threads, const DecodeArgs& a, int bits) {
+  return (size_t)threads * 128 + (size_t)kDecStages * decode_stage_bytes(threads, bits) +
+         (kDecStages + 2) * sizeof(uint64_t) + (size_t)a.K * sizeof(float2) +
          (size_t)(a.d_in / 2) * sizeof(float) + (size_t)a.d_in * sizeof(float);
 }
 
@@ -130,8 +207,9 @@ template <int BITS>
 cudaError_t run_decode(const DecodeArgs& a, cudaStream_t stream) {
   // 256 threads, or 128 when the per-column tables of a very wide matrix leave
   // no room for a 32 KB staging tile within the 227 KB a CTA may use
-  const int threads = decode_smem(kDecThreads, a) <= 227 * 1024 ? kDecThreads : kDecThreads / 2;
-  const size_t smem = decode_smem(threads, a);
+  const int threads =
+      decode_smem(kDecThreads, a, BITS) <= 227 * 1024 ? kDecThreads : kDecThreads / 2;
+  const size_t smem = decode_smem(threads, a, BITS);
   const void* fn = reinterpret_cast<const void*>(&k_decode<BITS>);
   cudaError_t err = allow_smem(fn, smem);
   if (err != cudaSuccess) return err;
@@ -145,8 +223,8 @@ cudaError_t run_decode(const DecodeArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_decode(const qamw_matrix& m, uint16_t* d_out, int32_t* d_status,
                           cudaStream_t stream) {
-  (void)d_status;
   DecodeArgs a;
+  a.status = d_status;
   a.packed = m.packed;
   a.rnorm = reinterpret_cast<const __half*>(m.row_norm);
   a.sigma = reinterpret_cast<const __half*>(m.sigma);

@@ -2,7 +2,7 @@
 // activation-aware per-channel scaling).
 //
 // Kernels, in stream order:
-//   k_scales        s_j = binary16((a_j / mean a)^alpha)          (1 CTA)
+//   k_scales        s_j = binary16((a_j / mean a)^alpha)          (thread/channel)
 //   k_rownorm       r_i = ||w_i * s||_2 (fp32), r_hat = binary16(r) (warp/row)
 //   k_calib_select  the first min(1024, #non-zero) non-zero rows   (1 CTA)
 //   k_calib_accum   per-CTA sums of |z_k| over those rows           (128 CTAs)
@@ -18,12 +18,15 @@ namespace {
 
 // ------------------------------------------------------------------ scales
 
-__global__ void __launch_bounds__(1024) k_scales(const float* __restrict__ a, int d_in,
-                                                 float alpha, __half* __restrict__ s,
-                                                 int32_t* status) {
-  __shared__ double red[32];
-  int bad = 0;
+// Every CTA sums the whole statistic in the same fixed order (fp64), so all
+// CTAs see the identical mean; each then rounds its slice of scales.
+__global__ void __launch_bounds__(256) k_scales(const float* __restrict__ a, int d_in,
+                                                float alpha, __half* __restrict__ s,
+                                                int32_t* status) {
+  __shared__ double red[8];
   double sum = 0.0;
+  int bad = 0;
+#pragma unroll 8
   for (int j = threadIdx.x; j < d_in; j += blockDim.x) {
     const float v = a[j];
     if (v > 0.f && isfinite(v))
@@ -31,21 +34,16 @@ __global__ void __launch_bounds__(1024) k_scales(const float* __restrict__ a, in
     else
       bad = 1;
   }
-  // fixed-order tree reduction (deterministic)
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sum;
   __syncthreads();
-  if (threadIdx.x < 32) {
-    double t = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-    if (threadIdx.x == 0) red[0] = t;
-  }
-  __syncthreads();
-  const double mean = red[0] / (double)d_in;
+  double total = 0.0;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) total += red[w];
+  const double mean = total / (double)d_in;
   int range = 0;
-  for (int j = threadIdx.x; j < d_in; j += blockDim.x) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j < d_in) {
     const float v = a[j];
     __half h;
     if (v > 0.f && isfinite(v)) {
@@ -57,7 +55,9 @@ __global__ void __launch_bounds__(1024) k_scales(const float* __restrict__ a, in
     }
     s[j] = h;
   }
-  raise_flag(status, (bad ? QAMW_STATUS_BAD_STAT : 0) | (range ? QAMW_STATUS_RANGE : 0));
+  if (blockIdx.x == 0) bad = __syncthreads_or(bad);
+  raise_flag(status, ((blockIdx.x == 0 && bad) ? QAMW_STATUS_BAD_STAT : 0) |
+                         (range ? QAMW_STATUS_RANGE : 0));
 }
 
 __global__ void k_fill_half(__half* p, int n, float v) {
@@ -179,11 +179,9 @@ __global__ void __launch_bounds__(MAXT) k_calib_accum(const T* __restrict__ W,
   const int C = d_in / kE, P = d_in / 2;
   float* fT = sm;            // [j][c]: D * s of column 64c + j
   float* red = sm + d_in;    // [g][q][c]
-#pragma unroll 4
-  for (int j = threadIdx.x; j < d_in; j += blockDim.x) {
-    const float v = __half2float(s[j]);
-    fT[(j % kE) * C + j / kE] = mask_negative(seed, (uint32_t)j) ? -v : v;
-  }
+  fill_interleaved<kE>(fT, s, d_in, C, [=](int j, float v) {
+    return mask_negative(seed, (uint32_t)j) ? -v : v;
+  });
   __syncthreads();
   const int g = threadIdx.x / C, c = threadIdx.x - g * C;
   const bool lane_ok = g < RPC;
@@ -231,13 +229,20 @@ __global__ void __launch_bounds__(MAXT) k_calib_accum(const T* __restrict__ W,
   }
 }
 
-__global__ void k_calib_finish(const float* __restrict__ partial, int nparts,
-                               const int32_t* __restrict__ n_cal_p, int P,
-                               __half* __restrict__ sigma, int32_t* status) {
-  const int k = blockIdx.x * blockDim.x + threadIdx.x;
-  if (k >= P) return;
+// 16 threads per pair k: thread i sums partials i, i+16, ... in fp64, then the
+// 16 sums are combined by a fixed shuffle tree (deterministic).
+__global__ void __launch_bounds__(256) k_calib_finish(const float* __restrict__ partial,
+                                                      int nparts, const int32_t* __restrict__ n_cal_p,
+                                                      int P, __half* __restrict__ sigma,
+                                                      int32_t* status) {
+  const int g = blockIdx.x * (blockDim.x / 16) + threadIdx.x / 16, i = threadIdx.x & 15;
+  const int k = min(g, P - 1);
   double sum = 0.0;
-  for (int p = 0; p < nparts; ++p) sum += (double)partial[(size_t)p * P + k];
+#pragma unroll 8
+  for (int p = i; p < nparts; p += 16) sum += (double)partial[(size_t)p * P + k];
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (i != 0 || g >= P) return;
   const int n = *n_cal_p;
   const double rayleigh = 1.2533141373155002512;  // sqrt(pi/2)
   __half h = __double2half(n > 0 ? sum / (double)n / rayleigh : 0.0);
@@ -284,14 +289,11 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
   // table fills: unrolled so that each thread's loads are in flight together
 #pragma unroll 4
   for (int i = threadIdx.x; i < a.K; i += blockDim.x) cbq[i] = codeword_q(a.codebook[i]);
-#pragma unroll 4
-  for (int j = threadIdx.x; j < a.d_in; j += blockDim.x) {
-    const float v = __half2float(a.scale[j]);
-    fT[(j % kE) * C + j / kE] = mask_negative(a.seed, (uint32_t)j) ? -v : v;
-  }
-#pragma unroll 4
-  for (int k = threadIdx.x; k < P; k += blockDim.x)
-    isgT[(k % kQ) * C + k / kQ] = 1.0f / __half2float(a.sigma[k]);
+  const uint64_t seed = a.seed;
+  fill_interleaved<kE>(fT, a.scale, a.d_in, C, [=](int j, float v) {
+    return mask_negative(seed, (uint32_t)j) ? -v : v;
+  });
+  fill_interleaved<kQ>(isgT, a.sigma, P, C, [](int, float v) { return 1.0f / v; });
   PrefilterView pf;
   if (a.prefilter != nullptr) {
     pf = prefilter_view(a.prefilter, a.K);
@@ -499,7 +501,7 @@ cudaError_t calibrate_typed(const T* W, const qamw_matrix& m, const EncodeWorksp
     k_calib_accum<T, 512><<<kCalCtas, threads, smem, stream>>>(
         W, s, ws.rnorm32, ws.cal_rows, ws.n_cal, d_in, m.block, m.mask_seed, RPC, ws.cal_partial);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  k_calib_finish<<<(P + 255) / 256, 256, 0, stream>>>(ws.cal_partial, kCalCtas, ws.n_cal, P,
+  k_calib_finish<<<(P + 15) / 16, 256, 0, stream>>>(ws.cal_partial, kCalCtas, ws.n_cal, P,
                                                       reinterpret_cast<__half*>(m.sigma), st);
   return cudaGetLastError();
 }
@@ -540,7 +542,7 @@ cudaError_t launch_channel_scales(const float* d_act_stat, int d_in, float alpha
                                   int32_t* d_status, cudaStream_t stream) {
   __half* s = reinterpret_cast<__half*>(d_scale);
   if (d_act_stat != nullptr && alpha != 0.0f)
-    k_scales<<<1, 1024, 0, stream>>>(d_act_stat, d_in, alpha, s, d_status);
+    k_scales<<<(d_in + 255) / 256, 256, 0, stream>>>(d_act_stat, d_in, alpha, s, d_status);
   else
     k_fill_half<<<(d_in + 255) / 256, 256, 0, stream>>>(s, d_in, 1.0f);
   return cudaGetLastError();

@@ -26,7 +26,7 @@ namespace {
 
 // ------------------------------------------------------------------ batch 1
 
-constexpr int kGemvStages = 3;
+constexpr int kGemvStages = 4;
 
 struct Gemv1Args {
   const uint8_t* packed;
@@ -66,89 +66,118 @@ __device__ __forceinline__ void dot_pairs(const uint32_t (&w)[BITS], const uint3
       ...);
 }
 
+__host__ __device__ inline size_t gemv1_region0(int K, int copies_log2, int d_in) {
+  const size_t t = (size_t)K * ((size_t)1 << copies_log2) * 4, x = (size_t)d_in * 4;
+  return align16(t > x ? t : x);
+}
+
+__device__ __forceinline__ void issue_tile(const Gemv1Args& a, int tile, unsigned char* dst,
+                                           uint64_t* bar) {
+  const int r0 = tile * a.R, nr = min(a.R, a.d_out - r0);
+  const unsigned bytes = (unsigned)(nr * a.row_bytes);
+  mbar_expect_tx(bar, bytes);
+  bulk_g2s(dst, a.packed + (int64_t)r0 * a.row_bytes, bytes, bar);
+}
+
+// Warps run through the tiles independently: after writing its partial dot
+// products for a tile, each warp bumps the stage's counter; the warp that
+// completes it sums the partials of every row of the tile (fixed order), writes
+// y, and refills the stage with the tile kGemvStages ahead.
 template <int BITS, int MAXT>
 __global__ void __launch_bounds__(MAXT, 1) k_gemv1(const Gemv1Args a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int copies = 1 << a.copies_log2;
-  uint32_t* tab = reinterpret_cast<uint32_t*>(smem);  // [K][copies] fp16x2
-  unsigned char* stage = smem + (size_t)a.K * copies * 4;
+  // region 0: first D x / s per column (d_in floats), then the fp16x2 codebook
+  // table [K][copies]
+  uint32_t* tab = reinterpret_cast<uint32_t*>(smem);
+  unsigned char* stage = smem + gemv1_region0(a.K, a.copies_log2, a.d_in);
   float* partial = reinterpret_cast<float*>(stage + (size_t)kGemvStages * a.stage_bytes);
+  const size_t part_floats = (size_t)a.R * a.S;
   uint64_t* bar = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(partial) +
-                                              align16((size_t)a.R * a.S * 4));
+                                              align16(kGemvStages * part_floats * 4));
+  int* done = reinterpret_cast<int*>(bar + kGemvStages);
+  int* issued = done + kGemvStages;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int C = a.d_in / kE;
+  const int nwarps = a.S * a.k;
 
   if (tid == 0) {
-    for (int s = 0; s < kGemvStages; ++s) mbar_init(&bar[s], 1);
+    for (int s = 0; s < kGemvStages; ++s) {
+      mbar_init(&bar[s], 1);
+      done[s] = 0;
+      issued[s] = 0;
+    }
     fence_mbar_init();
-  }
-  // fp16x2 codebook, `copies` replicas of each entry side by side; each thread
-  // loads its codewords together, then writes their replicas
-#pragma unroll 4
-  for (int j = tid; j < a.K; j += blockDim.x) {
-    const float2 c = a.codebook[j];
-    const __half2 h = __floats2half2_rn(c.x, c.y);
-    const uint32_t u = *reinterpret_cast<const uint32_t*>(&h);
-    for (int r = 0; r < copies; ++r) tab[(j << a.copies_log2) + r] = u;
-  }
-  __syncthreads();
-  // first tiles in flight while xbar is computed
-  if (tid == 0) {
+    // first tiles in flight while xbar and the codebook table are prepared
     for (int s = 0; s < kGemvStages; ++s) {
       const int tile = blockIdx.x + s * gridDim.x;
       if (tile >= a.ntiles) break;
-      const int r0 = tile * a.R, nr = min(a.R, a.d_out - r0);
-      const unsigned bytes = (unsigned)(nr * a.row_bytes);
-      mbar_expect_tx(&bar[s], bytes);
-      bulk_g2s(stage + (size_t)s * a.stage_bytes, a.packed + (int64_t)r0 * a.row_bytes, bytes,
-               &bar[s]);
+      issue_tile(a, tile, stage + (size_t)s * a.stage_bytes, &bar[s]);
+      issued[s] = 1;
     }
   }
+  // D_j x_j / s_j for every column, spread over the whole CTA, chunk-interleaved
+  // in the table area (free until the table is written below)
+  float* xsT = reinterpret_cast<float*>(tab);
+  const __nv_bfloat16* xin = a.x;
+  const uint64_t seed = a.seed;
+  int flags = 0;
+  fill_interleaved<kE>(xsT, a.scale, a.d_in, C, [&](int j, float sv) {
+    const float xv = __bfloat162float(xin[j]);
+    if (!isfinite(xv)) flags = QAMW_STATUS_NONFINITE;
+    const float q = __fdiv_rn(xv, sv);
+    return mask_negative(seed, (uint32_t)j) ? -q : q;
+  });
+  __syncthreads();
 
   // xbar of this lane's chunk c: sigma (.) R_fwd(x / s), in registers
   const int sl = warp % a.S, kk = warp / a.S;
   const int c = sl * 32 + lane;
   const bool active = c < C;
   float xr[kE];
-  int flags = 0;
+  float sg[kQ];
   if (active) {
-    load64(a.x + (int64_t)c * kE, xr);
+    load_halves<kQ>(a.sigma + (int64_t)c * kQ, sg);
 #pragma unroll
-    for (int j = 0; j < kE; ++j) {
-      const int col = c * kE + j;
-      if (!isfinite(xr[j])) flags = QAMW_STATUS_NONFINITE;
-      const float q = __fdiv_rn(xr[j], __half2float(a.scale[col]));
-      xr[j] = mask_negative(a.seed, (uint32_t)col) ? -q : q;
-    }
+    for (int j = 0; j < kE; ++j) xr[j] = xsT[j * C + c];
   } else {
 #pragma unroll
     for (int j = 0; j < kE; ++j) xr[j] = 0.f;
   }
+  __syncthreads();
+  // fp16x2 codebook, `copies` replicas of each entry side by side, written word
+  // by word so that consecutive lanes store consecutive words (no bank
+  // conflicts); the lanes of one entry read the same codeword (one transaction)
+#pragma unroll 8
+  for (int wd = tid; wd < (a.K << a.copies_log2); wd += blockDim.x) {
+    const float2 cw = __ldg(a.codebook + (wd >> a.copies_log2));
+    const __half2 h = __floats2half2_rn(cw.x, cw.y);
+    tab[wd] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  __syncthreads();
   fwht_reg<kE>(xr, min(a.block, kE));
   fwht_lanes<kE>(xr, max(a.block / kE, 1));
   if (active) {
     const float inv_sqrt_b = 1.0f / sqrtf((float)a.block);
 #pragma unroll
     for (int q = 0; q < kQ; ++q) {
-      const float sg = __half2float(a.sigma[c * kQ + q]) * inv_sqrt_b;
-      xr[2 * q] *= sg;
-      xr[2 * q + 1] *= sg;
+      const float f = sg[q] * inv_sqrt_b;
+      xr[2 * q] *= f;
+      xr[2 * q + 1] *= f;
     }
   }
 
-  const uint32_t cmask = (uint32_t)(copies - 1);
+  const uint32_t copy = (uint32_t)lane & (uint32_t)(copies - 1);
   int it = 0;
-  bool timed_out = false;
   for (int tile = blockIdx.x; tile < a.ntiles; tile += gridDim.x, ++it) {
     const int st = it % kGemvStages;
-    const unsigned parity = (unsigned)(it / kGemvStages) & 1u;
-    const bool ok = mbar_wait_bounded(&bar[st], parity);
-    if (__syncthreads_or(!ok)) {
-      timed_out = true;
+    if (!mbar_wait_bounded(&bar[st], (unsigned)(it / kGemvStages) & 1u)) {
+      flags |= QAMW_STATUS_TIMEOUT;
       break;
     }
     const int r0 = tile * a.R, nr = min(a.R, a.d_out - r0);
     const unsigned char* buf = stage + (size_t)st * a.stage_bytes;
+    float* part = partial + st * part_floats;
     for (int rl = kk; rl < nr; rl += a.k) {
       float acc0 = 0.f, acc1 = 0.f;
       if (active) {
@@ -157,51 +186,53 @@ __global__ void __launch_bounds__(MAXT, 1) k_gemv1(const Gemv1Args a) {
         uint32_t w[BITS];
 #pragma unroll
         for (int t = 0; t < BITS; ++t) w[t] = src[t];
-        dot_pairs<BITS>(w, tab, a.copies_log2, (uint32_t)lane & cmask, xr, acc0, acc1,
+        dot_pairs<BITS>(w, tab, a.copies_log2, copy, xr, acc0, acc1,
                         std::make_integer_sequence<int, kQ>{});
       }
       float acc = acc0 + acc1;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) partial[rl * a.S + sl] = acc;
+      if (lane == 0) part[rl * a.S + sl] = acc;
     }
-    __syncthreads();
-    for (int r = tid; r < nr; r += blockDim.x) {
-      float sum = 0.f;
-      for (int s = 0; s < a.S; ++s) sum += partial[r * a.S + s];
-      a.y[r0 + r] = __float2bfloat16_rn(sum * __half2float(a.rnorm[r0 + r]));
+    int last = 0;
+    if (lane == 0) {
+      __threadfence_block();
+      last = atomicAdd(&done[st], 1) == nwarps - 1;
     }
-    if (tid == 0) {
-      const int next = tile + kGemvStages * gridDim.x;
-      if (next < a.ntiles) {
-        const int n0 = next * a.R, nn = min(a.R, a.d_out - n0);
-        const unsigned bytes = (unsigned)(nn * a.row_bytes);
-        mbar_expect_tx(&bar[st], bytes);
-        bulk_g2s(stage + (size_t)st * a.stage_bytes, a.packed + (int64_t)n0 * a.row_bytes, bytes,
-                 &bar[st]);
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) {
+      __threadfence_block();
+      for (int r = lane; r < nr; r += 32) {
+        float sum = 0.f;
+        for (int s = 0; s < a.S; ++s) sum += part[r * a.S + s];
+        a.y[r0 + r] = __float2bfloat16_rn(sum * __half2float(a.rnorm[r0 + r]));
+      }
+      __syncwarp();
+      if (lane == 0) {
+        done[st] = 0;
+        const int next = tile + kGemvStages * gridDim.x;
+        if (next < a.ntiles) {
+          issue_tile(a, next, stage + (size_t)st * a.stage_bytes, &bar[st]);
+          issued[st] += 1;
+        }
       }
     }
-    __syncthreads();
   }
-  if (timed_out) {
-    // let this CTA's copies still in flight land before its shared memory goes away
-    if (tid == 0) {
-      for (int s = 0; s < kGemvStages; ++s) {
-        const int t2 = it + s;
-        const int tile = blockIdx.x + t2 * gridDim.x;
-        if (tile >= a.ntiles) break;
-        mbar_wait_bounded(&bar[t2 % kGemvStages], (unsigned)(t2 / kGemvStages) & 1u);
-      }
-    }
-    flags |= QAMW_STATUS_TIMEOUT;
+  // after a timeout: let the copies still in flight land before this CTA's
+  // shared memory goes away
+  __syncthreads();
+  if (tid == 0) {
+    for (int s = 0; s < kGemvStages; ++s)
+      if (issued[s] > 0) mbar_wait_bounded(&bar[s], (unsigned)(issued[s] - 1) & 1u);
   }
   raise_flag(a.status, flags);
 }
 
 // Shared memory of k_gemv1 for given replicas and tile rows.
-size_t gemv1_smem(int K, int copies_log2, unsigned stage_bytes, int R, int S) {
-  return (size_t)K * ((size_t)1 << copies_log2) * 4 + (size_t)kGemvStages * stage_bytes +
-         align16((size_t)R * S * 4) + kGemvStages * sizeof(uint64_t);
+size_t gemv1_smem(int K, int copies_log2, unsigned stage_bytes, int R, int S, int d_in) {
+  return gemv1_region0(K, copies_log2, d_in) + (size_t)kGemvStages * stage_bytes +
+         align16((size_t)kGemvStages * R * S * 4) + kGemvStages * sizeof(uint64_t) +
+         2 * kGemvStages * sizeof(int);
 }
 
 template <int BITS>
@@ -225,16 +256,16 @@ cudaError_t run_gemv1(const qamw_matrix& m, const uint16_t* d_x, uint16_t* d_y,
   const int C = m.d_in / kE;
   a.S = (C + 31) / 32;
   a.k = a.S <= 8 ? 8 / a.S : 1;
-  // ~24 KB of indices per stage, whole rows, a multiple of k rows
-  int R = (int)(24576 / m.row_bytes);
+  // ~20 KB of indices per stage, whole rows, a multiple of k rows
+  int R = (int)(20480 / m.row_bytes);
   R = R < a.k ? a.k : (R / a.k) * a.k;
   a.R = R;
   a.stage_bytes = (unsigned)(R * m.row_bytes);
   a.ntiles = (m.d_out + R - 1) / R;
   int cl = a.K <= 1024 ? 5 : 4;
-  while (cl > 0 && gemv1_smem(a.K, cl, a.stage_bytes, R, a.S) > 227 * 1024) --cl;
+  while (cl > 0 && gemv1_smem(a.K, cl, a.stage_bytes, R, a.S, a.d_in) > 227 * 1024) --cl;
   a.copies_log2 = cl;
-  const size_t smem = gemv1_smem(a.K, cl, a.stage_bytes, R, a.S);
+  const size_t smem = gemv1_smem(a.K, cl, a.stage_bytes, R, a.S, a.d_in);
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   const int threads = 32 * a.S * a.k;
   // 256-thread bound (up to 255 registers) unless a row needs more than 8 slices
@@ -273,12 +304,14 @@ __global__ void __launch_bounds__(256) k_rotate(const __nv_bfloat16* __restrict_
     const bool real = active && t < batch;
     float xv[kE];
     if (real) {
+      float sc[kE];
       load64(x + t * d_in + (int64_t)c * kE, xv);
+      load_halves<kE>(s + (int64_t)c * kE, sc);
 #pragma unroll
       for (int j = 0; j < kE; ++j) {
         const int col = c * kE + j;
         if (!isfinite(xv[j])) flags = QAMW_STATUS_NONFINITE;
-        const float q = __fdiv_rn(xv[j], __half2float(s[col]));
+        const float q = __fdiv_rn(xv[j], sc[j]);
         xv[j] = mask_negative(seed, (uint32_t)col) ? -q : q;
       }
     } else {
@@ -288,11 +321,13 @@ __global__ void __launch_bounds__(256) k_rotate(const __nv_bfloat16* __restrict_
     fwht_reg<kE>(xv, nb);
     fwht_lanes<kE>(xv, lanes);
     if (active) {
+      float sg[kQ];
+      load_halves<kQ>(sigma + (int64_t)c * kQ, sg);
       float2* dst = xbarT + t * P + c;
 #pragma unroll
       for (int q = 0; q < kQ; ++q) {
-        const float sg = __half2float(sigma[c * kQ + q]) * inv_sqrt_b;
-        dst[(size_t)q * C] = make_float2(xv[2 * q] * sg, xv[2 * q + 1] * sg);
+        const float f = sg[q] * inv_sqrt_b;
+        dst[(size_t)q * C] = make_float2(xv[2 * q] * f, xv[2 * q + 1] * f);
       }
     }
   }

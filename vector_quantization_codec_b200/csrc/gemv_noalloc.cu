@@ -75,6 +75,7 @@ extern "C" QAMW_API int qamw_decode_gemv_noalloc(const qamw_matrix* m, const uin
   if (m->d_out == 0) return QAMW_OK;
   if (!m->packed || !m->row_norm || !m->sigma || !m->chan_scale || !m->codebook) return QAMW_ERR_INVALID;
   if (!aligned16(m->packed) || !aligned16(m->codebook)) return QAMW_ERR_ALIGN;
+  if (!aligned16(m->sigma) || !aligned16(m->chan_scale)) return QAMW_ERR_ALIGN;
   if (!d_x || !d_y) return QAMW_ERR_INVALID;
   if (!aligned16(d_x)) return QAMW_ERR_ALIGN;
   void* scratch = nullptr;

@@ -66,6 +66,24 @@ __global__ void __launch_bounds__(1024) k_pf_header(const float2* __restrict__ c
 constexpr int kBuildWarps = 8;
 constexpr int kMaxCand = 256;
 
+// Slot 0: count (kPfOverflow when the list did not fit); slots 1..m: the m
+// candidates; slots up to 7 repeat the first candidate (scored without a
+// branch by the encoder); the rest zero.  Called by all 32 lanes of a warp.
+__device__ void write_list(void* table, int G, int NS, size_t n, bool overflow, int m,
+                           const uint16_t* keep) {
+  const int lane = threadIdx.x & 31;
+  for (int t = lane; t < kPfSlots; t += 32) {
+    uint16_t v;
+    if (t == 0)
+      v = overflow ? (uint16_t)kPfOverflow : (uint16_t)m;
+    else if (overflow)
+      v = 0;
+    else
+      v = t - 1 < m ? keep[t - 1] : (t < 8 ? keep[0] : (uint16_t)0);
+    *prefilter_slot(table, G, NS, n, t) = v;
+  }
+}
+
 // One warp per cell.
 __global__ void __launch_bounds__(kBuildWarps * 32) k_pf_build(const float2* __restrict__ cb,
                                                                void* __restrict__ table) {
@@ -76,24 +94,27 @@ __global__ void __launch_bounds__(kBuildWarps * 32) k_pf_build(const float2* __r
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int cell = blockIdx.x * kBuildWarps + wib;
   if (cell >= G * G) return;
-  uint16_t* lists = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(table) +
-                                                prefilter_lists_offset());
   const int gx = cell % G, gy = cell / G;
   const double R = hdr.R, h = hdr.h, M = hdr.margin;
   const double eps = ldexp(R, -16);
   const double x0 = -R + gx * h - eps, x1 = -R + (gx + 1) * h + eps;
   const double y0 = -R + gy * h - eps, y1 = -R + (gy + 1) * h + eps;
 
+  // Passes 1-2 run in fp32 over all K codewords, with slack (relative 2^-12,
+  // far above fp32 rounding) that can only add candidates; the pruning of
+  // step 3 is exact (fp64).
+  const float fx0 = (float)x0, fx1 = (float)x1, fy0 = (float)y0, fy1 = (float)y1;
   // 1. D2 = min_j maxdist^2(cell, c_j)
-  double D2 = INFINITY;
+  float D2 = INFINITY;
   for (int j = lane; j < K; j += 32) {
     const float2 c = cb[j];
-    const double dx = fmax(fabs(x0 - c.x), fabs(x1 - c.x));
-    const double dy = fmax(fabs(y0 - c.y), fabs(y1 - c.y));
-    D2 = fmin(D2, dx * dx + dy * dy);
+    const float dx = fmaxf(fabsf(fx0 - c.x), fabsf(fx1 - c.x));
+    const float dy = fmaxf(fabsf(fy0 - c.y), fabsf(fy1 - c.y));
+    D2 = fminf(D2, fmaf(dx, dx, dy * dy));
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) D2 = fmin(D2, __shfl_xor_sync(0xffffffffu, D2, o));
+  for (int o = 16; o > 0; o >>= 1) D2 = fminf(D2, __shfl_xor_sync(0xffffffffu, D2, o));
+  const float bound = D2 * (1.0f + 1.0f / 4096) + 2.0f * (float)M;
 
   // 2. codewords whose distance to the cell can be within D2 (+M), ascending j
   int n = 0;
@@ -103,9 +124,9 @@ __global__ void __launch_bounds__(kBuildWarps * 32) k_pf_build(const float2* __r
     bool ok = false;
     if (j < K) {
       const float2 c = cb[j];
-      const double dx = fmax(fmax(x0 - c.x, c.x - x1), 0.0);
-      const double dy = fmax(fmax(y0 - c.y, c.y - y1), 0.0);
-      ok = dx * dx + dy * dy <= D2 + M;
+      const float dx = fmaxf(fmaxf(fx0 - c.x, c.x - fx1), 0.f);
+      const float dy = fmaxf(fmaxf(fy0 - c.y, c.y - fy1), 0.f);
+      ok = fmaf(dx, dx, dy * dy) <= bound;
     }
     const unsigned bal = __ballot_sync(0xffffffffu, ok);
     const int pos = n + __popc(bal & ((1u << lane) - 1u));
@@ -145,16 +166,7 @@ __global__ void __launch_bounds__(kBuildWarps * 32) k_pf_build(const float2* __r
     }
   }
   __syncwarp();
-  uint16_t* L = lists + (size_t)cell * kPfSlots;
-  if (overflow || m > kPfCap) {
-    if (lane == 0) L[0] = (uint16_t)kPfOverflow;
-    return;
-  }
-  // slot 0: count; slots 1..m: candidates; slots up to 7 repeat the first
-  // candidate (scored without a branch by the encoder); the rest zero
-  if (lane == 0) L[0] = (uint16_t)m;
-  for (int t = lane; t < kPfCap; t += 32)
-    L[1 + t] = t < m ? keep[wib][t] : (t < 7 ? keep[wib][0] : (uint16_t)0);
+  write_list(table, G, hdr.NS, (size_t)cell, overflow || m > kPfCap, m, keep[wib]);
 }
 
 // Warp-wide argmin_j |q - c_j|^2 (any minimiser will do: it only seeds the
@@ -194,6 +206,20 @@ struct SectorGeom {
   double p0x, p0y, p1x, p1y, e0x, e0y, e1x, e1y, M, min_slope;
 };
 
+// Single-precision form of `dominated` with doubled margins and a relative
+// slack on the gaps: it can only answer "dominated" where the exact test would.
+__device__ bool dominated_f(const SectorGeom& g, float2 cj, float2 ck) {
+  const float dx = ck.x - cj.x, dy = ck.y - cj.y;
+  const float ms = 2.0f * (float)g.min_slope;
+  if ((float)g.e0x * dx + (float)g.e0y * dy < ms) return false;
+  if ((float)g.e1x * dx + (float)g.e1y * dy < ms) return false;
+  const float cj2 = cj.x * cj.x + cj.y * cj.y, ck2 = ck.x * ck.x + ck.y * ck.y;
+  const float slack = 2.0f * (float)g.M + 1e-4f * (cj2 + ck2 + 1.0f);
+  const float f0 = 2.0f * ((float)g.p0x * dx + (float)g.p0y * dy) + cj2 - ck2;
+  const float f1 = 2.0f * ((float)g.p1x * dx + (float)g.p1y * dy) + cj2 - ck2;
+  return f0 > slack + 1e-4f * fabsf(f0) && f1 > slack + 1e-4f * fabsf(f1);
+}
+
 __device__ bool dominated(const SectorGeom& g, float2 cj, float2 ck) {
   const double dx = (double)ck.x - cj.x, dy = (double)ck.y - cj.y;
   if (g.e0x * dx + g.e0y * dy < g.min_slope) return false;
@@ -217,9 +243,7 @@ __global__ void __launch_bounds__(kBuildWarps * 32) k_pf_sectors(const float2* _
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int sct = blockIdx.x * kBuildWarps + wib;
   if (sct >= NS) return;
-  uint16_t* L = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(table) +
-                                            prefilter_lists_offset()) +
-                ((size_t)G * G + sct) * kPfSlots;
+  const size_t n_list = (size_t)G * G + sct;
   const double pi = 3.14159265358979323846, eps = 1e-4;
   const double t0 = -pi + 2.0 * pi * sct / NS - eps, t1 = -pi + 2.0 * pi * (sct + 1) / NS + eps;
   const double Rin = (double)hdr.R * (1.0 - 1.0 / 1024);
@@ -252,7 +276,7 @@ __global__ void __launch_bounds__(kBuildWarps * 32) k_pf_sectors(const float2* _
     if (ok) {
       const float2 cj = cb[j];
       for (int r = 0; r < kRefs && ok; ++r)
-        if (refs[r] != j && dominated(g, cj, cb[refs[r]])) ok = false;
+        if (refs[r] != j && dominated_f(g, cj, cb[refs[r]])) ok = false;
     }
     const unsigned bal = __ballot_sync(0xffffffffu, ok);
     const int pos = n + __popc(bal & ((1u << lane) - 1u));
@@ -261,7 +285,7 @@ __global__ void __launch_bounds__(kBuildWarps * 32) k_pf_sectors(const float2* _
   }
   __syncwarp();
   if (n > kMaxCand) {
-    if (lane == 0) L[0] = (uint16_t)kPfOverflow;
+    write_list(table, G, NS, n_list, true, 0, keep[wib]);
     return;
   }
   // 2. candidates not dominated by another candidate
@@ -280,13 +304,7 @@ __global__ void __launch_bounds__(kBuildWarps * 32) k_pf_sectors(const float2* _
     m += __popc(bal);
   }
   __syncwarp();
-  if (m > kPfCap) {
-    if (lane == 0) L[0] = (uint16_t)kPfOverflow;
-    return;
-  }
-  if (lane == 0) L[0] = (uint16_t)m;
-  for (int t = lane; t < kPfCap; t += 32)
-    L[1 + t] = t < m ? keep[wib][t] : (t < 7 ? keep[wib][0] : (uint16_t)0);
+  write_list(table, G, NS, n_list, m > kPfCap, m, keep[wib]);
 }
 
 }  // namespace
