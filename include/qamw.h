@@ -78,6 +78,8 @@ extern "C" {
 
 #define QAMW_SIGMA_GIVEN 0x1  /* encode: use m->sigma as given, skip eq. (1)  */
 #define QAMW_SCALES_GIVEN 0x2 /* encode: use m->chan_scale as given           */
+#define QAMW_POLAR 0x4        /* encode: polar baseline quantiser (section    */
+                              /* 3.5) against a qamw_polar_codebook table     */
 
 #define QAMW_OP_TRAIN 0
 #define QAMW_OP_ENCODE 1
@@ -170,7 +172,7 @@ QAMW_API int qamw_build_prefilter(const float *d_codebook, int bits, void *d_tab
  *              activation RMS), nullable.  s_j = binary16((a_j/mean a)^alpha);
  *              NULL or alpha == 0 gives s_j = 1.  Ignored with
  *              QAMW_SCALES_GIVEN (then m->chan_scale is read).
- *   flags      QAMW_SIGMA_GIVEN | QAMW_SCALES_GIVEN.
+ *   flags      QAMW_SIGMA_GIVEN | QAMW_SCALES_GIVEN | QAMW_POLAR.
  *   m          shape, block, bits, mask_seed, row_bytes and buffers (in);
  *              packed, row_norm, sigma (unless given), chan_scale (unless
  *              given) (out).
@@ -213,6 +215,24 @@ QAMW_API int qamw_calibrate_sigma(const void *d_W, int dtype, const qamw_matrix 
  *   roofline; costs one reduction per CTA).  Flags: NONFINITE, RANGE. */
 QAMW_API int qamw_encode_rows(const void *d_W, int dtype, const qamw_matrix *m,
                               uint64_t *d_candidates, int32_t *d_status, void *stream);
+
+/* Section 3.5, the polar baseline: the amplitude |z_k|/sigma_k is quantised
+ * with an N_a-level Lloyd-Max codebook of the unit Rayleigh density
+ * r exp(-r^2/2) and the phase arg z_k is rounded to one of N_p uniform bins;
+ * B = B_a + B_p bits per pair with B_a = floor(B/2) (5 + 6 for B = 11, 3 + 4 for
+ * B = 7).  qamw_polar_codebook computes the levels (continuous Lloyd-Max in
+ * fp64, 20000 iterations from the equal-probability partition) and writes the
+ * expanded table d_codebook[ia * N_p + ip] = a_ia (cos 2 pi ip/N_p,
+ * sin 2 pi ip/N_p), [2^bits][2] fp32, 16-byte aligned.  That table is an
+ * ordinary codebook for qamw_decode and qamw_decode_gemv. */
+QAMW_API int qamw_polar_codebook(int bits, float *d_codebook, void *stream);
+
+/* qamw_encode_rows with the polar quantiser: amplitude to the nearest level
+ * (lowest index on ties), phase to the nearest bin centre 2 pi ip/N_p; the
+ * levels are read from m->codebook (a qamw_polar_codebook table); m->prefilter
+ * is ignored.  Same as qamw_encode with QAMW_POLAR. */
+QAMW_API int qamw_encode_rows_polar(const void *d_W, int dtype, const qamw_matrix *m,
+                                    int32_t *d_status, void *stream);
 
 /* Section 3.2 decoder: unpack, look up the codeword, rescale pair k by
  * sigma_k, reassemble, apply R_inv = diag(D) blockdiag(H_b) / sqrt(b),

@@ -67,6 +67,10 @@ def _load():
         "ref_decode_rows": (None, [P, I64, I, I, I, U64, P, P, P, P, I, I, P]),
         "ref_gemv": (None, [P, I, I, P, I, I, I, P]),
         "ref_lloyd": (None, [P, I64, I, I, P, P]),
+        "ref_rayleigh_lloyd_max": (None, [I, I, P]),
+        "ref_polar_codebook": (None, [I, P, P]),
+        "ref_polar_index": (I, [D, D, P, I]),
+        "ref_encode_rows_polar": (None, [P, I, I, I, U64, P, P, P, I, I, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -302,3 +306,68 @@ def lloyd(samples: np.ndarray, K: int, iters: int):
     dist = np.empty(max(iters, 1), dtype=np.float64)
     _load().ref_lloyd(_p(s), s.shape[0], K, iters, _p(cb), _p(dist))
     return cb, dist[:iters]
+
+
+# ------------------------------------------------------------- polar baseline
+
+def rayleigh_lloyd_max(N: int, iters: int = 20000) -> np.ndarray:
+    """Section 3.5: N-level Lloyd-Max codebook of the unit Rayleigh density."""
+    lv = np.empty(N, dtype=np.float64)
+    _load().ref_rayleigh_lloyd_max(N, iters, _p(lv))
+    return lv
+
+
+def polar_split(bits: int) -> tuple[int, int]:
+    """(amplitude bits, phase bits) = (floor(B/2), B - floor(B/2))."""
+    return bits // 2, bits - bits // 2
+
+
+def polar_levels(bits: int, iters: int = 20000) -> np.ndarray:
+    return rayleigh_lloyd_max(1 << polar_split(bits)[0], iters)
+
+
+def polar_codebook(bits: int, levels: np.ndarray | None = None) -> np.ndarray:
+    """Expanded K-entry table: entry ia * Np + ip = a_ia (cos 2 pi ip/Np, sin 2 pi ip/Np)."""
+    if levels is None:
+        levels = polar_levels(bits)
+    lv = np.ascontiguousarray(levels, dtype=np.float64)
+    cb = np.empty((1 << bits, 2), dtype=np.float64)
+    _load().ref_polar_codebook(bits, _p(lv), _p(cb))
+    return cb
+
+
+def polar_index(points: np.ndarray, levels: np.ndarray, bits: int) -> np.ndarray:
+    lib = _load()
+    lv = np.ascontiguousarray(levels, dtype=np.float64)
+    pts = np.asarray(points, dtype=np.float64).reshape(-1, 2)
+    return np.array([lib.ref_polar_index(float(x), float(y), _p(lv), bits) for x, y in pts],
+                    dtype=np.int32)
+
+
+def encode_polar(W: np.ndarray, bits: int, block: int, levels: np.ndarray, *, mask_seed: int = 0,
+                 s_half: np.ndarray, sigma_half: np.ndarray, want_points: bool = False,
+                 threads: int | None = None) -> dict:
+    """Encoder of section 3.1 with the polar quantiser of section 3.5 (given s, sigma)."""
+    W = np.ascontiguousarray(W, dtype=np.float64)
+    d_out, d_in = W.shape
+    P = d_in // 2
+    lv = np.ascontiguousarray(levels, dtype=np.float64)
+    s_half = np.ascontiguousarray(s_half, dtype=np.uint16)
+    sigma_half = np.ascontiguousarray(sigma_half, dtype=np.uint16)
+    rnorm = np.zeros(d_out, dtype=np.uint16)
+    idx = np.zeros((d_out, P), dtype=np.int32)
+    pts = np.zeros((d_out, P, 2), dtype=np.float64) if want_points else None
+    lib = _load()
+
+    def run(a, b):
+        lib.ref_encode_rows_polar(_p(W), d_out, d_in, block, mask_seed, _p(s_half),
+                                  _p(sigma_half), _p(lv), bits, a, b, _p(rnorm), _p(idx), _p(pts))
+
+    _parallel_rows(d_out, run, threads)
+    rb = row_bytes(d_in, bits)
+    out = dict(s_half=s_half, sigma_half=sigma_half, rnorm_half=rnorm, idx=idx,
+               packed=pack(idx, bits, rb), row_bytes=rb, bits=bits, block=block,
+               mask_seed=mask_seed, d_in=d_in, d_out=d_out)
+    if want_points:
+        out["points"] = pts
+    return out

@@ -469,3 +469,113 @@ void ref_lloyd(const double *samples, int64_t n, int K, int iters, double *codeb
     free(sy);
     free(cnt);
 }
+
+/* ------------------------------------------------------------------------ */
+/* Section 3.5, polar baseline: the amplitude |z_k|/sigma_k is quantised     */
+/* with an N_a-level Lloyd-Max codebook of the unit Rayleigh density          */
+/* f(r) = r exp(-r^2/2), the phase arg(z_k) is rounded to one of N_p uniform  */
+/* bins, B = B_a + B_p bits per pair.  Readings: B_a = floor(B/2),            */
+/* B_p = B - B_a (5 + 6 for B = 11, as the paper pairs them; 3 + 4 for        */
+/* B = 7); the phase bins are centred on 2 pi i / N_p and a phase is rounded  */
+/* to the nearest centre; index = i_a * N_p + i_p, so that the polar code is  */
+/* an ordinary K-entry table a_i (cos phi, sin phi) for the decoder.          */
+/* ------------------------------------------------------------------------ */
+
+/* Probability mass and first moment of the unit Rayleigh density on [t0, t1)
+ * (t1 = INFINITY allowed):  mass = e^{-t0^2/2} - e^{-t1^2/2};
+ * int r * r e^{-r^2/2} dr = t0 e^{-t0^2/2} - t1 e^{-t1^2/2}
+ *                           + sqrt(pi/2) (erf(t1/sqrt2) - erf(t0/sqrt2)). */
+static void rayleigh_cell(double t0, double t1, double *mass, double *moment)
+{
+    double e0 = exp(-0.5 * t0 * t0);
+    double e1 = isinf(t1) ? 0.0 : exp(-0.5 * t1 * t1);
+    double te1 = isinf(t1) ? 0.0 : t1 * e1;
+    double erf1 = isinf(t1) ? 1.0 : erf(t1 / sqrt(2.0));
+    *mass = e0 - e1;
+    *moment = t0 * e0 - te1 + sqrt(M_PI / 2.0) * (erf1 - erf(t0 / sqrt(2.0)));
+}
+
+/* Lloyd-Max on the continuous density: start from the equal-probability
+ * thresholds t_i = sqrt(-2 ln(1 - i/N)); alternate centroids (conditional
+ * means) and midpoint thresholds for `iters` iterations (20000 reach a fixed
+ * point to 1e-13 for every N <= 32 the codec uses; the paper gives no count). */
+void ref_rayleigh_lloyd_max(int N, int iters, double *levels)
+{
+    double *t = malloc(sizeof(double) * (size_t)(N + 1));
+    for (int i = 0; i <= N; ++i)
+        t[i] = (i == N) ? INFINITY : sqrt(-2.0 * log(1.0 - (double)i / N));
+    for (int it = 0; it < iters; ++it) {
+        for (int i = 0; i < N; ++i) {
+            double m, mom;
+            rayleigh_cell(t[i], t[i + 1], &m, &mom);
+            levels[i] = mom / m;
+        }
+        for (int i = 1; i < N; ++i)
+            t[i] = 0.5 * (levels[i - 1] + levels[i]);
+    }
+    for (int i = 0; i < N; ++i) {
+        double m, mom;
+        rayleigh_cell(t[i], t[i + 1], &m, &mom);
+        levels[i] = mom / m;
+    }
+    free(t);
+}
+
+void ref_polar_codebook(int bits, const double *levels, double *codebook)
+{
+    int ba = bits / 2, Na = 1 << ba, Np = 1 << (bits - ba);
+    for (int ia = 0; ia < Na; ++ia)
+        for (int ip = 0; ip < Np; ++ip) {
+            double phi = 2.0 * M_PI * ip / Np;
+            codebook[2 * (ia * Np + ip)] = levels[ia] * cos(phi);
+            codebook[2 * (ia * Np + ip) + 1] = levels[ia] * sin(phi);
+        }
+}
+
+/* Amplitude: nearest level (ascending, strict '<'); phase: nearest bin centre. */
+int ref_polar_index(double px, double py, const double *levels, int bits)
+{
+    int ba = bits / 2, Na = 1 << ba, Np = 1 << (bits - ba);
+    double r = hypot(px, py);
+    int ia = 0;
+    double bd = INFINITY;
+    for (int i = 0; i < Na; ++i) {
+        double d = fabs(r - levels[i]);
+        if (d < bd) {
+            bd = d;
+            ia = i;
+        }
+    }
+    double u = atan2(py, px) * Np / (2.0 * M_PI);
+    long ip = (long)floor(u + 0.5);
+    ip = ((ip % Np) + Np) % Np;
+    return ia * Np + (int)ip;
+}
+
+/* Encoder rows with the polar quantiser in place of the joint 2D one. */
+void ref_encode_rows_polar(const double *W, int d_out, int d_in, int b, uint64_t mask_seed,
+                           const uint16_t *s_half, const uint16_t *sigma_half,
+                           const double *levels, int bits, int row_begin, int row_end,
+                           uint16_t *rnorm_half, int32_t *idx, double *points_out)
+{
+    (void)d_out;
+    int P = d_in / 2;
+    double *scratch = malloc(sizeof(double) * (size_t)d_in);
+    double *y = malloc(sizeof(double) * (size_t)d_in);
+    for (int i = row_begin; i < row_end; ++i) {
+        double r = row_to_rotated(W + (int64_t)i * d_in, d_in, b, mask_seed, s_half, scratch, y);
+        rnorm_half[i] = ref_double_to_half(r);
+        for (int k = 0; k < P; ++k) {
+            double sg = ref_half_to_double(sigma_half[k]);
+            double px = y[2 * k] / sg, py = y[2 * k + 1] / sg;
+            int64_t o = (int64_t)i * P + k;
+            idx[o] = (r == 0.0) ? 0 : ref_polar_index(px, py, levels, bits);
+            if (points_out) {
+                points_out[2 * o] = px;
+                points_out[2 * o + 1] = py;
+            }
+        }
+    }
+    free(scratch);
+    free(y);
+}

@@ -430,6 +430,26 @@ __device__ __forceinline__ int pf_finish(const PfCursor& cur, float px, float py
   return pf_finish_slow(cur.tail, cnt, m2x, m2y, cbq, K, be, bi, &scored);
 }
 
+// Polar baseline (paper section 3.5): amplitude |p| to the nearest of the Na
+// Lloyd-Max levels (lowest index on ties), phase to the nearest of Np uniform
+// bin centres 2 pi i / Np; index = ia * Np + ip.
+__device__ __forceinline__ int polar_index(float px, float py, const float* lev, int Na, int Np,
+                                           float np_over_2pi) {
+  const float r = sqrtf(fmaf(px, px, py * py));
+  int ia = 0;
+  float bd = INFINITY;
+  for (int i = 0; i < Na; ++i) {
+    const float d = fabsf(r - lev[i]);
+    if (d < bd) {
+      bd = d;
+      ia = i;
+    }
+  }
+  int ip = (int)floorf(fmaf(atan2f(py, px), np_over_2pi, 0.5f));
+  ip = ((ip % Np) + Np) % Np;
+  return ia * Np + ip;
+}
+
 // Nearest codeword through the prefilter (same result as nearest_all).
 __device__ __forceinline__ int nearest_pf(float px, float py, const float4* cbq, int K,
                                           const PrefilterView& pf, unsigned& scored) {

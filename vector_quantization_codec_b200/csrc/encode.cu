@@ -275,7 +275,7 @@ struct EncodeArgs {
 // Steps 1-6 of section 3.1 in one pass over W: scale by s, sum of squares
 // (reduced per row in a fixed order, so r is bitwise reproducible), Hadamard
 // butterflies, division by r sqrt(b) and sigma_k, nearest codeword, packing.
-template <int BITS, typename T>
+template <int BITS, typename T, bool POLAR>
 __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
   extern __shared__ __align__(16) unsigned char smem[];
   float4* cbq = reinterpret_cast<float4*>(smem);
@@ -286,9 +286,16 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
   float* isgT = fT + a.d_in;                        // [q][c]: 1 / sigma of pair 32c + q
   float* part = isgT + P;                           // [blockDim] partial sums of squares
   float* rsum = part + blockDim.x;                  // [R] row norms
-  // table fills: unrolled so that each thread's loads are in flight together
+  // polar: amplitude levels a_i = codeword (i Np).x of the expanded table
+  constexpr int kBa = BITS / 2, kNa = 1 << kBa, kNp = 1 << (BITS - kBa);
+  float* lev = reinterpret_cast<float*>(cbq);
+  if constexpr (POLAR) {
+    for (int i = threadIdx.x; i < kNa; i += blockDim.x) lev[i] = a.codebook[i * kNp].x;
+  } else {
+    // table fills: unrolled so that each thread's loads are in flight together
 #pragma unroll 4
-  for (int i = threadIdx.x; i < a.K; i += blockDim.x) cbq[i] = codeword_q(a.codebook[i]);
+    for (int i = threadIdx.x; i < a.K; i += blockDim.x) cbq[i] = codeword_q(a.codebook[i]);
+  }
   const uint64_t seed = a.seed;
   fill_interleaved<kE>(fT, a.scale, a.d_in, C, [=](int j, float v) {
     return mask_negative(seed, (uint32_t)j) ? -v : v;
@@ -354,26 +361,40 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
     uint32_t w[BITS];
 #pragma unroll
     for (int t = 0; t < BITS; ++t) w[t] = 0u;
-    float is = isgT[c];
-    float px = (x[0] * inv) * is, py = (x[1] * inv) * is;
-    PfCursor cur = pf_locate(px, py, pf);
+    if constexpr (POLAR) {
+      const float np_over_2pi = (float)kNp * 0.159154943f;
 #pragma unroll
-    for (int q = 0; q < kQ; ++q) {
-      float nx = 0.f, ny = 0.f;
-      PfCursor nxt = cur;
-      if (q + 1 < kQ) {
-        const float is1 = isgT[(q + 1) * C + c];
-        nx = (x[2 * q + 2] * inv) * is1;
-        ny = (x[2 * q + 3] * inv) * is1;
-        nxt = pf_locate(nx, ny, pf);
+      for (int q = 0; q < kQ; ++q) {
+        const float is = isgT[q * C + c];
+        const float px = (x[2 * q] * inv) * is, py = (x[2 * q + 1] * inv) * is;
+        const uint32_t id = zero ? 0u : (uint32_t)polar_index(px, py, lev, kNa, kNp, np_over_2pi);
+        scored += kNa;
+        const int bit = q * BITS, wi = bit >> 5, sh = bit & 31;
+        w[wi] |= id << sh;
+        if (sh + BITS > 32) w[wi + 1] |= id >> (32 - sh);
       }
-      const uint32_t id = zero ? 0u : (uint32_t)pf_finish(cur, px, py, cbq, a.K, scored);
-      const int bit = q * BITS, wi = bit >> 5, sh = bit & 31;
-      w[wi] |= id << sh;
-      if (sh + BITS > 32) w[wi + 1] |= id >> (32 - sh);
-      cur = nxt;
-      px = nx;
-      py = ny;
+    } else {
+      float is = isgT[c];
+      float px = (x[0] * inv) * is, py = (x[1] * inv) * is;
+      PfCursor cur = pf_locate(px, py, pf);
+#pragma unroll
+      for (int q = 0; q < kQ; ++q) {
+        float nx = 0.f, ny = 0.f;
+        PfCursor nxt = cur;
+        if (q + 1 < kQ) {
+          const float is1 = isgT[(q + 1) * C + c];
+          nx = (x[2 * q + 2] * inv) * is1;
+          ny = (x[2 * q + 3] * inv) * is1;
+          nxt = pf_locate(nx, ny, pf);
+        }
+        const uint32_t id = zero ? 0u : (uint32_t)pf_finish(cur, px, py, cbq, a.K, scored);
+        const int bit = q * BITS, wi = bit >> 5, sh = bit & 31;
+        w[wi] |= id << sh;
+        if (sh + BITS > 32) w[wi + 1] |= id >> (32 - sh);
+        cur = nxt;
+        px = nx;
+        py = ny;
+      }
     }
     uint32_t* dst = reinterpret_cast<uint32_t*>(a.packed + row * a.row_bytes) + (size_t)c * BITS;
 #pragma unroll
@@ -412,7 +433,7 @@ void encode_shape(int C, int* R_out, int* threads_out) {
   *threads_out = bestT;
 }
 
-template <int BITS, typename T>
+template <int BITS, typename T, bool POLAR>
 cudaError_t run_encode(EncodeArgs<T> a, cudaStream_t stream) {
   const int C = a.d_in / kE;
   int R, threads;
@@ -421,15 +442,15 @@ cudaError_t run_encode(EncodeArgs<T> a, cudaStream_t stream) {
   const size_t smem = (size_t)a.K * sizeof(float4) + (size_t)a.d_in * sizeof(float) +
                       (size_t)(a.d_in / 2) * sizeof(float) + (size_t)threads * sizeof(float) +
                       (size_t)R * sizeof(float);
-  const void* fn = reinterpret_cast<const void*>(&k_encode<BITS, T>);
+  const void* fn = reinterpret_cast<const void*>(&k_encode<BITS, T, POLAR>);
   cudaError_t err = allow_smem(fn, smem);
   if (err != cudaSuccess) return err;
   const int grid = persistent_grid(fn, threads, smem, (a.d_out + R - 1) / R);
-  k_encode<BITS, T><<<grid, threads, smem, stream>>>(a);
+  k_encode<BITS, T, POLAR><<<grid, threads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
-template <typename T>
+template <typename T, bool POLAR>
 cudaError_t encode_rows_typed(const T* W, const qamw_matrix& m, int32_t* st,
                               unsigned long long* cand, cudaStream_t stream) {
   EncodeArgs<T> a;
@@ -450,17 +471,17 @@ cudaError_t encode_rows_typed(const T* W, const qamw_matrix& m, int32_t* st,
   a.rows_per_cta = 1;
   a.seed = m.mask_seed;
   switch (m.bits) {
-    case 1: return run_encode<1, T>(a, stream);
-    case 2: return run_encode<2, T>(a, stream);
-    case 3: return run_encode<3, T>(a, stream);
-    case 4: return run_encode<4, T>(a, stream);
-    case 5: return run_encode<5, T>(a, stream);
-    case 6: return run_encode<6, T>(a, stream);
-    case 7: return run_encode<7, T>(a, stream);
-    case 8: return run_encode<8, T>(a, stream);
-    case 9: return run_encode<9, T>(a, stream);
-    case 10: return run_encode<10, T>(a, stream);
-    case 11: return run_encode<11, T>(a, stream);
+    case 1: return run_encode<1, T, POLAR>(a, stream);
+    case 2: return run_encode<2, T, POLAR>(a, stream);
+    case 3: return run_encode<3, T, POLAR>(a, stream);
+    case 4: return run_encode<4, T, POLAR>(a, stream);
+    case 5: return run_encode<5, T, POLAR>(a, stream);
+    case 6: return run_encode<6, T, POLAR>(a, stream);
+    case 7: return run_encode<7, T, POLAR>(a, stream);
+    case 8: return run_encode<8, T, POLAR>(a, stream);
+    case 9: return run_encode<9, T, POLAR>(a, stream);
+    case 10: return run_encode<10, T, POLAR>(a, stream);
+    case 11: return run_encode<11, T, POLAR>(a, stream);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -506,7 +527,43 @@ cudaError_t calibrate_typed(const T* W, const qamw_matrix& m, const EncodeWorksp
   return cudaGetLastError();
 }
 
+// Section 3.5: Lloyd-Max levels of the unit Rayleigh density on one warp (lane
+// i owns level i, Na <= 32), fp64, from the equal-probability thresholds, then
+// the expanded table c[ia Np + ip] = a_ia (cos 2 pi ip / Np, sin 2 pi ip / Np).
+__global__ void __launch_bounds__(32) k_polar_codebook(int bits, int iters, float2* __restrict__ cb) {
+  const int ba = bits / 2, Na = 1 << ba, Np = 1 << (bits - ba);
+  const int i = threadIdx.x;
+  const double rt2 = 1.4142135623730950488, c = 1.2533141373155002512;  // sqrt 2, sqrt(pi/2)
+  auto lower = [&](int k) { return k == 0 ? 0.0 : sqrt(-2.0 * log(1.0 - (double)k / Na)); };
+  double t0 = lower(i), t1 = i + 1 < Na ? lower(i + 1) : INFINITY;
+  double lv = 0.0;
+  for (int it = 0; it <= iters; ++it) {
+    // centroid of [t0, t1): (t0 e0 - t1 e1 + c (erf(t1/rt2) - erf(t0/rt2))) / (e0 - e1)
+    const double e0 = exp(-0.5 * t0 * t0);
+    const double e1 = isinf(t1) ? 0.0 : exp(-0.5 * t1 * t1);
+    const double te1 = isinf(t1) ? 0.0 : t1 * e1;
+    const double erf1 = isinf(t1) ? 1.0 : erf(t1 / rt2);
+    lv = (t0 * e0 - te1 + c * (erf1 - erf(t0 / rt2))) / (e0 - e1);
+    if (it == iters) break;
+    const double below = __shfl_up_sync(0xffffffffu, lv, 1);
+    const double above = __shfl_down_sync(0xffffffffu, lv, 1);
+    if (i > 0 && i < Na) t0 = 0.5 * (below + lv);
+    if (i + 1 < Na) t1 = 0.5 * (lv + above);
+  }
+  if (i < Na) {
+    for (int ip = 0; ip < Np; ++ip) {
+      const double phi = 6.283185307179586477 * ip / Np;
+      cb[i * Np + ip] = make_float2((float)(lv * cos(phi)), (float)(lv * sin(phi)));
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_polar_codebook(int bits, float* d_codebook, cudaStream_t stream) {
+  k_polar_codebook<<<1, 32, 0, stream>>>(bits, 20000, reinterpret_cast<float2*>(d_codebook));
+  return cudaGetLastError();
+}
 
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -557,12 +614,19 @@ cudaError_t launch_calibrate(const void* d_W, int dtype, const qamw_matrix& m,
 }
 
 cudaError_t launch_encode_rows(const void* d_W, int dtype, const qamw_matrix& m, int32_t* d_status,
-                               unsigned long long* d_candidates, cudaStream_t stream) {
+                               unsigned long long* d_candidates, bool polar, cudaStream_t stream) {
+  if (polar) {
+    if (dtype == QAMW_DTYPE_F32)
+      return encode_rows_typed<float, true>(static_cast<const float*>(d_W), m, d_status,
+                                            d_candidates, stream);
+    return encode_rows_typed<__nv_bfloat16, true>(static_cast<const __nv_bfloat16*>(d_W), m,
+                                                  d_status, d_candidates, stream);
+  }
   if (dtype == QAMW_DTYPE_F32)
-    return encode_rows_typed<float>(static_cast<const float*>(d_W), m, d_status, d_candidates,
-                                    stream);
-  return encode_rows_typed<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(d_W), m, d_status,
-                                          d_candidates, stream);
+    return encode_rows_typed<float, false>(static_cast<const float*>(d_W), m, d_status,
+                                           d_candidates, stream);
+  return encode_rows_typed<__nv_bfloat16, false>(static_cast<const __nv_bfloat16*>(d_W), m,
+                                                 d_status, d_candidates, stream);
 }
 
 cudaError_t launch_encode(const void* d_W, int dtype, const float* d_act_stat, float alpha,
@@ -577,13 +641,14 @@ cudaError_t launch_encode(const void* d_W, int dtype, const float* d_act_stat, f
     err = launch_calibrate(d_W, dtype, m, ws, d_status, stream);
     if (err != cudaSuccess) return err;
   }
+  if (flags & QAMW_POLAR) return launch_encode_rows(d_W, dtype, m, d_status, nullptr, true, stream);
   qamw_matrix mm = m;
   if (mm.prefilter == nullptr) {
     err = launch_build_prefilter(m.codebook, m.bits, ws.prefilter, stream);
     if (err != cudaSuccess) return err;
     mm.prefilter = ws.prefilter;
   }
-  return launch_encode_rows(d_W, dtype, mm, d_status, nullptr, stream);
+  return launch_encode_rows(d_W, dtype, mm, d_status, nullptr, false, stream);
 }
 
 }  // namespace qamw

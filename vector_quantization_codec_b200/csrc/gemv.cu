@@ -145,14 +145,16 @@ __global__ void __launch_bounds__(MAXT, 1) k_gemv1(const Gemv1Args a) {
     for (int j = 0; j < kE; ++j) xr[j] = 0.f;
   }
   __syncthreads();
-  // fp16x2 codebook, `copies` replicas of each entry side by side, written word
-  // by word so that consecutive lanes store consecutive words (no bank
-  // conflicts); the lanes of one entry read the same codeword (one transaction)
-#pragma unroll 8
-  for (int wd = tid; wd < (a.K << a.copies_log2); wd += blockDim.x) {
-    const float2 cw = __ldg(a.codebook + (wd >> a.copies_log2));
+  // fp16x2 codebook, `copies` replicas of each entry side by side: one load per
+  // codeword, then its replicas in a lane-rotated order, (r + lane) mod copies,
+  // so that a warp's stores spread over the banks (at most 2-way conflicts)
+#pragma unroll 4
+  for (int j = tid; j < a.K; j += blockDim.x) {
+    const float2 cw = __ldg(a.codebook + j);
     const __half2 h = __floats2half2_rn(cw.x, cw.y);
-    tab[wd] = *reinterpret_cast<const uint32_t*>(&h);
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(&h);
+    for (int r = 0; r < copies; ++r)
+      tab[(j << a.copies_log2) + ((r + lane) & (copies - 1))] = u;
   }
   __syncthreads();
   fwht_reg<kE>(xr, min(a.block, kE));

@@ -44,7 +44,8 @@ cudaError_t launch_channel_scales(const float* d_act_stat, int d_in, float alpha
 cudaError_t launch_calibrate(const void* d_W, int dtype, const qamw_matrix& m,
                              const EncodeWorkspace& ws, int32_t* d_status, cudaStream_t stream);
 cudaError_t launch_encode_rows(const void* d_W, int dtype, const qamw_matrix& m, int32_t* d_status,
-                               unsigned long long* d_candidates, cudaStream_t stream);
+                               unsigned long long* d_candidates, bool polar, cudaStream_t stream);
+cudaError_t launch_polar_codebook(int bits, float* d_codebook, cudaStream_t stream);
 cudaError_t launch_encode(const void* d_W, int dtype, const float* d_act_stat, float alpha,
                           int flags, const qamw_matrix& m, const EncodeWorkspace& ws,
                           int32_t* d_status, cudaStream_t stream);

@@ -34,6 +34,7 @@ QAMW_DTYPE_F32 = 0
 QAMW_DTYPE_BF16 = 1
 QAMW_SIGMA_GIVEN = 0x1
 QAMW_SCALES_GIVEN = 0x2
+QAMW_POLAR = 0x4
 QAMW_OP_TRAIN = 0
 QAMW_OP_ENCODE = 1
 QAMW_OP_GEMV = 2
@@ -44,7 +45,7 @@ EXPORTS = ("qamw_row_bytes", "qamw_default_block", "qamw_bits_per_weight",
            "qamw_workspace_bytes", "qamw_prefilter_bytes", "qamw_status_string",
            "qamw_train_codebook", "qamw_build_prefilter", "qamw_encode", "qamw_channel_scales",
            "qamw_calibrate_sigma", "qamw_encode_rows", "qamw_decode", "qamw_decode_gemv",
-           "qamw_decode_gemv_noalloc")
+           "qamw_decode_gemv_noalloc", "qamw_polar_codebook", "qamw_encode_rows_polar")
 
 
 class QamwError(RuntimeError):
@@ -82,6 +83,8 @@ def _load() -> C.CDLL:
         "qamw_decode": (I, [C.POINTER(qamw_matrix), V, V, V]),
         "qamw_decode_gemv": (I, [C.POINTER(qamw_matrix), V, I, V, V, SZ, V, V]),
         "qamw_decode_gemv_noalloc": (I, [C.POINTER(qamw_matrix), V, I, V, V, V]),
+        "qamw_polar_codebook": (I, [I, V, V]),
+        "qamw_encode_rows_polar": (I, [V, I, C.POINTER(qamw_matrix), V, V]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -261,6 +264,24 @@ def qamw_encode_rows(W: torch.Tensor, m: EncodedMatrix, status: torch.Tensor | N
     rc = _lib.qamw_encode_rows(_p(W), _dtype_code(W), C.byref(st), _p(candidates), _p(status),
                                _s(stream))
     _check("qamw_encode_rows", rc)
+    return m
+
+
+def qamw_polar_codebook(bits: int, codebook: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """Expanded [2^bits, 2] table of the polar baseline (section 3.5)."""
+    if codebook is None:
+        codebook = torch.empty((1 << bits, 2), dtype=torch.float32, device="cuda")
+    _check("qamw_polar_codebook", _lib.qamw_polar_codebook(bits, _p(codebook), _s(stream)))
+    return codebook
+
+
+def qamw_encode_rows_polar(W: torch.Tensor, m: EncodedMatrix, status: torch.Tensor | None = None,
+                           stream=None) -> EncodedMatrix:
+    """Steps 1-6 of section 3.1 with the polar quantiser of section 3.5."""
+    st = m.struct()
+    rc = _lib.qamw_encode_rows_polar(_p(W), _dtype_code(W), C.byref(st), _p(status), _s(stream))
+    _check("qamw_encode_rows_polar", rc)
     return m
 
 
