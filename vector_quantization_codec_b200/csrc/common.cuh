@@ -257,15 +257,19 @@ struct PrefilterHeader {
   int32_t NS;    // angular sectors for points off the grid (|p| >= R)
 };
 
-// Each cell's list is 32 uint16 slots: slot 0 is the count (kPfOverflow:
-// search exhaustively), slots 1..count the candidate indices in ascending
-// order.  Slots 0-7 of every list (the "head") are stored together in one
-// array of 16-byte entries -- one load fetches the count and the first 7
-// candidates, and a 128-byte line holds 8 neighbouring heads -- and slots
-// 8-31 (the "tail", rarely needed) in a second array.
+// Each cell's (or sector's) list: the count and the candidate indices in
+// ascending order.  It is stored twice:
+//   head (8 bytes, one per list, all heads side by side): bits 0-3 hold
+//     min(count, 15) -- 15 meaning "15 or more, or overflowed: see the tail" --
+//     and bits 4-63 five 12-bit candidate slots; slots past the count repeat
+//     the first candidate.  One 8-byte load resolves almost every point, and
+//     a 128-byte line holds 16 neighbouring heads.
+//   tail (64 bytes): 32 uint16 slots, slot 0 the exact count (kPfOverflow:
+//     search exhaustively), slots 1..count the candidates.
 constexpr int kPfSlots = 32;
-constexpr int kPfCap = kPfSlots - 1;         // candidates per cell
+constexpr int kPfCap = kPfSlots - 1;         // candidates per list
 constexpr uint32_t kPfOverflow = 0xffffu;
+constexpr int kPfHeadSlots = 5;
 
 __host__ __device__ inline int prefilter_grid(int bits) {
   return bits <= 5 ? 0 : (bits <= 7 ? 64 : (bits <= 9 ? 128 : 256));
@@ -284,30 +288,22 @@ __host__ __device__ inline int prefilter_sectors(int bits) {
 }
 
 __host__ __device__ inline size_t prefilter_bytes_for(int bits) {
-  const int G = prefilter_grid(bits);
-  return prefilter_lists_offset() +
-         ((size_t)G * G + prefilter_sectors(bits)) * kPfSlots * sizeof(uint16_t);
+  const size_t n = (size_t)prefilter_grid(bits) * prefilter_grid(bits) + prefilter_sectors(bits);
+  return prefilter_lists_offset() + ((n * 8 + 15) / 16) * 16 + n * kPfSlots * sizeof(uint16_t);
 }
 
-// List n (cells 0..G*G-1, then sectors): head at heads[n], tail at tails[3n..3n+2].
-__host__ __device__ inline size_t prefilter_tails_offset(int bits) {
-  const int G = prefilter_grid(bits);
-  return prefilter_lists_offset() + ((size_t)G * G + prefilter_sectors(bits)) * 16;
-}
-
-__device__ __forceinline__ uint16_t* prefilter_slot(void* table, int G, int NS, size_t n, int t) {
-  uint8_t* base = reinterpret_cast<uint8_t*>(table) + prefilter_lists_offset();
-  if (t < 8) return reinterpret_cast<uint16_t*>(base + n * 16) + t;
-  const size_t nlists = (size_t)G * G + NS;
-  return reinterpret_cast<uint16_t*>(base + nlists * 16 + n * 48) + (t - 8);
+// List n (cells 0..G*G-1, then sectors): head at heads[n] (8 bytes), tail at
+// tails[n] (32 uint16).
+__host__ __device__ inline size_t prefilter_tails_offset(size_t nlists) {
+  return prefilter_lists_offset() + ((nlists * 8 + 15) / 16) * 16;
 }
 
 struct PrefilterView {
   float R, inv_h, Gf;
   int G;  // 0: exhaustive search only
   int NS;
-  const uint4* heads;  // [G*G + NS]
-  const uint4* tails;  // [G*G + NS][3]
+  const uint2* heads;     // [G*G + NS]
+  const uint16_t* tails;  // [G*G + NS][32]
 };
 
 // A table built for another codebook size is ignored (exhaustive search), so a
@@ -320,9 +316,11 @@ __device__ __forceinline__ PrefilterView prefilter_view(const void* table, int K
   v.G = (h->K == K && h->cap == kPfCap && h->NS == kPfSectors) ? h->G : 0;
   v.NS = h->NS;
   v.Gf = (float)v.G;
-  v.heads = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(table) +
+  const size_t nlists = (size_t)h->G * h->G + h->NS;
+  v.heads = reinterpret_cast<const uint2*>(reinterpret_cast<const uint8_t*>(table) +
                                            prefilter_lists_offset());
-  v.tails = v.heads + ((size_t)h->G * h->G + h->NS);
+  v.tails = reinterpret_cast<const uint16_t*>(reinterpret_cast<const uint8_t*>(table) +
+                                              prefilter_tails_offset(nlists));
   return v;
 }
 
@@ -363,14 +361,14 @@ __device__ __forceinline__ void score(float m2x, float m2y, const float4* cbq, u
 // Split form of nearest_pf, so that a caller can fetch the next point's list
 // head while it scores the current point.
 struct PfCursor {
-  const uint4* tail;  // nullptr: exhaustive search
-  uint4 head;
+  const uint16_t* tail;  // nullptr: exhaustive search
+  uint2 head;
 };
 
 __device__ __forceinline__ PfCursor pf_locate(float px, float py, const PrefilterView& pf) {
   PfCursor cur;
   cur.tail = nullptr;
-  cur.head = make_uint4(0u, 0u, 0u, 0u);
+  cur.head = make_uint2(0u, 0u);
   if (pf.G > 0 && isfinite(px) && isfinite(py)) {
     const float gx = (px + pf.R) * pf.inv_h;
     const float gy = (py + pf.R) * pf.inv_h;
@@ -382,52 +380,47 @@ __device__ __forceinline__ PfCursor pf_locate(float px, float py, const Prefilte
       n = (size_t)pf.G * pf.G + min(max((int)t, 0), pf.NS - 1);
     }
     cur.head = __ldg(pf.heads + n);
-    cur.tail = pf.tails + 3 * n;
+    cur.tail = pf.tails + n * kPfSlots;
   }
   return cur;
 }
 
-// Rare paths of pf_finish: lists longer than 7 (tail slots 8..count),
-// overflowed lists and points that are not finite (exhaustive search).  Kept
-// out of line so that the common path stays small.
-static __device__ __noinline__ int pf_finish_slow(const uint4* tail, uint32_t cnt, float m2x,
-                                                  float m2y, const float4* cbq, int K, float be,
-                                                  int bi, unsigned* scored) {
-  if (tail == nullptr || cnt == kPfOverflow) return nearest_all(m2x, m2y, cbq, K, *scored);
-  for (uint32_t g = 1; g * 8 <= cnt; ++g) {
-    const uint4 q = __ldg(tail + (g - 1));
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      if (g * 8 + e > cnt) break;
-      const uint32_t w = e < 2 ? q.x : (e < 4 ? q.y : (e < 6 ? q.z : q.w));
-      score(m2x, m2y, cbq, (e & 1) ? (w >> 16) : (w & 0xffffu), be, bi);
-    }
-  }
+// Rare paths of pf_finish: lists longer than the 5 head slots (tail slots
+// 6..count), overflowed lists and points that are not finite (exhaustive
+// search).  Kept out of line so that the common path stays small.
+static __device__ __noinline__ int pf_finish_slow(const uint16_t* tail, float m2x, float m2y,
+                                                  const float4* cbq, int K, float be, int bi,
+                                                  unsigned* scored) {
+  const uint32_t cnt = tail == nullptr ? kPfOverflow : (uint32_t)__ldg(tail);
+  if (cnt == kPfOverflow) return nearest_all(m2x, m2y, cbq, K, *scored);
+  *scored += cnt - kPfHeadSlots;
+  for (uint32_t t = kPfHeadSlots + 1; t <= cnt; ++t) score(m2x, m2y, cbq, __ldg(tail + t), be, bi);
   return bi;
 }
 
-// Slots 1..7 of every list are filled (unused ones repeat the first
-// candidate, which cannot change a strict-'<' argmin taken in ascending slot
-// order), so the common case scores 7 codewords without branching.
+// The 5 head slots are always filled (unused ones repeat the first candidate,
+// which cannot change a strict-'<' argmin taken in ascending slot order), so
+// the common case scores 5 codewords without branching.
 __device__ __forceinline__ int pf_finish(const PfCursor& cur, float px, float py,
                                          const float4* cbq, int K, unsigned& scored) {
   const float m2x = -2.f * px, m2y = -2.f * py;
-  const uint4 q = cur.head;
-  const uint32_t cnt = q.x & 0xffffu;
+  const uint2 h = cur.head;
+  const uint32_t n5 = h.x & 15u;
   float be = INFINITY;
   int bi = 0;
-  if (cur.tail != nullptr && cnt != kPfOverflow) {
-    scored += cnt;
-    score(m2x, m2y, cbq, q.x >> 16, be, bi);
-    score(m2x, m2y, cbq, q.y & 0xffffu, be, bi);
-    score(m2x, m2y, cbq, q.y >> 16, be, bi);
-    score(m2x, m2y, cbq, q.z & 0xffffu, be, bi);
-    score(m2x, m2y, cbq, q.z >> 16, be, bi);
-    score(m2x, m2y, cbq, q.w & 0xffffu, be, bi);
-    score(m2x, m2y, cbq, q.w >> 16, be, bi);
-    if (cnt < 8) return bi;
+  if (cur.tail != nullptr) {
+    score(m2x, m2y, cbq, (h.x >> 4) & 0xfffu, be, bi);
+    score(m2x, m2y, cbq, (h.x >> 16) & 0xfffu, be, bi);
+    score(m2x, m2y, cbq, (h.x >> 28) | ((h.y & 0xffu) << 4), be, bi);
+    score(m2x, m2y, cbq, (h.y >> 8) & 0xfffu, be, bi);
+    score(m2x, m2y, cbq, h.y >> 20, be, bi);
+    if (n5 <= (uint32_t)kPfHeadSlots) {
+      scored += n5;
+      return bi;
+    }
+    scored += kPfHeadSlots;
   }
-  return pf_finish_slow(cur.tail, cnt, m2x, m2y, cbq, K, be, bi, &scored);
+  return pf_finish_slow(cur.tail, m2x, m2y, cbq, K, be, bi, &scored);
 }
 
 // Polar baseline (paper section 3.5): amplitude |p| to the nearest of the Na

@@ -66,21 +66,27 @@ __global__ void __launch_bounds__(1024) k_pf_header(const float2* __restrict__ c
 constexpr int kBuildWarps = 8;
 constexpr int kMaxCand = 256;
 
-// Slot 0: count (kPfOverflow when the list did not fit); slots 1..m: the m
-// candidates; slots up to 7 repeat the first candidate (scored without a
-// branch by the encoder); the rest zero.  Called by all 32 lanes of a warp.
-__device__ void write_list(void* table, int G, int NS, size_t n, bool overflow, int m,
+// Tail: slot 0 the count (kPfOverflow when the list did not fit), slots 1..m
+// the candidates, the rest zero.  Head: min(count, 15) (15 for overflow) and 5
+// 12-bit slots, unused ones repeating the first candidate (scored without a
+// branch by the encoder).  Called by all 32 lanes of a warp.
+__device__ void write_list(void* table, size_t nlists, size_t n, bool overflow, int m,
                            const uint16_t* keep) {
   const int lane = threadIdx.x & 31;
-  for (int t = lane; t < kPfSlots; t += 32) {
-    uint16_t v;
-    if (t == 0)
-      v = overflow ? (uint16_t)kPfOverflow : (uint16_t)m;
-    else if (overflow)
-      v = 0;
-    else
-      v = t - 1 < m ? keep[t - 1] : (t < 8 ? keep[0] : (uint16_t)0);
-    *prefilter_slot(table, G, NS, n, t) = v;
+  uint16_t* tail = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(table) +
+                                               prefilter_tails_offset(nlists)) +
+                   n * kPfSlots;
+  tail[lane] = lane == 0 ? (overflow ? (uint16_t)kPfOverflow : (uint16_t)m)
+                         : (!overflow && lane - 1 < m ? keep[lane - 1] : (uint16_t)0);
+  if (lane == 0) {
+    unsigned long long h = overflow ? 15ull : (unsigned long long)(m < 15 ? m : 15);
+    const uint32_t first = overflow ? 0u : keep[0];
+    for (int t = 0; t < kPfHeadSlots; ++t) {
+      const uint32_t v = (!overflow && t < m) ? keep[t] : first;
+      h |= (unsigned long long)(v & 0xfffu) << (4 + 12 * t);
+    }
+    *reinterpret_cast<unsigned long long*>(reinterpret_cast<uint8_t*>(table) +
+                                           prefilter_lists_offset() + n * 8) = h;
   }
 }
 
@@ -166,7 +172,7 @@ __global__ void __launch_bounds__(kBuildWarps * 32) k_pf_build(const float2* __r
     }
   }
   __syncwarp();
-  write_list(table, G, hdr.NS, (size_t)cell, overflow || m > kPfCap, m, keep[wib]);
+  write_list(table, (size_t)G * G + hdr.NS, (size_t)cell, overflow || m > kPfCap, m, keep[wib]);
 }
 
 // Warp-wide argmin_j |q - c_j|^2 (any minimiser will do: it only seeds the
@@ -285,7 +291,7 @@ __global__ void __launch_bounds__(kBuildWarps * 32) k_pf_sectors(const float2* _
   }
   __syncwarp();
   if (n > kMaxCand) {
-    write_list(table, G, NS, n_list, true, 0, keep[wib]);
+    write_list(table, (size_t)G * G + NS, n_list, true, 0, keep[wib]);
     return;
   }
   // 2. candidates not dominated by another candidate
@@ -304,7 +310,7 @@ __global__ void __launch_bounds__(kBuildWarps * 32) k_pf_sectors(const float2* _
     m += __popc(bal);
   }
   __syncwarp();
-  write_list(table, G, NS, n_list, m > kPfCap, m, keep[wib]);
+  write_list(table, (size_t)G * G + NS, n_list, m > kPfCap, m, keep[wib]);
 }
 
 }  // namespace
