@@ -353,3 +353,23 @@ def test_far_points_use_exact_sector_lists(bits):
                   enc["points"], cb)
     pairs = d_out * d_in // 2
     assert cand.item() < 40 * pairs
+
+
+def test_calibration_rows_past_the_first_scan():
+    # Rows 0..2047 hold only 80 non-zero rows, so the first 1024 non-zero rows
+    # of eq. (1) reach past the rows whose norms are computed up front.
+    d_out, d_in, block, bits = 3000, 256, 64, 6
+    W = synth.student_t_weights(d_out, d_in, seed=12)
+    keep = np.zeros(d_out, dtype=bool)
+    keep[np.random.default_rng(0).choice(2048, 80, replace=False)] = True
+    keep[2048:] = True
+    keep[2100:2110] = False
+    W[~keep] = 0.0
+    cb = codebook(bits)
+    m, status = gpu_encode(torch.from_numpy(W).to(DEV), d_in, block, bits, cb)
+    assert status == 0
+    sig_o = oracle.calibrate_sigma(W.astype(np.float64), block, halves(m.chan_scale))
+    assert ulp_diff(halves(m.sigma), sig_o).max() <= 1
+    # and rows of only zeros anywhere: all calibration rows zero -> sigma = 1
+    m0, _ = gpu_encode(torch.zeros((5, d_in), device=DEV), d_in, block, bits, cb)
+    assert np.all(halves(m0.sigma) == 0x3C00)

@@ -3,13 +3,10 @@
 //
 // Kernels, in stream order:
 //   k_scales        s_j = binary16((a_j / mean a)^alpha)          (thread/channel)
-//   k_rownorm       r_i = ||w_i * s||_2 (fp32), r_hat = binary16(r) (warp/row)
-//   k_calib_select  the first min(1024, #non-zero) non-zero rows   (1 CTA)
-//   k_calib_accum   per-CTA sums of |z_k| over those rows           (128 CTAs)
-//   k_calib_finish  sigma_k = binary16(sum / (n sqrt(pi/2)))        (thread/pair)
-//   k_encode        rotate, normalise, nearest codeword, pack        (thread/chunk)
-// W is read twice from HBM-sized storage (norms, then encode); per matrix both
-// passes fit in L2 for the matrix sizes of LLM layers.
+//   k_calib_rows    |z_k| sums of the first 1024 rows, per CTA       (128 CTAs)
+//   k_calib_ext     later rows when those held zero rows             (1 CTA)
+//   k_calib_finish  sigma_k = binary16(sum / (n sqrt(pi/2)))        (16 threads/pair)
+//   k_encode        norm, rotate, normalise, nearest codeword, pack  (row groups)
 #include "common.cuh"
 #include "launch.cuh"
 
@@ -102,138 +99,194 @@ __device__ __forceinline__ void load_half8(const __half* p, float (&x)[8]) {
   }
 }
 
-// fp32 row norms of W*s, used to pick and normalise the calibration rows.
-template <typename T>
-__global__ void __launch_bounds__(256) k_rownorm(const T* __restrict__ W,
-                                                 const __half* __restrict__ s, int d_out,
-                                                 int d_in, float* __restrict__ r32,
-                                                 int32_t* status) {
-  const int lane = threadIdx.x & 31;
-  const int warps = (gridDim.x * blockDim.x) >> 5;
-  int flags = 0;
-  for (int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < d_out; row += warps) {
-    const T* w = W + (int64_t)row * d_in;
-    float ss = 0.f;
-    int nonfinite = 0;
-    for (int j = lane * 8; j < d_in; j += 256) {
-      float x[8], sv[8];
-      Vec8<T>::load(w + j, x);
-      load_half8(s + j, sv);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if (!isfinite(x[e])) nonfinite = 1;
-        const float t = x[e] * sv[e];
-        ss = fmaf(t, t, ss);
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    nonfinite = __any_sync(0xffffffffu, nonfinite);
-    if (lane == 0) {
-      const float r = sqrtf(ss);
-      r32[row] = r;
-      if (nonfinite || !isfinite(r)) flags |= QAMW_STATUS_NONFINITE;
-    }
-  }
-  raise_flag(status, flags);
-}
-
 // ------------------------------------------------------------- calibration
 
-__global__ void __launch_bounds__(1024) k_calib_select(const float* __restrict__ r32, int d_out,
-                                                       int32_t* __restrict__ cal_rows,
-                                                       int32_t* __restrict__ n_cal) {
-  __shared__ int scan[1024];
-  const int t = threadIdx.x, T = blockDim.x;
-  const int per = (d_out + T - 1) / T;
-  const int lo = min(t * per, d_out), hi = min(lo + per, d_out);
-  int cnt = 0;
-  for (int i = lo; i < hi; ++i) cnt += (r32[i] > 0.f);
-  scan[t] = cnt;
-  __syncthreads();
-  for (int off = 1; off < T; off <<= 1) {  // inclusive Hillis-Steele scan
-    const int v = t >= off ? scan[t - off] : 0;
-    __syncthreads();
-    scan[t] += v;
-    __syncthreads();
-  }
-  int rank = scan[t] - cnt;
-  for (int i = lo; i < hi && rank < kCalRows; ++i)
-    if (r32[i] > 0.f) cal_rows[rank++] = i;
-  if (t == T - 1) *n_cal = min(scan[T - 1], kCalRows);
-}
-
-// CTA b owns calibration ranks [8b, 8b + 8) and processes RPC of those rows at
-// once (thread (g, c): chunk c of row g of the batch), accumulating |z_k| in
-// registers; the RPC row groups are then summed in a fixed order through a
-// transposed shared buffer into partial[b][k].
+// Eq. (1) over the first min(1024, #non-zero) non-zero rows, in three launches:
+//   k_calib_rows   CTA b takes rows [8b, 8b + 8) of the first 1024: row norm
+//                  (fixed-order reduction), rotation, |z_k| / r summed over
+//                  its non-zero rows into partial[b][k]; nonzero[b] = count.
+//   k_calib_ext    if the first 1024 rows held zero rows, one CTA walks on
+//                  from row 1024 in order, adding the next non-zero rows into
+//                  ext[k] until there are 1024 (a path only matrices with zero
+//                  rows take); else it only records the count.
+//   k_calib_finish sigma_k = binary16((sum_b partial[b][k] + ext[k]) /
+//                  (n sqrt(pi/2))), 1 when that rounds to 0.
+// Thread (g, c) holds chunk c of row group g; RPC row groups run at once.
 template <typename T, int MAXT>
-__global__ void __launch_bounds__(MAXT) k_calib_accum(const T* __restrict__ W,
-                                                      const __half* __restrict__ s,
-                                                      const float* __restrict__ r32,
-                                                      const int32_t* __restrict__ cal_rows,
-                                                      const int32_t* __restrict__ n_cal_p,
-                                                      int d_in, int block, uint64_t seed, int RPC,
-                                                      float* __restrict__ partial) {
+__global__ void __launch_bounds__(MAXT) k_calib_rows(const T* __restrict__ W,
+                                                     const __half* __restrict__ s, int d_out,
+                                                     int d_in, int block, uint64_t seed, int RPC,
+                                                     float* __restrict__ partial,
+                                                     int32_t* __restrict__ nonzero,
+                                                     int32_t* status) {
   extern __shared__ __align__(16) float sm[];
   const int C = d_in / kE, P = d_in / 2;
-  float* fT = sm;            // [j][c]: D * s of column 64c + j
-  float* red = sm + d_in;    // [g][q][c]
+  float* fT = sm;                     // [j][c]: D * s of column 64c + j
+  float* red = sm + d_in;             // [g][q][c]
+  float* part = red + (size_t)RPC * P;  // [blockDim] partial sums of squares
+  float* rsum = part + blockDim.x;     // [RPC]
   fill_interleaved<kE>(fT, s, d_in, C, [=](int j, float v) {
     return mask_negative(seed, (uint32_t)j) ? -v : v;
   });
   __syncthreads();
   const int g = threadIdx.x / C, c = threadIdx.x - g * C;
   const bool lane_ok = g < RPC;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int nb = min(block, kE), lanes = max(block / kE, 1);
   const float inv_sqrt_b = 1.0f / sqrtf((float)block);
-  const int n_cal = *n_cal_p;
-  const int per = (kCalRows + gridDim.x - 1) / gridDim.x;
-  const int t0 = blockIdx.x * per, t1 = min(t0 + per, n_cal);
+  const int rows = min(d_out, kCalRows);
+  const int per = kCalRows / gridDim.x;
+  const int t0 = blockIdx.x * per, t1 = min(t0 + per, rows);
   float acc[kQ];
 #pragma unroll
   for (int q = 0; q < kQ; ++q) acc[q] = 0.f;
+  int nz = 0, flags = 0;
   for (int base = t0; base < t1; base += RPC) {
-    const int t = base + g;
-    const bool active = lane_ok && t < t1;
-    const int row = active ? cal_rows[t] : 0;
+    const int row = base + g;
+    const bool active = lane_ok && row < t1;
     float x[kE];
+    float ss = 0.f;
     if (active) {
       load64(W + (int64_t)row * d_in + (int64_t)c * kE, x);
 #pragma unroll
-      for (int j = 0; j < kE; ++j) x[j] *= fT[j * C + c];
+      for (int j = 0; j < kE; ++j) {
+        x[j] *= fT[j * C + c];
+        ss = fmaf(x[j], x[j], ss);
+      }
     } else {
 #pragma unroll
       for (int j = 0; j < kE; ++j) x[j] = 0.f;
     }
+    part[threadIdx.x] = ss;
     fwht_reg<kE>(x, nb);
     fwht_lanes<kE>(x, lanes);
-    if (active) {
-      const float inv = inv_sqrt_b / r32[row];
+    __syncthreads();
+    for (int q = warp; q < RPC; q += nwarps) {
+      float t = 0.f;
+      for (int k = lane; k < C; k += 32) t += part[q * C + k];
 #pragma unroll
-      for (int q = 0; q < kQ; ++q) {
-        const float zx = x[2 * q] * inv, zy = x[2 * q + 1] * inv;
-        acc[q] += sqrtf(fmaf(zx, zx, zy * zy));
+      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      if (lane == 0) rsum[q] = sqrtf(t);
+    }
+    __syncthreads();
+    if (active) {
+      const float r = rsum[g];
+      if (!isfinite(r)) flags = QAMW_STATUS_NONFINITE;
+      if (r > 0.f) {
+        if (c == 0) ++nz;
+        const float inv = inv_sqrt_b / r;
+#pragma unroll
+        for (int q = 0; q < kQ; ++q) {
+          const float zx = x[2 * q] * inv, zy = x[2 * q + 1] * inv;
+          acc[q] += sqrtf(fmaf(zx, zx, zy * zy));
+        }
       }
     }
+    __syncthreads();  // part / rsum are rewritten by the next batch
   }
   if (lane_ok) {
 #pragma unroll
     for (int q = 0; q < kQ; ++q) red[(size_t)g * P + q * C + c] = acc[q];
   }
+  // non-zero rows of this CTA: thread (g, 0) counted those of group g
+  __shared__ int cnt_sh;
+  if (threadIdx.x == 0) cnt_sh = 0;
   __syncthreads();
+  if (nz) atomicAdd(&cnt_sh, nz);
   for (int k = threadIdx.x; k < P; k += blockDim.x) {
     float v = 0.f;
     for (int gg = 0; gg < RPC; ++gg) v += red[(size_t)gg * P + (k % kQ) * C + k / kQ];
     partial[(size_t)blockIdx.x * P + k] = v;
   }
+  __syncthreads();
+  if (threadIdx.x == 0) nonzero[blockIdx.x] = cnt_sh;
+  raise_flag(status, flags);
+}
+
+// One CTA of at least C threads; thread c < C holds chunk c of the current row.
+template <typename T>
+__global__ void __launch_bounds__(512) k_calib_ext(const T* __restrict__ W,
+                                                   const __half* __restrict__ s, int d_out,
+                                                   int d_in, int block, uint64_t seed,
+                                                   const int32_t* __restrict__ nonzero, int nparts,
+                                                   float* __restrict__ ext,
+                                                   int32_t* __restrict__ n_cal) {
+  extern __shared__ __align__(16) float fT[];  // [j][c]
+  __shared__ float part[512];
+  __shared__ float rtot;
+  __shared__ int total;
+  const int C = d_in / kE;
+  const int c = threadIdx.x;
+  const bool active_c = c < C;
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int b = 0; b < nparts; ++b) n += nonzero[b];
+    total = n;
+  }
+  float acc[kQ];
+#pragma unroll
+  for (int q = 0; q < kQ; ++q) acc[q] = 0.f;
+  __syncthreads();
+  if (total < kCalRows && d_out > kCalRows) {
+    fill_interleaved<kE>(fT, s, d_in, C, [=](int j, float v) {
+      return mask_negative(seed, (uint32_t)j) ? -v : v;
+    });
+    __syncthreads();
+    const int nb = min(block, kE), lanes = max(block / kE, 1);
+    const float inv_sqrt_b = 1.0f / sqrtf((float)block);
+    for (int row = kCalRows; row < d_out && total < kCalRows; ++row) {
+      float x[kE];
+      float ss = 0.f;
+      if (active_c) {
+        load64(W + (int64_t)row * d_in + (int64_t)c * kE, x);
+#pragma unroll
+        for (int j = 0; j < kE; ++j) {
+          x[j] *= fT[j * C + c];
+          ss = fmaf(x[j], x[j], ss);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < kE; ++j) x[j] = 0.f;
+      }
+      part[threadIdx.x] = ss;
+      fwht_reg<kE>(x, nb);
+      fwht_lanes<kE>(x, lanes);
+      __syncthreads();
+      if (threadIdx.x < 32) {
+        float t = 0.f;
+        for (int k = threadIdx.x; k < C; k += 32) t += part[k];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        if (threadIdx.x == 0) rtot = sqrtf(t);
+      }
+      __syncthreads();
+      const float r = rtot;
+      if (r > 0.f && active_c) {
+        const float inv = inv_sqrt_b / r;
+#pragma unroll
+        for (int q = 0; q < kQ; ++q) {
+          const float zx = x[2 * q] * inv, zy = x[2 * q + 1] * inv;
+          acc[q] += sqrtf(fmaf(zx, zx, zy * zy));
+        }
+      }
+      __syncthreads();
+      if (threadIdx.x == 0 && r > 0.f) ++total;
+      __syncthreads();
+    }
+  }
+  if (active_c) {
+#pragma unroll
+    for (int q = 0; q < kQ; ++q) ext[c * kQ + q] = acc[q];
+  }
+  if (threadIdx.x == 0) *n_cal = min(total, kCalRows);
 }
 
 // 16 threads per pair k: thread i sums partials i, i+16, ... in fp64, then the
 // 16 sums are combined by a fixed shuffle tree (deterministic).
 __global__ void __launch_bounds__(256) k_calib_finish(const float* __restrict__ partial,
-                                                      int nparts, const int32_t* __restrict__ n_cal_p,
-                                                      int P, __half* __restrict__ sigma,
+                                                      int nparts, const float* __restrict__ ext,
+                                                      const int32_t* __restrict__ n_cal_p, int P,
+                                                      __half* __restrict__ sigma,
                                                       int32_t* status) {
   const int g = blockIdx.x * (blockDim.x / 16) + threadIdx.x / 16, i = threadIdx.x & 15;
   const int k = min(g, P - 1);
@@ -243,6 +296,7 @@ __global__ void __launch_bounds__(256) k_calib_finish(const float* __restrict__ 
 #pragma unroll
   for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   if (i != 0 || g >= P) return;
+  sum += (double)ext[k];
   const int n = *n_cal_p;
   const double rayleigh = 1.2533141373155002512;  // sqrt(pi/2)
   __half h = __double2half(n > 0 ? sum / (double)n / rayleigh : 0.0);
@@ -490,40 +544,47 @@ template <typename T>
 cudaError_t calibrate_typed(const T* W, const qamw_matrix& m, const EncodeWorkspace& ws,
                             int32_t* st, cudaStream_t stream) {
   const int d_out = m.d_out, d_in = m.d_in, P = d_in / 2;
+  const int C = d_in / kE;
   const __half* s = reinterpret_cast<const __half*>(m.chan_scale);
   cudaError_t err;
-  {
-    const int threads = 256;
-    const void* fn = reinterpret_cast<const void*>(&k_rownorm<T>);
-    const int grid = persistent_grid(fn, threads, 0, ((int64_t)d_out * 32 + threads - 1) / threads);
-    k_rownorm<T><<<grid, threads, 0, stream>>>(W, s, d_out, d_in, ws.rnorm32, st);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  }
-  k_calib_select<<<1, 1024, 0, stream>>>(ws.rnorm32, d_out, ws.cal_rows, ws.n_cal);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  const int C = d_in / kE;
-  // rows per batch: at most the 8 rows a CTA owns, 256 threads, ~200 KB of shared memory
-  // rows per batch: at most the 8 rows a CTA owns, 256 threads (512 when one
-  // row has more than 256 chunks), ~200 KB of shared memory
+  // rows per batch: at most the 8 rows a CTA owns; 256 threads (512 when one
+  // row has more than 256 chunks); ~200 KB of shared memory
   const int maxt = C > 256 ? 512 : 256;
-  int RPC = 8;
+  auto smem_for = [&](int rpc) {
+    const size_t threads = ((size_t)rpc * C + 31) / 32 * 32;
+    return (size_t)d_in * sizeof(float) + (size_t)rpc * P * sizeof(float) +
+           threads * sizeof(float) + (size_t)rpc * sizeof(float);
+  };
+  int RPC = kCalRows / kCalCtas;
   if (RPC * C > maxt) RPC = maxt / C;
-  while (RPC > 1 && (size_t)d_in * 4 * (1 + RPC / 2) > 200 * 1024) --RPC;
   if (RPC < 1) RPC = 1;
+  while (RPC > 1 && smem_for(RPC) > 200 * 1024) --RPC;
   const int threads = ((RPC * C + 31) / 32) * 32;
-  const size_t smem = (size_t)d_in * sizeof(float) + (size_t)RPC * P * sizeof(float);
-  const void* fn = maxt == 256 ? reinterpret_cast<const void*>(&k_calib_accum<T, 256>)
-                               : reinterpret_cast<const void*>(&k_calib_accum<T, 512>);
+  const size_t smem = smem_for(RPC);
+  const void* fn = maxt == 256 ? reinterpret_cast<const void*>(&k_calib_rows<T, 256>)
+                               : reinterpret_cast<const void*>(&k_calib_rows<T, 512>);
   if ((err = allow_smem(fn, smem)) != cudaSuccess) return err;
   if (maxt == 256)
-    k_calib_accum<T, 256><<<kCalCtas, threads, smem, stream>>>(
-        W, s, ws.rnorm32, ws.cal_rows, ws.n_cal, d_in, m.block, m.mask_seed, RPC, ws.cal_partial);
+    k_calib_rows<T, 256><<<kCalCtas, threads, smem, stream>>>(W, s, d_out, d_in, m.block,
+                                                              m.mask_seed, RPC, ws.cal_partial,
+                                                              ws.cal_nonzero, st);
   else
-    k_calib_accum<T, 512><<<kCalCtas, threads, smem, stream>>>(
-        W, s, ws.rnorm32, ws.cal_rows, ws.n_cal, d_in, m.block, m.mask_seed, RPC, ws.cal_partial);
+    k_calib_rows<T, 512><<<kCalCtas, threads, smem, stream>>>(W, s, d_out, d_in, m.block,
+                                                              m.mask_seed, RPC, ws.cal_partial,
+                                                              ws.cal_nonzero, st);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  k_calib_finish<<<(P + 15) / 16, 256, 0, stream>>>(ws.cal_partial, kCalCtas, ws.n_cal, P,
-                                                      reinterpret_cast<__half*>(m.sigma), st);
+  {
+    const int et = ((C + 31) / 32) * 32;
+    const size_t esmem = (size_t)d_in * sizeof(float);
+    const void* efn = reinterpret_cast<const void*>(&k_calib_ext<T>);
+    if ((err = allow_smem(efn, esmem)) != cudaSuccess) return err;
+    k_calib_ext<T><<<1, et, esmem, stream>>>(W, s, d_out, d_in, m.block, m.mask_seed,
+                                             ws.cal_nonzero, kCalCtas, ws.cal_ext, ws.n_cal);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  k_calib_finish<<<(P + 15) / 16, 256, 0, stream>>>(ws.cal_partial, kCalCtas, ws.cal_ext,
+                                                    ws.n_cal, P,
+                                                    reinterpret_cast<__half*>(m.sigma), st);
   return cudaGetLastError();
 }
 
@@ -568,21 +629,22 @@ cudaError_t launch_polar_codebook(int bits, float* d_codebook, cudaStream_t stre
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 size_t calibrate_workspace_bytes(int d_out, int d_in, EncodeWorkspace* carve, void* base) {
+  (void)d_out;
   const size_t P = (size_t)d_in / 2;
   size_t off = 0;
-  const size_t o_r = off;
-  off += align256((size_t)d_out * sizeof(float));
-  const size_t o_rows = off;
-  off += align256(kCalRows * sizeof(int32_t));
+  const size_t o_nz = off;
+  off += align256(kCalCtas * sizeof(int32_t));
   const size_t o_n = off;
   off += align256(sizeof(int32_t));
+  const size_t o_ext = off;
+  off += align256(P * sizeof(float));
   const size_t o_part = off;
   off += align256((size_t)kCalCtas * P * sizeof(float));
   if (carve) {
     char* b = static_cast<char*>(base);
-    carve->rnorm32 = reinterpret_cast<float*>(b + o_r);
-    carve->cal_rows = reinterpret_cast<int32_t*>(b + o_rows);
+    carve->cal_nonzero = reinterpret_cast<int32_t*>(b + o_nz);
     carve->n_cal = reinterpret_cast<int32_t*>(b + o_n);
+    carve->cal_ext = reinterpret_cast<float*>(b + o_ext);
     carve->cal_partial = reinterpret_cast<float*>(b + o_part);
     carve->prefilter = nullptr;
   }

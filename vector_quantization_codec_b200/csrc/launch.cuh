@@ -23,11 +23,11 @@ cudaError_t allow_smem(const void* kernel, size_t smem);
 
 // Workspace carve-up of qamw_encode.
 struct EncodeWorkspace {
-  float* rnorm32;       // [d_out] fp32 row norms of W*s
-  int32_t* cal_rows;    // [1024] rows used by eq. (1)
-  int32_t* n_cal;       // [1]
-  float* cal_partial;   // [kCalCtas][P] partial sums of |z_k|
-  void* prefilter;      // prefilter table (when the matrix carries none)
+  int32_t* cal_nonzero;  // [kCalCtas] non-zero rows each CTA found among rows 0..1023
+  int32_t* n_cal;        // [1] rows used by eq. (1)
+  float* cal_ext;        // [P] |z_k| sums of rows past 1023 (zero rows present)
+  float* cal_partial;    // [kCalCtas][P] partial sums of |z_k|
+  void* prefilter;       // prefilter table (when the matrix carries none)
 };
 constexpr int kCalRows = 1024;
 constexpr int kCalCtas = 128;
