@@ -168,7 +168,7 @@ double qamw_bits_per_weight(int d_in, int bits) {
 
 size_t qamw_prefilter_bytes(int bits) {
   if (bits < 1 || bits > 11) return 0;
-  return prefilter_bytes_for(bits);
+  return prefilter_bytes_for(prefilter_grid(bits));
 }
 
 size_t qamw_workspace_bytes(int op, int d_out, int d_in, int bits, int batch) {
@@ -223,8 +223,8 @@ int qamw_build_prefilter(const float* d_codebook, int bits, void* d_table, size_
                          void* stream) {
   if (bits < 1 || bits > 11 || !d_codebook || !d_table) return QAMW_ERR_INVALID;
   if (!aligned16(d_codebook) || !aligned16(d_table)) return QAMW_ERR_ALIGN;
-  if (table_bytes < prefilter_bytes_for(bits)) return QAMW_ERR_WORKSPACE;
-  return cuda_rc(launch_build_prefilter(d_codebook, bits, d_table,
+  if (table_bytes < prefilter_bytes_for(prefilter_grid(bits))) return QAMW_ERR_WORKSPACE;
+  return cuda_rc(launch_build_prefilter(d_codebook, bits, prefilter_grid(bits), d_table,
                                         static_cast<cudaStream_t>(stream)));
 }
 

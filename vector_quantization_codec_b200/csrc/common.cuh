@@ -73,11 +73,13 @@ template <int N>
 __device__ __forceinline__ void fwht_lanes(float (&v)[N], int lanes) {
   const unsigned lane = threadIdx.x & 31u;
   for (int s = 1; s < lanes; s <<= 1) {
-    const bool upper = (lane & (unsigned)s) != 0;
+    // lower lane: v + o; upper lane: o - v -- one fma with a +-1 factor, the
+    // same single rounding as the add or subtract
+    const float sg = (lane & (unsigned)s) ? -1.f : 1.f;
 #pragma unroll
     for (int j = 0; j < N; ++j) {
       const float o = __shfl_xor_sync(0xffffffffu, v[j], s);
-      v[j] = upper ? (o - v[j]) : (v[j] + o);
+      v[j] = fmaf(sg, v[j], o);
     }
   }
 }
@@ -188,6 +190,25 @@ __device__ __forceinline__ void fill_interleaved(float* dst, const __half* src, 
   }
 }
 
+// The same table as fill_interleaved in groups of four: element j of chunk c
+// (c = j / PERIOD, i = j % PERIOD) at float4 slot (i / 4) * C + c, component
+// i % 4, so that one 16-byte shared load gives a thread four consecutive
+// entries of its chunk and the 32 lanes of a warp read 512 consecutive bytes.
+// Consecutive threads fill consecutive slots.
+template <int PERIOD, typename F>
+__device__ __forceinline__ void fill_quads(float4* dst, const __half* src, int n, int C, F f) {
+  const int slots = n / 4;
+#pragma unroll 2
+  for (int t = threadIdx.x; t < slots; t += blockDim.x) {
+    const int i4 = t / C, c = t - i4 * C;
+    const int j = c * PERIOD + i4 * 4;
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(src + j));
+    const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&v.x));
+    const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&v.y));
+    dst[t] = make_float4(f(j, lo.x), f(j + 1, lo.y), f(j + 2, hi.x), f(j + 3, hi.y));
+  }
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -228,6 +249,12 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned by
       : "memory");
 }
 
+// Prefetch [src, src + bytes) into L2 (16-byte aligned, a multiple of 16
+// bytes, inside one allocation); no completion to wait for.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, unsigned bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
   unsigned ok;
   asm volatile(
@@ -259,19 +286,31 @@ struct PrefilterHeader {
 
 // Each cell's (or sector's) list: the count and the candidate indices in
 // ascending order.  It is stored twice:
-//   head (8 bytes, one per list, all heads side by side): bits 0-3 hold
-//     min(count, 15) -- 15 meaning "15 or more, or overflowed: see the tail" --
-//     and bits 4-63 five 12-bit candidate slots; slots past the count repeat
-//     the first candidate.  One 8-byte load resolves almost every point, and
-//     a 128-byte line holds 16 neighbouring heads.
+//   head (8 bytes, one per list, all heads side by side): four 16-bit slots,
+//     slot k holding 8 x (index of candidate k) -- the candidate's byte offset
+//     in a float2 codeword table -- in bits 0-13; slots past the count repeat
+//     the first candidate.  Bits 14-15 of slot 0: min(count, 4) - 1.  Bit 14
+//     of slot 2: the list has more than 4 candidates (the rest are in the
+//     tail) or overflowed.  One 8-byte load and four scores resolve almost
+//     every point.
 //   tail (64 bytes): 32 uint16 slots, slot 0 the exact count (kPfOverflow:
 //     search exhaustively), slots 1..count the candidates.
 constexpr int kPfSlots = 32;
 constexpr int kPfCap = kPfSlots - 1;         // candidates per list
 constexpr uint32_t kPfOverflow = 0xffffu;
-constexpr int kPfHeadSlots = 5;
+constexpr int kPfHeadSlots = 4;
+constexpr uint32_t kPfMoreBit = 0x4000u;     // in the upper word of a head
 
+// Cells per side of the encoder's table: about 8 sqrt(K) rounded up to a
+// power of two, so that near the origin a cell is under half a Voronoi cell
+// across and, for Lloyd codebooks of N(0, I_2), lists longer than 4 are rare
+// (K >= 8; smaller codebooks are searched exhaustively).  K = 2048: 512 x 512.
 __host__ __device__ inline int prefilter_grid(int bits) {
+  return bits < 3 ? 0 : 1 << ((bits + 8) / 2);
+}
+
+// The training table is rebuilt every Lloyd iteration: one step coarser.
+__host__ __device__ inline int prefilter_grid_train(int bits) {
   return bits <= 5 ? 0 : (bits <= 7 ? 64 : (bits <= 9 ? 128 : 256));
 }
 
@@ -283,12 +322,11 @@ __host__ __device__ inline size_t prefilter_lists_offset() {
 // the region |p| >= R (list of every codeword that can win there).
 constexpr int kPfSectors = 256;
 
-__host__ __device__ inline int prefilter_sectors(int bits) {
-  return prefilter_grid(bits) > 0 ? kPfSectors : 0;
-}
+__host__ __device__ inline int prefilter_sectors(int G) { return G > 0 ? kPfSectors : 0; }
 
-__host__ __device__ inline size_t prefilter_bytes_for(int bits) {
-  const size_t n = (size_t)prefilter_grid(bits) * prefilter_grid(bits) + prefilter_sectors(bits);
+// Bytes of a table with G x G cells.
+__host__ __device__ inline size_t prefilter_bytes_for(int G) {
+  const size_t n = (size_t)G * G + prefilter_sectors(G);
   return prefilter_lists_offset() + ((n * 8 + 15) / 16) * 16 + n * kPfSlots * sizeof(uint16_t);
 }
 
@@ -324,103 +362,124 @@ __device__ __forceinline__ PrefilterView prefilter_view(const void* table, int K
   return v;
 }
 
-// Codeword j in shared memory as (x, y, x^2 + y^2, 0).  The nearest codeword of
-// p minimises |c|^2 - 2 p.c (= |p - c|^2 - |p|^2), two FMAs per candidate.
-__device__ __forceinline__ float4 codeword_q(float2 c) {
-  return make_float4(c.x, c.y, fmaf(c.x, c.x, c.y * c.y), 0.f);
+// Codeword j sits in shared memory as a plain (x, y) pair.  The nearest
+// codeword of p minimises |c|^2 - 2 p.c (= |p - c|^2 - |p|^2), with |c|^2
+// formed as fma(x, x, y * y): three FMAs and a multiply per candidate.
+__device__ __forceinline__ float score_cw(float m2x, float m2y, float2 c) {
+  return fmaf(m2x, c.x, fmaf(m2y, c.y, fmaf(c.x, c.x, c.y * c.y)));
 }
 
-// Exhaustive search, ascending j with a strict '<' (lowest index on ties).
-// `scored` accumulates the number of codewords evaluated.
-__device__ __forceinline__ int nearest_all(float m2x, float m2y, const float4* cbq, int K,
-                                           unsigned& scored) {
-  scored += (unsigned)K;
-  float be = INFINITY;
-  int bi = 0;
-  for (int j = 0; j < K; ++j) {
-    const float4 c = cbq[j];
-    const float e = fmaf(m2x, c.x, fmaf(m2y, c.y, c.z));
-    if (e < be) {
-      be = e;
-      bi = j;
-    }
-  }
-  return bi;
-}
-
-__device__ __forceinline__ void score(float m2x, float m2y, const float4* cbq, uint32_t j,
-                                      float& be, int& bi) {
-  const float4 c = cbq[j];
-  const float e = fmaf(m2x, c.x, fmaf(m2y, c.y, c.z));
+__device__ __forceinline__ void score2(float m2x, float m2y, const float2* cb, uint32_t j,
+                                       float& be, int& bi) {
+  const float e = score_cw(m2x, m2y, cb[j]);
   if (e < be) {
     be = e;
     bi = (int)j;
   }
 }
 
-// Split form of nearest_pf, so that a caller can fetch the next point's list
-// head while it scores the current point.
-struct PfCursor {
-  const uint16_t* tail;  // nullptr: exhaustive search
-  uint2 head;
-};
-
-__device__ __forceinline__ PfCursor pf_locate(float px, float py, const PrefilterView& pf) {
-  PfCursor cur;
-  cur.tail = nullptr;
-  cur.head = make_uint2(0u, 0u);
-  if (pf.G > 0 && isfinite(px) && isfinite(py)) {
-    const float gx = (px + pf.R) * pf.inv_h;
-    const float gy = (py + pf.R) * pf.inv_h;
-    size_t n;
-    if (gx >= 0.f && gx < pf.Gf && gy >= 0.f && gy < pf.Gf) {
-      n = (size_t)((int)gy * pf.G + (int)gx);
-    } else {
-      const float t = (atan2f(py, px) + 3.14159265f) * ((float)pf.NS * 0.159154943f);
-      n = (size_t)pf.G * pf.G + min(max((int)t, 0), pf.NS - 1);
-    }
-    cur.head = __ldg(pf.heads + n);
-    cur.tail = pf.tails + n * kPfSlots;
-  }
-  return cur;
-}
-
-// Rare paths of pf_finish: lists longer than the 5 head slots (tail slots
-// 6..count), overflowed lists and points that are not finite (exhaustive
-// search).  Kept out of line so that the common path stays small.
-static __device__ __noinline__ int pf_finish_slow(const uint16_t* tail, float m2x, float m2y,
-                                                  const float4* cbq, int K, float be, int bi,
-                                                  unsigned* scored) {
-  const uint32_t cnt = tail == nullptr ? kPfOverflow : (uint32_t)__ldg(tail);
-  if (cnt == kPfOverflow) return nearest_all(m2x, m2y, cbq, K, *scored);
-  *scored += cnt - kPfHeadSlots;
-  for (uint32_t t = kPfHeadSlots + 1; t <= cnt; ++t) score(m2x, m2y, cbq, __ldg(tail + t), be, bi);
+// Exhaustive search, ascending j with a strict '<' (lowest index on ties).
+// `scored` accumulates the number of codewords evaluated.
+__device__ __forceinline__ int nearest_all2(float m2x, float m2y, const float2* cb, int K,
+                                            unsigned& scored) {
+  scored += (unsigned)K;
+  float be = INFINITY;
+  int bi = 0;
+  for (int j = 0; j < K; ++j) score2(m2x, m2y, cb, (uint32_t)j, be, bi);
   return bi;
 }
 
-// The 5 head slots are always filled (unused ones repeat the first candidate,
-// which cannot change a strict-'<' argmin taken in ascending slot order), so
-// the common case scores 5 codewords without branching.
-__device__ __forceinline__ int pf_finish(const PfCursor& cur, float px, float py,
-                                         const float4* cbq, int K, unsigned& scored) {
-  const float m2x = -2.f * px, m2y = -2.f * py;
-  const uint2 h = cur.head;
-  const uint32_t n5 = h.x & 15u;
-  float be = INFINITY;
-  int bi = 0;
-  if (cur.tail != nullptr) {
-    score(m2x, m2y, cbq, (h.x >> 4) & 0xfffu, be, bi);
-    score(m2x, m2y, cbq, (h.x >> 16) & 0xfffu, be, bi);
-    score(m2x, m2y, cbq, (h.x >> 28) | ((h.y & 0xffu) << 4), be, bi);
-    score(m2x, m2y, cbq, (h.y >> 8) & 0xfffu, be, bi);
-    score(m2x, m2y, cbq, h.y >> 20, be, bi);
-    if (n5 <= (uint32_t)kPfHeadSlots) {
-      scored += n5;
-      return bi;
+// List number of a point: its cell, or for a point off the grid the angular
+// sector; kPfNoList without a table or for a point that is not finite.
+constexpr uint32_t kPfNoList = 0xffffffffu;
+// Head given to points without a list (never written by the builder, whose
+// slots stay below 0x4000): bit 15 of slot 2.
+constexpr uint32_t kPfNoListBit = 0x8000u;
+
+__device__ __forceinline__ uint32_t pf_list(float px, float py, const PrefilterView& pf) {
+  uint32_t n = kPfNoList;
+  if (pf.G > 0) {
+    const float gx = (px + pf.R) * pf.inv_h;
+    const float gy = (py + pf.R) * pf.inv_h;
+    if (gx >= 0.f && gx < pf.Gf && gy >= 0.f && gy < pf.Gf) {
+      n = (uint32_t)((int)gy * pf.G + (int)gx);
+    } else if (isfinite(px) && isfinite(py)) {
+      const float t = (atan2f(py, px) + 3.14159265f) * ((float)pf.NS * 0.159154943f);
+      n = (uint32_t)(pf.G * pf.G + min(max((int)t, 0), pf.NS - 1));
     }
-    scored += kPfHeadSlots;
   }
-  return pf_finish_slow(cur.tail, m2x, m2y, cbq, K, be, bi, &scored);
+  return n;
+}
+
+// The head of a point's list (fetched ahead of its scoring by the callers).
+__device__ __forceinline__ uint2 pf_head(float px, float py, const PrefilterView& pf) {
+  const uint32_t n = pf_list(px, py, pf);
+  return n == kPfNoList ? make_uint2(0u, kPfNoListBit) : __ldg(pf.heads + n);
+}
+
+// Rare ends of pf_finish2: a list longer than the head (its tail continues
+// from slot 5 with the best of the head as the incumbent), an overflowed list
+// or a point without one (exhaustive search).
+__device__ __forceinline__ int pf_finish_rare(uint32_t hx, uint32_t hy, float px, float py,
+                                              float m2x, float m2y, const float2* cb, int K,
+                                              const PrefilterView& pf, float be, int bi,
+                                              unsigned& scored, bool count) {
+  const uint32_t head_cnt = ((hx >> 14) & 3u) + 1u;
+  if (hy & kPfNoListBit) {
+    if (count) scored -= head_cnt;
+    return nearest_all2(m2x, m2y, cb, K, scored);
+  }
+  const uint16_t* tail = pf.tails + (size_t)pf_list(px, py, pf) * kPfSlots;
+  const uint32_t cnt = __ldg(tail);
+  if (cnt == kPfOverflow) {
+    if (count) scored -= head_cnt;
+    return nearest_all2(m2x, m2y, cb, K, scored);
+  }
+  if (count) scored += cnt - kPfHeadSlots;
+  for (uint32_t t = kPfHeadSlots + 1; t <= cnt; ++t) score2(m2x, m2y, cb, __ldg(tail + t), be, bi);
+  return bi;
+}
+
+// Nearest codeword of p from its list head; the same index as nearest_all2.
+// Slot t of the head is scored when t < min(count, 4) -- a predicated shared
+// load, so that lanes with short lists add no traffic -- and the others score
+// +inf; the minimum of the four is taken as a tree in which the left operand
+// wins ties (the slots hold ascending indices).  With `count`, `scored`
+// accumulates the distinct candidates of each list.
+__device__ __forceinline__ int pf_finish2(uint2 h, float px, float py, const float2* cb, int K,
+                                          const PrefilterView& pf, unsigned& scored, bool count) {
+  const float m2x = -2.f * px, m2y = -2.f * py;
+  const uint32_t hx = h.x, hy = h.y;
+  const uint32_t o0 = hx & 0x3fffu, o1 = hx >> 16, o2 = hy & 0x3fffu, o3 = hy >> 16;
+  const uint32_t n4 = (hx >> 14) & 3u;  // min(count, 4) - 1
+  const unsigned char* base = reinterpret_cast<const unsigned char*>(cb);
+  const float e0 = score_cw(m2x, m2y, *reinterpret_cast<const float2*>(base + o0));
+  float e1 = INFINITY, e2 = INFINITY, e3 = INFINITY;
+  if (n4 >= 1u) e1 = score_cw(m2x, m2y, *reinterpret_cast<const float2*>(base + o1));
+  if (n4 >= 2u) e2 = score_cw(m2x, m2y, *reinterpret_cast<const float2*>(base + o2));
+  if (n4 >= 3u) e3 = score_cw(m2x, m2y, *reinterpret_cast<const float2*>(base + o3));
+  float ea = e0, eb = e2;
+  uint32_t oa = o0, ob = o2;
+  if (e1 < ea) {
+    ea = e1;
+    oa = o1;
+  }
+  if (e3 < eb) {
+    eb = e3;
+    ob = o3;
+  }
+  if (eb < ea) {
+    ea = eb;
+    oa = ob;
+  }
+  if (count) scored += n4 + 1u;
+  if (!(hy & (kPfMoreBit | kPfNoListBit))) return (int)(oa >> 3);
+  return pf_finish_rare(hx, hy, px, py, m2x, m2y, cb, K, pf, ea, (int)(oa >> 3), scored, count);
+}
+
+__device__ __forceinline__ int nearest_pf2(float px, float py, const float2* cb, int K,
+                                           const PrefilterView& pf, unsigned& scored, bool count) {
+  return pf_finish2(pf_head(px, py, pf), px, py, cb, K, pf, scored, count);
 }
 
 // Polar baseline (paper section 3.5): amplitude |p| to the nearest of the Na
@@ -443,10 +502,5 @@ __device__ __forceinline__ int polar_index(float px, float py, const float* lev,
   return ia * Np + ip;
 }
 
-// Nearest codeword through the prefilter (same result as nearest_all).
-__device__ __forceinline__ int nearest_pf(float px, float py, const float4* cbq, int K,
-                                          const PrefilterView& pf, unsigned& scored) {
-  return pf_finish(pf_locate(px, py, pf), px, py, cbq, K, scored);
-}
 
 }  // namespace qamw

@@ -7,6 +7,8 @@
 //   k_calib_ext     later rows when those held zero rows             (1 CTA)
 //   k_calib_finish  sigma_k = binary16(sum / (n sqrt(pi/2)))        (16 threads/pair)
 //   k_encode        norm, rotate, normalise, nearest codeword, pack  (row groups)
+#include <algorithm>
+
 #include "common.cuh"
 #include "launch.cuh"
 
@@ -60,43 +62,6 @@ __global__ void __launch_bounds__(256) k_scales(const float* __restrict__ a, int
 __global__ void k_fill_half(__half* p, int n, float v) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) p[i] = __float2half(v);
-}
-
-// --------------------------------------------------------------- row norms
-
-template <typename T>
-struct Vec8;  // 8 consecutive weights
-template <>
-struct Vec8<float> {
-  __device__ static void load(const float* p, float (&x)[8]) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-  }
-};
-template <>
-struct Vec8<__nv_bfloat16> {
-  __device__ static void load(const __nv_bfloat16* p, float (&x)[8]) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
-    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      x[2 * e] = __uint_as_float(u[e] << 16);
-      x[2 * e + 1] = __uint_as_float(u[e] & 0xffff0000u);
-    }
-  }
-};
-
-__device__ __forceinline__ void load_half8(const __half* p, float (&x)[8]) {
-  const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
-  const __half2* h = reinterpret_cast<const __half2*>(&v);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float2 f = __half22float2(h[e]);
-    x[2 * e] = f.x;
-    x[2 * e + 1] = f.y;
-  }
 }
 
 // ------------------------------------------------------------- calibration
@@ -329,26 +294,28 @@ struct EncodeArgs {
 // Steps 1-6 of section 3.1 in one pass over W: scale by s, sum of squares
 // (reduced per row in a fixed order, so r is bitwise reproducible), Hadamard
 // butterflies, division by r sqrt(b) and sigma_k, nearest codeword, packing.
+// This form searches straight from the 64 rotated values in registers; it
+// serves rows too wide for k_encode's shared-memory point buffer.
 template <int BITS, typename T, bool POLAR>
-__global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
+__global__ void __launch_bounds__(512, 1) k_encode_wide(const EncodeArgs<T> a) {
   extern __shared__ __align__(16) unsigned char smem[];
-  float4* cbq = reinterpret_cast<float4*>(smem);
+  float2* cb2 = reinterpret_cast<float2*>(smem);
   // per-column tables transposed, [position in chunk][chunk], so that the lanes
   // of a warp (consecutive chunks) read consecutive words
   const int P = a.d_in >> 1, C = a.d_in / kE;
-  float* fT = reinterpret_cast<float*>(cbq + a.K);  // [j][c]: D * s of column 64c + j
+  float* fT = reinterpret_cast<float*>(cb2 + ((a.K + 1) & ~1));  // [j][c]: D * s of column 64c + j
   float* isgT = fT + a.d_in;                        // [q][c]: 1 / sigma of pair 32c + q
   float* part = isgT + P;                           // [blockDim] partial sums of squares
   float* rsum = part + blockDim.x;                  // [R] row norms
   // polar: amplitude levels a_i = codeword (i Np).x of the expanded table
   constexpr int kBa = BITS / 2, kNa = 1 << kBa, kNp = 1 << (BITS - kBa);
-  float* lev = reinterpret_cast<float*>(cbq);
+  float* lev = reinterpret_cast<float*>(cb2);
   if constexpr (POLAR) {
     for (int i = threadIdx.x; i < kNa; i += blockDim.x) lev[i] = a.codebook[i * kNp].x;
   } else {
     // table fills: unrolled so that each thread's loads are in flight together
 #pragma unroll 4
-    for (int i = threadIdx.x; i < a.K; i += blockDim.x) cbq[i] = codeword_q(a.codebook[i]);
+    for (int i = threadIdx.x; i < a.K; i += blockDim.x) cb2[i] = a.codebook[i];
   }
   const uint64_t seed = a.seed;
   fill_interleaved<kE>(fT, a.scale, a.d_in, C, [=](int j, float v) {
@@ -371,6 +338,7 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
   const float sqrt_b = sqrtf((float)a.block);
   int flags = 0;
   unsigned scored = 0;
+  const bool count = a.candidates != nullptr;
   for (int64_t r0 = (int64_t)blockIdx.x * R; r0 < a.d_out; r0 += (int64_t)gridDim.x * R) {
     const int64_t row = r0 + rl;
     const bool active = rl < R && row < a.d_out;
@@ -430,18 +398,19 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
     } else {
       float is = isgT[c];
       float px = (x[0] * inv) * is, py = (x[1] * inv) * is;
-      PfCursor cur = pf_locate(px, py, pf);
+      uint2 cur = pf_head(px, py, pf);
 #pragma unroll
       for (int q = 0; q < kQ; ++q) {
         float nx = 0.f, ny = 0.f;
-        PfCursor nxt = cur;
+        uint2 nxt = cur;
         if (q + 1 < kQ) {
           const float is1 = isgT[(q + 1) * C + c];
           nx = (x[2 * q + 2] * inv) * is1;
           ny = (x[2 * q + 3] * inv) * is1;
-          nxt = pf_locate(nx, ny, pf);
+          nxt = pf_head(nx, ny, pf);
         }
-        const uint32_t id = zero ? 0u : (uint32_t)pf_finish(cur, px, py, cbq, a.K, scored);
+        const uint32_t id =
+            zero ? 0u : (uint32_t)pf_finish2(cur, px, py, cb2, a.K, pf, scored, count);
         const int bit = q * BITS, wi = bit >> 5, sh = bit & 31;
         w[wi] |= id << sh;
         if (sh + BITS > 32) w[wi + 1] |= id >> (32 - sh);
@@ -467,8 +436,196 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
   }
 }
 
-// Rows per CTA iteration and the CTA size: R whole rows of C chunk-threads,
-// R * C <= 512, chosen so that few threads idle and the CTA has 128-512 threads.
+// The same steps in two phases per CTA iteration, so that the 64 rotated
+// values leave the registers before the search:
+//   phase 1  load, scale, sum of squares, butterflies, row norm, normalise;
+//            thread t writes its 32 points to pts[q][t] (its own column of the
+//            buffer: no barrier between the phases, conflict-free accesses);
+//   phase 2  a rolled loop over the 32 points: the list head of point q + 2 is
+//            fetched while point q is scored against the codewords (a plain
+//            (x, y) table, scores bitwise those of k_encode_wide), and the
+//            indices are packed through a 64-bit bit accumulator that emits
+//            each 32-bit word as it fills.
+// Shared memory: cb2 float2[K] | fT4 float4[16][C] | isg4 float4[8][C] |
+// pts float2[32][T] | part float[T] | rsum float[R].
+template <int BITS, typename T, bool POLAR>
+__global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int C = a.d_in / kE, NT = blockDim.x;
+  float2* cb2 = reinterpret_cast<float2*>(smem);
+  float4* fT4 = reinterpret_cast<float4*>(smem + (((size_t)a.K * sizeof(float2) + 15) & ~15));
+  float4* isg4 = fT4 + (kE / 4) * C;
+  float2* pts = reinterpret_cast<float2*>(isg4 + (kQ / 4) * C);
+  float* part = reinterpret_cast<float*>(pts + (size_t)kQ * NT);
+  float* rsum = part + NT;
+  constexpr int kBa = BITS / 2, kNa = 1 << kBa, kNp = 1 << (BITS - kBa);
+  float* lev = reinterpret_cast<float*>(cb2);
+  if constexpr (POLAR) {
+    for (int i = threadIdx.x; i < kNa; i += NT) lev[i] = a.codebook[i * kNp].x;
+  } else {
+#pragma unroll 4
+    for (int i = threadIdx.x; i < a.K; i += NT) cb2[i] = a.codebook[i];
+  }
+  const uint64_t seed = a.seed;
+  fill_quads<kE>(fT4, a.scale, a.d_in, C, [=](int j, float v) {
+    return mask_negative(seed, (uint32_t)j) ? -v : v;
+  });
+  fill_quads<kQ>(isg4, a.sigma, a.d_in / 2, C, [](int, float v) { return 1.0f / v; });
+  PrefilterView pf;
+  if (a.prefilter != nullptr) {
+    pf = prefilter_view(a.prefilter, a.K);
+  } else {
+    pf.G = 0;
+    pf.Gf = 0.f;
+  }
+  __syncthreads();
+
+  const int R = a.rows_per_cta;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = NT >> 5;
+  // W of row group r0 (R rows from r0, clipped to the matrix) into L2
+  auto prefetch_rows = [&](int64_t r0) {
+    if (threadIdx.x == 0 && r0 < a.d_out) {
+      const int64_t nr = min((int64_t)R, (int64_t)a.d_out - r0);
+      bulk_prefetch_l2(a.W + r0 * a.d_in, (unsigned)(nr * a.d_in * (int64_t)sizeof(T)));
+    }
+  };
+  prefetch_rows((int64_t)blockIdx.x * R);
+  const int rl = threadIdx.x / C, c = threadIdx.x - rl * C;
+  const int nb = min(a.block, kE), lanes = max(a.block / kE, 1);
+  const float sqrt_b = sqrtf((float)a.block);
+  float2* mypts = pts + threadIdx.x;
+  int flags = 0;
+  unsigned scored = 0;
+  const bool count = a.candidates != nullptr;
+  for (int64_t r0 = (int64_t)blockIdx.x * R; r0 < a.d_out; r0 += (int64_t)gridDim.x * R) {
+    const int64_t row = r0 + rl;
+    const bool active = rl < R && row < a.d_out;
+    float x[kE];
+    float ss = 0.f;
+    if (active) {
+      load64(a.W + row * a.d_in + (int64_t)c * kE, x);
+#pragma unroll
+      for (int i = 0; i < kE / 4; ++i) {
+        const float4 f = fT4[i * C + c];
+        x[4 * i] *= f.x;
+        ss = fmaf(x[4 * i], x[4 * i], ss);
+        x[4 * i + 1] *= f.y;
+        ss = fmaf(x[4 * i + 1], x[4 * i + 1], ss);
+        x[4 * i + 2] *= f.z;
+        ss = fmaf(x[4 * i + 2], x[4 * i + 2], ss);
+        x[4 * i + 3] *= f.w;
+        ss = fmaf(x[4 * i + 3], x[4 * i + 3], ss);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < kE; ++j) x[j] = 0.f;
+    }
+    part[threadIdx.x] = ss;
+    fwht_reg<kE>(x, nb);
+    fwht_lanes<kE>(x, lanes);
+    __syncthreads();
+    for (int q = warp; q < R; q += nwarps) {
+      float t = 0.f;
+      for (int k = lane; k < C; k += 32) t += part[q * C + k];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      if (lane == 0) rsum[q] = sqrtf(t);
+    }
+    __syncthreads();
+    prefetch_rows(r0 + (int64_t)gridDim.x * R);  // the next row group, during the search
+    if (!active) continue;
+
+    const float r = rsum[rl];
+    if (c == 0) {
+      const __half h = __float2half_rn(r);
+      a.rnorm[row] = h;
+      if (!isfinite(r)) flags |= QAMW_STATUS_NONFINITE;
+      else if (isinf(__half2float(h))) flags |= QAMW_STATUS_RANGE;
+    }
+    uint32_t* dst = reinterpret_cast<uint32_t*>(a.packed + row * a.row_bytes) + (size_t)c * BITS;
+    if (!(r > 0.f)) {  // zero row: every index 0
+#pragma unroll
+      for (int t = 0; t < BITS; ++t) dst[t] = 0u;
+    } else {
+      const float inv = 1.0f / (r * sqrt_b);
+#pragma unroll
+      for (int i = 0; i < kQ / 4; ++i) {
+        const float4 is = isg4[i * C + c];
+        mypts[(4 * i + 0) * NT] = make_float2((x[8 * i + 0] * inv) * is.x, (x[8 * i + 1] * inv) * is.x);
+        mypts[(4 * i + 1) * NT] = make_float2((x[8 * i + 2] * inv) * is.y, (x[8 * i + 3] * inv) * is.y);
+        mypts[(4 * i + 2) * NT] = make_float2((x[8 * i + 4] * inv) * is.z, (x[8 * i + 5] * inv) * is.z);
+        mypts[(4 * i + 3) * NT] = make_float2((x[8 * i + 6] * inv) * is.w, (x[8 * i + 7] * inv) * is.w);
+      }
+      uint64_t acc = 0;
+      int nbits = 0;
+      if constexpr (POLAR) {
+        const float np_over_2pi = (float)kNp * 0.159154943f;
+#pragma unroll 1
+        for (int q = 0; q < kQ; ++q) {
+          const float2 p = mypts[q * NT];
+          const uint32_t id = (uint32_t)polar_index(p.x, p.y, lev, kNa, kNp, np_over_2pi);
+          scored += kNa;
+          acc |= (uint64_t)id << nbits;
+          nbits += BITS;
+          if (nbits >= 32) {
+            *dst++ = (uint32_t)acc;
+            acc >>= 32;
+            nbits -= 32;
+          }
+        }
+      } else {
+        // list heads of kGrp points are fetched one group ahead of their
+        // scoring, so that the L2 latency of a head load is hidden
+        constexpr int kGrp = 4;
+        uint2 hc[kGrp], hn[kGrp];
+#pragma unroll
+        for (int k = 0; k < kGrp; ++k) {
+          const float2 p = mypts[k * NT];
+          hc[k] = pf_head(p.x, p.y, pf);
+        }
+#pragma unroll 1
+        for (int g = 0; g < kQ / kGrp; ++g) {
+          if (g + 1 < kQ / kGrp) {
+#pragma unroll
+            for (int k = 0; k < kGrp; ++k) {
+              const float2 p = mypts[((g + 1) * kGrp + k) * NT];
+              hn[k] = pf_head(p.x, p.y, pf);
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < kGrp; ++k) {
+            const float2 p = mypts[(g * kGrp + k) * NT];
+            const uint32_t id = (uint32_t)pf_finish2(hc[k], p.x, p.y, cb2, a.K, pf, scored, count);
+            acc |= (uint64_t)id << nbits;
+            nbits += BITS;
+            if (nbits >= 32) {
+              *dst++ = (uint32_t)acc;
+              acc >>= 32;
+              nbits -= 32;
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < kGrp; ++k) hc[k] = hn[k];
+        }
+      }
+    }
+    if (c == C - 1) {  // zero the row's padding words
+      for (int64_t o = (int64_t)C * BITS * 4; o < a.row_bytes; o += 4)
+        *reinterpret_cast<uint32_t*>(a.packed + row * a.row_bytes + o) = 0u;
+    }
+  }
+  raise_flag(a.status, flags);
+  if (a.candidates != nullptr) {
+    unsigned long long v = scored;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) atomicAdd(a.candidates, v);
+  }
+}
+
+// Rows per CTA iteration and the CTA size for k_encode_wide: R whole rows of C
+// chunk-threads, R * C <= 512, chosen so that few threads idle and the CTA has
+// 128-512 threads.
 void encode_shape(int C, int* R_out, int* threads_out) {
   int bestR = 1, bestT = ((C + 31) / 32) * 32;
   double bestScore = -1.0;
@@ -487,21 +644,62 @@ void encode_shape(int C, int* R_out, int* threads_out) {
   *threads_out = bestT;
 }
 
+size_t encode_staged_smem(int K, int d_in, int T, int R) {
+  return (((size_t)K * sizeof(float2) + 15) & ~(size_t)15) + (size_t)d_in * sizeof(float) +
+         (size_t)(d_in / 2) * sizeof(float) + (size_t)T * kQ * sizeof(float2) +
+         (size_t)T * sizeof(float) + (size_t)R * sizeof(float);
+}
+
+// k_encode's shape: the R (rows per CTA iteration, R * C <= 512 threads) that
+// keeps the most busy threads resident per SM (228 KB of shared memory, 512
+// threads at <= 128 registers); ties go to the smaller CTA.  Returns false when
+// not even one row fits.
+bool encode_staged_shape(int C, int K, int d_in, int* R_out, int* threads_out, size_t* smem_out) {
+  int bestR = 0, bestT = 0;
+  size_t bestS = 0;
+  long best = -1;
+  for (int R = 1; R * C <= 512; ++R) {
+    const int T = ((R * C + 31) / 32) * 32;
+    const size_t sm = encode_staged_smem(K, d_in, T, R);
+    if (sm > 227 * 1024) break;
+    const int by_smem = (int)((228 * 1024) / (sm + 1024));
+    const int ctas = std::min(by_smem, 512 / T);
+    const long busy = (long)ctas * R * C;
+    if (ctas >= 1 && busy > best) {
+      best = busy;
+      bestR = R;
+      bestT = T;
+      bestS = sm;
+    }
+  }
+  if (bestR == 0) return false;
+  *R_out = bestR;
+  *threads_out = bestT;
+  *smem_out = bestS;
+  return true;
+}
+
 template <int BITS, typename T, bool POLAR>
 cudaError_t run_encode(EncodeArgs<T> a, cudaStream_t stream) {
   const int C = a.d_in / kE;
   int R, threads;
-  encode_shape(C, &R, &threads);
+  size_t smem;
+  const void* fn;
+  if (encode_staged_shape(C, a.K, a.d_in, &R, &threads, &smem)) {
+    fn = reinterpret_cast<const void*>(&k_encode<BITS, T, POLAR>);
+  } else {
+    encode_shape(C, &R, &threads);
+    smem = (size_t)((a.K + 1) & ~1) * sizeof(float2) + (size_t)a.d_in * sizeof(float) +
+           (size_t)(a.d_in / 2) * sizeof(float) + (size_t)threads * sizeof(float) +
+           (size_t)R * sizeof(float);
+    fn = reinterpret_cast<const void*>(&k_encode_wide<BITS, T, POLAR>);
+  }
   a.rows_per_cta = R;
-  const size_t smem = (size_t)a.K * sizeof(float4) + (size_t)a.d_in * sizeof(float) +
-                      (size_t)(a.d_in / 2) * sizeof(float) + (size_t)threads * sizeof(float) +
-                      (size_t)R * sizeof(float);
-  const void* fn = reinterpret_cast<const void*>(&k_encode<BITS, T, POLAR>);
   cudaError_t err = allow_smem(fn, smem);
   if (err != cudaSuccess) return err;
   const int grid = persistent_grid(fn, threads, smem, (a.d_out + R - 1) / R);
-  k_encode<BITS, T, POLAR><<<grid, threads, smem, stream>>>(a);
-  return cudaGetLastError();
+  void* args[] = {&a};
+  return cudaLaunchKernel(fn, dim3(grid), dim3(threads), args, smem, stream);
 }
 
 template <typename T, bool POLAR>
@@ -654,7 +852,7 @@ size_t calibrate_workspace_bytes(int d_out, int d_in, EncodeWorkspace* carve, vo
 size_t encode_workspace_bytes(int d_out, int d_in, int bits, EncodeWorkspace* carve, void* base) {
   const size_t off = calibrate_workspace_bytes(d_out, d_in, carve, base);
   if (carve) carve->prefilter = static_cast<char*>(base) + off;
-  return off + align256(prefilter_bytes_for(bits));
+  return off + align256(prefilter_bytes_for(prefilter_grid(bits)));
 }
 
 cudaError_t launch_channel_scales(const float* d_act_stat, int d_in, float alpha, uint16_t* d_scale,
@@ -706,7 +904,7 @@ cudaError_t launch_encode(const void* d_W, int dtype, const float* d_act_stat, f
   if (flags & QAMW_POLAR) return launch_encode_rows(d_W, dtype, m, d_status, nullptr, true, stream);
   qamw_matrix mm = m;
   if (mm.prefilter == nullptr) {
-    err = launch_build_prefilter(m.codebook, m.bits, ws.prefilter, stream);
+    err = launch_build_prefilter(m.codebook, m.bits, prefilter_grid(m.bits), ws.prefilter, stream);
     if (err != cudaSuccess) return err;
     mm.prefilter = ws.prefilter;
   }

@@ -49,7 +49,9 @@ cudaError_t launch_polar_codebook(int bits, float* d_codebook, cudaStream_t stre
 cudaError_t launch_encode(const void* d_W, int dtype, const float* d_act_stat, float alpha,
                           int flags, const qamw_matrix& m, const EncodeWorkspace& ws,
                           int32_t* d_status, cudaStream_t stream);
-cudaError_t launch_build_prefilter(const float* d_codebook, int bits, void* d_table,
+// Table of G x G cells (prefilter_grid(bits) for the encoder) for the
+// codebook of 2^bits entries; d_table holds prefilter_bytes_for(G) bytes.
+cudaError_t launch_build_prefilter(const float* d_codebook, int bits, int G, void* d_table,
                                    cudaStream_t stream);
 cudaError_t launch_train(const float* d_samples, int64_t n, int bits, int iters,
                          float* d_codebook, double* d_distortion, void* d_ws,

@@ -26,29 +26,20 @@ namespace {
 
 __global__ void __launch_bounds__(1024) k_pf_header(const float2* __restrict__ cb, int K, int G,
                                                     PrefilterHeader* __restrict__ hdr) {
-  __shared__ float red[2][32];
-  float mc = 0.f, mr = 0.f;
+  __shared__ float red[32];
+  float mr = 0.f;
   for (int j = threadIdx.x; j < K; j += blockDim.x) {
     const float2 c = cb[j];
-    mc = fmaxf(mc, fmaxf(fabsf(c.x), fabsf(c.y)));
     mr = fmaxf(mr, sqrtf(c.x * c.x + c.y * c.y));
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, o));
-    mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, o));
-  }
-  if ((threadIdx.x & 31) == 0) {
-    red[0][threadIdx.x >> 5] = mc;
-    red[1][threadIdx.x >> 5] = mr;
-  }
+  for (int o = 16; o > 0; o >>= 1) mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mr;
   __syncthreads();
   if (threadIdx.x == 0) {
-    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) {
-      mc = fmaxf(mc, red[0][w]);
-      mr = fmaxf(mr, red[1][w]);
-    }
-    const float R = 1.25f * mc + 0.25f;
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) mr = fmaxf(mr, red[w]);
+    // the grid just covers the codebook; points beyond use the sector lists
+    const float R = 1.0625f * mr + 0.0625f;
     PrefilterHeader h;
     h.R = R;
     h.inv_h = (float)G / (2.f * R);
@@ -67,26 +58,29 @@ constexpr int kBuildWarps = 8;
 constexpr int kMaxCand = 256;
 
 // Tail: slot 0 the count (kPfOverflow when the list did not fit), slots 1..m
-// the candidates, the rest zero.  Head: min(count, 15) (15 for overflow) and 5
-// 12-bit slots, unused ones repeating the first candidate (scored without a
-// branch by the encoder).  Called by all 32 lanes of a warp.
+// the candidates, the rest zero.  Head: four 16-bit slots with 8 x the first
+// four candidates (unused ones repeating the first, scored without a branch
+// by the encoder), min(m, 4) - 1 in bits 14-15 of slot 0, and the "more in the
+// tail" bit in slot 2.  Called by all 32 lanes of a warp.
 __device__ void write_list(void* table, size_t nlists, size_t n, bool overflow, int m,
                            const uint16_t* keep) {
   const int lane = threadIdx.x & 31;
+  overflow = overflow || m <= 0;
   uint16_t* tail = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(table) +
                                                prefilter_tails_offset(nlists)) +
                    n * kPfSlots;
   tail[lane] = lane == 0 ? (overflow ? (uint16_t)kPfOverflow : (uint16_t)m)
                          : (!overflow && lane - 1 < m ? keep[lane - 1] : (uint16_t)0);
   if (lane == 0) {
-    unsigned long long h = overflow ? 15ull : (unsigned long long)(m < 15 ? m : 15);
     const uint32_t first = overflow ? 0u : keep[0];
-    for (int t = 0; t < kPfHeadSlots; ++t) {
-      const uint32_t v = (!overflow && t < m) ? keep[t] : first;
-      h |= (unsigned long long)(v & 0xfffu) << (4 + 12 * t);
-    }
-    *reinterpret_cast<unsigned long long*>(reinterpret_cast<uint8_t*>(table) +
-                                           prefilter_lists_offset() + n * 8) = h;
+    uint32_t slot[kPfHeadSlots];
+    for (int t = 0; t < kPfHeadSlots; ++t)
+      slot[t] = (((!overflow && t < m) ? (uint32_t)keep[t] : first) << 3) & 0x3fffu;
+    slot[0] |= (uint32_t)((overflow ? kPfHeadSlots : min(m, kPfHeadSlots)) - 1) << 14;
+    if (overflow || m > kPfHeadSlots) slot[2] |= kPfMoreBit;
+    const uint2 h = make_uint2(slot[0] | (slot[1] << 16), slot[2] | (slot[3] << 16));
+    *reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(table) + prefilter_lists_offset() +
+                              n * 8) = h;
   }
 }
 
@@ -315,9 +309,8 @@ __global__ void __launch_bounds__(kBuildWarps * 32) k_pf_sectors(const float2* _
 
 }  // namespace
 
-cudaError_t launch_build_prefilter(const float* d_codebook, int bits, void* d_table,
+cudaError_t launch_build_prefilter(const float* d_codebook, int bits, int G, void* d_table,
                                    cudaStream_t stream) {
-  const int G = prefilter_grid(bits);
   const int K = 1 << bits;
   const float2* cb = reinterpret_cast<const float2*>(d_codebook);
   PrefilterHeader* hdr = reinterpret_cast<PrefilterHeader*>(d_table);
@@ -327,7 +320,7 @@ cudaError_t launch_build_prefilter(const float* d_codebook, int bits, void* d_ta
   const int cells = G * G;
   k_pf_build<<<(cells + kBuildWarps - 1) / kBuildWarps, kBuildWarps * 32, 0, stream>>>(cb, d_table);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  const int NS = prefilter_sectors(bits);
+  const int NS = prefilter_sectors(G);
   k_pf_sectors<<<(NS + kBuildWarps - 1) / kBuildWarps, kBuildWarps * 32, 0, stream>>>(cb, d_table);
   return cudaGetLastError();
 }

@@ -45,13 +45,13 @@ __global__ void __launch_bounds__(512) k_assign(const float2* __restrict__ sampl
                                                 const void* __restrict__ table, TrainAccum acc,
                                                 int32_t* status) {
   extern __shared__ __align__(16) unsigned char smem[];
-  float4* cbq = reinterpret_cast<float4*>(smem);
-  unsigned long long* ssx = reinterpret_cast<unsigned long long*>(cbq + K);
+  float2* cb2 = reinterpret_cast<float2*>(smem);
+  unsigned long long* ssx = reinterpret_cast<unsigned long long*>(cb2 + K);
   unsigned long long* ssy = ssx + K;
   unsigned int* scnt = reinterpret_cast<unsigned int*>(ssy + K);
   __shared__ unsigned long long sd, sn;
   for (int j = threadIdx.x; j < K; j += blockDim.x) {
-    cbq[j] = codeword_q(cb[j]);
+    cb2[j] = cb[j];
     ssx[j] = 0ull;
     ssy[j] = 0ull;
     scnt[j] = 0u;
@@ -82,8 +82,8 @@ __global__ void __launch_bounds__(512) k_assign(const float2* __restrict__ sampl
       continue;
     }
     unsigned scored = 0;
-    const int j = nearest_pf(p.x, p.y, cbq, K, pf, scored);
-    const float dx = p.x - cbq[j].x, dy = p.y - cbq[j].y;
+    const int j = nearest_pf2(p.x, p.y, cb2, K, pf, scored, false);
+    const float dx = p.x - cb2[j].x, dy = p.y - cb2[j].y;
     const float d = fmaf(dx, dx, dy * dy);
     atomicAdd(&ssx[j], (unsigned long long)__float2ll_rn(p.x * kFix));
     atomicAdd(&ssy[j], (unsigned long long)__float2ll_rn(p.y * kFix));
@@ -140,7 +140,7 @@ __global__ void k_zero_u64(unsigned long long* p, int n) {
 size_t train_workspace_bytes(int bits) {
   const size_t K = (size_t)1 << bits;
   const size_t acc = ((3 * K + 2) * sizeof(unsigned long long) + 255) & ~(size_t)255;
-  return acc + prefilter_bytes_for(bits);
+  return acc + prefilter_bytes_for(prefilter_grid_train(bits));
 }
 
 cudaError_t launch_train(const float* d_samples, int64_t n, int bits, int iters, float* d_codebook,
@@ -152,20 +152,21 @@ cudaError_t launch_train(const float* d_samples, int64_t n, int bits, int iters,
   unsigned long long* w = static_cast<unsigned long long*>(d_ws);
   TrainAccum acc{w, w + K, w + 2 * K, w + 3 * K, w + 3 * K + 1};
   const size_t acc_bytes = ((3 * (size_t)K + 2) * sizeof(unsigned long long) + 255) & ~(size_t)255;
-  void* table = prefilter_grid(bits) > 0 ? static_cast<char*>(d_ws) + acc_bytes : nullptr;
+  const int G = prefilter_grid_train(bits);
+  void* table = G > 0 ? static_cast<char*>(d_ws) + acc_bytes : nullptr;
   const int nz = 3 * K + 2;
   k_zero_u64<<<(nz + 255) / 256, 256, 0, stream>>>(w, nz);
   k_init<<<(K + 255) / 256, 256, 0, stream>>>(samples, K, cb);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   const int threads = 512;
-  const size_t smem = (size_t)K * (sizeof(float4) + 2 * sizeof(unsigned long long) + sizeof(unsigned));
+  const size_t smem = (size_t)K * (sizeof(float2) + 2 * sizeof(unsigned long long) + sizeof(unsigned));
   const void* fn = reinterpret_cast<const void*>(&k_assign);
   if ((err = allow_smem(fn, smem)) != cudaSuccess) return err;
   const int grid = persistent_grid(fn, threads, smem, (n + threads - 1) / threads);
   for (int it = 0; it < iters; ++it) {
     if (table != nullptr) {
-      if ((err = launch_build_prefilter(d_codebook, bits, table, stream)) != cudaSuccess) return err;
+      if ((err = launch_build_prefilter(d_codebook, bits, G, table, stream)) != cudaSuccess) return err;
     }
     k_assign<<<grid, threads, smem, stream>>>(samples, n, cb, K, table, acc, d_status);
     k_update<<<(K + 255) / 256, 256, 0, stream>>>(cb, K, acc, d_distortion, it);
