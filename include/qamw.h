@@ -211,8 +211,10 @@ QAMW_API int qamw_calibrate_sigma(const void *d_W, int dtype, const qamw_matrix 
  *   m->chan_scale and m->sigma; writes m->packed and m->row_norm.  One kernel,
  *   no workspace.  m->prefilter may be NULL (exhaustive search; same result,
  *   slower for large K).  d_candidates (nullable, 8-byte aligned): the number
- *   of codewords the search scored is added to it (work accounting for the
- *   roofline; costs one reduction per CTA).  Flags: NONFINITE, RANGE. */
+ *   of distinct list candidates the search scored is added to it (work
+ *   accounting for the roofline; costs one reduction per CTA).  A row whose
+ *   norm is zero, or not finite (NaN/Inf in the row; flagged NONFINITE), is
+ *   stored with all indices 0.  Flags: NONFINITE, RANGE. */
 QAMW_API int qamw_encode_rows(const void *d_W, int dtype, const qamw_matrix *m,
                               uint64_t *d_candidates, int32_t *d_status, void *stream);
 

@@ -224,6 +224,23 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
 }
 
+// Shared-memory loads at a 32-bit shared address (base + byte offset), so
+// that gathers need no 64-bit address arithmetic.  lds_f2_ge loads only when
+// n >= k (a predicated load), else keeps v.
+__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
+  float2 v;
+  asm("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+
+template <int k>
+__device__ __forceinline__ float2 lds_f2_ge(uint32_t n, uint32_t addr, float2 v) {
+  asm("{\n .reg .pred q;\n setp.ge.u32 q, %2, %3;\n @q ld.shared.v2.f32 {%0, %1}, [%4];\n}"
+      : "+f"(v.x), "+f"(v.y)
+      : "r"(n), "n"(k), "r"(addr));
+  return v;
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
                : "memory");
@@ -282,6 +299,7 @@ struct PrefilterHeader {
   int32_t cap;   // list capacity per cell
   int32_t K;
   int32_t NS;    // angular sectors for points off the grid (|p| >= R)
+  int32_t Gi;    // inner grid: G / 2 cells per side, heads only (0: none)
 };
 
 // Each cell's (or sector's) list: the count and the candidate indices in
@@ -324,10 +342,19 @@ constexpr int kPfSectors = 256;
 
 __host__ __device__ inline int prefilter_sectors(int G) { return G > 0 ? kPfSectors : 0; }
 
-// Bytes of a table with G x G cells.
+// The inner grid has cells twice as wide (G / 2 per side, over the same
+// square); cell (ix, iy) covers main cells 2ix..2ix+1 x 2iy..2iy+1 and its head
+// holds the union of their lists (ascending), or the "more" bit when that
+// union has more than 4 candidates or a child list overflowed.  It exists to
+// be copied, in part, into shared memory.
+__host__ __device__ inline int prefilter_inner(int G) { return G / 2; }
+
+// Bytes of a table with G x G cells: header, heads, tails, inner heads.
 __host__ __device__ inline size_t prefilter_bytes_for(int G) {
   const size_t n = (size_t)G * G + prefilter_sectors(G);
-  return prefilter_lists_offset() + ((n * 8 + 15) / 16) * 16 + n * kPfSlots * sizeof(uint16_t);
+  const size_t gi = (size_t)prefilter_inner(G);
+  return prefilter_lists_offset() + ((n * 8 + 15) / 16) * 16 + n * kPfSlots * sizeof(uint16_t) +
+         gi * gi * 8;
 }
 
 // List n (cells 0..G*G-1, then sectors): head at heads[n] (8 bytes), tail at
@@ -336,12 +363,20 @@ __host__ __device__ inline size_t prefilter_tails_offset(size_t nlists) {
   return prefilter_lists_offset() + ((nlists * 8 + 15) / 16) * 16;
 }
 
+// Inner heads, row-major [Gi][Gi] (16-byte aligned).
+__host__ __device__ inline size_t prefilter_inner_offset(size_t nlists) {
+  return prefilter_tails_offset(nlists) + nlists * kPfSlots * sizeof(uint16_t);
+}
+
 struct PrefilterView {
   float R, inv_h, Gf;
+  float Rih;  // R * inv_h: grid coordinate of p = fma(p, inv_h, Rih)
   int G;  // 0: exhaustive search only
   int NS;
   const uint2* heads;     // [G*G + NS]
   const uint16_t* tails;  // [G*G + NS][32]
+  const uint2* inner;     // [Gi][Gi]
+  int Gi;
 };
 
 // A table built for another codebook size is ignored (exhaustive search), so a
@@ -351,6 +386,7 @@ __device__ __forceinline__ PrefilterView prefilter_view(const void* table, int K
   PrefilterView v;
   v.R = h->R;
   v.inv_h = h->inv_h;
+  v.Rih = h->R * h->inv_h;
   v.G = (h->K == K && h->cap == kPfCap && h->NS == kPfSectors) ? h->G : 0;
   v.NS = h->NS;
   v.Gf = (float)v.G;
@@ -359,6 +395,9 @@ __device__ __forceinline__ PrefilterView prefilter_view(const void* table, int K
                                            prefilter_lists_offset());
   v.tails = reinterpret_cast<const uint16_t*>(reinterpret_cast<const uint8_t*>(table) +
                                               prefilter_tails_offset(nlists));
+  v.inner = reinterpret_cast<const uint2*>(reinterpret_cast<const uint8_t*>(table) +
+                                           prefilter_inner_offset(nlists));
+  v.Gi = v.G > 0 ? h->Gi : 0;
   return v;
 }
 
@@ -399,8 +438,8 @@ constexpr uint32_t kPfNoListBit = 0x8000u;
 __device__ __forceinline__ uint32_t pf_list(float px, float py, const PrefilterView& pf) {
   uint32_t n = kPfNoList;
   if (pf.G > 0) {
-    const float gx = (px + pf.R) * pf.inv_h;
-    const float gy = (py + pf.R) * pf.inv_h;
+    const float gx = fmaf(px, pf.inv_h, pf.Rih);
+    const float gy = fmaf(py, pf.inv_h, pf.Rih);
     if (gx >= 0.f && gx < pf.Gf && gy >= 0.f && gy < pf.Gf) {
       n = (uint32_t)((int)gy * pf.G + (int)gx);
     } else if (isfinite(px) && isfinite(py)) {
@@ -452,12 +491,16 @@ __device__ __forceinline__ int pf_finish2(uint2 h, float px, float py, const flo
   const uint32_t hx = h.x, hy = h.y;
   const uint32_t o0 = hx & 0x3fffu, o1 = hx >> 16, o2 = hy & 0x3fffu, o3 = hy >> 16;
   const uint32_t n4 = (hx >> 14) & 3u;  // min(count, 4) - 1
-  const unsigned char* base = reinterpret_cast<const unsigned char*>(cb);
-  const float e0 = score_cw(m2x, m2y, *reinterpret_cast<const float2*>(base + o0));
-  float e1 = INFINITY, e2 = INFINITY, e3 = INFINITY;
-  if (n4 >= 1u) e1 = score_cw(m2x, m2y, *reinterpret_cast<const float2*>(base + o1));
-  if (n4 >= 2u) e2 = score_cw(m2x, m2y, *reinterpret_cast<const float2*>(base + o2));
-  if (n4 >= 3u) e3 = score_cw(m2x, m2y, *reinterpret_cast<const float2*>(base + o3));
+  const uint32_t base = smem_u32(cb);
+  const float2 z = make_float2(0.f, 0.f);
+  const float2 c0 = lds_f2(base + o0);
+  const float2 c1 = lds_f2_ge<1>(n4, base + o1, z);
+  const float2 c2 = lds_f2_ge<2>(n4, base + o2, z);
+  const float2 c3 = lds_f2_ge<3>(n4, base + o3, z);
+  const float e0 = score_cw(m2x, m2y, c0);
+  const float e1 = n4 >= 1u ? score_cw(m2x, m2y, c1) : INFINITY;
+  const float e2 = n4 >= 2u ? score_cw(m2x, m2y, c2) : INFINITY;
+  const float e3 = n4 >= 3u ? score_cw(m2x, m2y, c3) : INFINITY;
   float ea = e0, eb = e2;
   uint32_t oa = o0, ob = o2;
   if (e1 < ea) {
@@ -475,6 +518,24 @@ __device__ __forceinline__ int pf_finish2(uint2 h, float px, float py, const flo
   if (count) scored += n4 + 1u;
   if (!(hy & (kPfMoreBit | kPfNoListBit))) return (int)(oa >> 3);
   return pf_finish_rare(hx, hy, px, py, m2x, m2y, cb, K, pf, ea, (int)(oa >> 3), scored, count);
+}
+
+// Head of p's list for a caller holding the inner-grid cells [c0, c0 + S)^2
+// in shared memory (hs, row-major S x S): that copy when p falls in it and the
+// union there fits the head, else the main table (a global load).  Both loads
+// are predicated; only points off the grid (or without a table) branch.
+__device__ __forceinline__ uint2 pf_head_shared(float px, float py, const PrefilterView& pf,
+                                                const uint2* hs, int S, int c0) {
+  const float gx = fmaf(px, pf.inv_h, pf.Rih);
+  const float gy = fmaf(py, pf.inv_h, pf.Rih);
+  if (!(gx >= 0.f && gx < pf.Gf && gy >= 0.f && gy < pf.Gf))
+    return pf_head(px, py, pf);  // off the grid, without a table, or not finite
+  const int ix = (int)gx, iy = (int)gy;
+  const unsigned sx = (unsigned)((ix >> 1) - c0), sy = (unsigned)((iy >> 1) - c0);
+  uint2 h = make_uint2(0u, kPfMoreBit);
+  if (sx < (unsigned)S && sy < (unsigned)S) h = hs[sy * S + sx];
+  if (h.y & kPfMoreBit) h = __ldg(pf.heads + (iy * pf.G + ix));
+  return h;
 }
 
 __device__ __forceinline__ int nearest_pf2(float px, float py, const float2* cb, int K,

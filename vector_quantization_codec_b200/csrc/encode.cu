@@ -8,6 +8,7 @@
 //   k_calib_finish  sigma_k = binary16(sum / (n sqrt(pi/2)))        (16 threads/pair)
 //   k_encode        norm, rotate, normalise, nearest codeword, pack  (row groups)
 #include <algorithm>
+#include <cmath>
 
 #include "common.cuh"
 #include "launch.cuh"
@@ -287,6 +288,8 @@ struct EncodeArgs {
   int64_t row_bytes;
   int d_out, d_in, block, K;
   int rows_per_cta;  // R: whole rows per CTA iteration, R * C <= blockDim
+  int hs_side;       // k_encode: inner-grid cells per side copied to shared memory
+  int hs_gi;         // k_encode: inner-grid size the launch was sized for
   uint64_t seed;
 };
 
@@ -328,6 +331,8 @@ __global__ void __launch_bounds__(512, 1) k_encode_wide(const EncodeArgs<T> a) {
   } else {
     pf.G = 0;
     pf.Gf = 0.f;
+    pf.R = 0.f;
+    pf.inv_h = 0.f;
   }
   __syncthreads();
 
@@ -376,7 +381,7 @@ __global__ void __launch_bounds__(512, 1) k_encode_wide(const EncodeArgs<T> a) {
       if (!isfinite(r)) flags |= QAMW_STATUS_NONFINITE;
       else if (isinf(__half2float(h))) flags |= QAMW_STATUS_RANGE;
     }
-    const bool zero = !(r > 0.f);
+    const bool zero = !(r > 0.f) || !isfinite(r);  // zero or not finite (flagged): indices 0
     const float inv = 1.0f / (r * sqrt_b);
     // nearest codeword of each pair, packing as we go; the list head of pair
     // q+1 is fetched while pair q is scored
@@ -387,8 +392,8 @@ __global__ void __launch_bounds__(512, 1) k_encode_wide(const EncodeArgs<T> a) {
       const float np_over_2pi = (float)kNp * 0.159154943f;
 #pragma unroll
       for (int q = 0; q < kQ; ++q) {
-        const float is = isgT[q * C + c];
-        const float px = (x[2 * q] * inv) * is, py = (x[2 * q + 1] * inv) * is;
+        const float f = inv * isgT[q * C + c];
+        const float px = x[2 * q] * f, py = x[2 * q + 1] * f;
         const uint32_t id = zero ? 0u : (uint32_t)polar_index(px, py, lev, kNa, kNp, np_over_2pi);
         scored += kNa;
         const int bit = q * BITS, wi = bit >> 5, sh = bit & 31;
@@ -396,17 +401,17 @@ __global__ void __launch_bounds__(512, 1) k_encode_wide(const EncodeArgs<T> a) {
         if (sh + BITS > 32) w[wi + 1] |= id >> (32 - sh);
       }
     } else {
-      float is = isgT[c];
-      float px = (x[0] * inv) * is, py = (x[1] * inv) * is;
+      const float f0 = inv * isgT[c];
+      float px = x[0] * f0, py = x[1] * f0;
       uint2 cur = pf_head(px, py, pf);
 #pragma unroll
       for (int q = 0; q < kQ; ++q) {
         float nx = 0.f, ny = 0.f;
         uint2 nxt = cur;
         if (q + 1 < kQ) {
-          const float is1 = isgT[(q + 1) * C + c];
-          nx = (x[2 * q + 2] * inv) * is1;
-          ny = (x[2 * q + 3] * inv) * is1;
+          const float f1 = inv * isgT[(q + 1) * C + c];
+          nx = x[2 * q + 2] * f1;
+          ny = x[2 * q + 3] * f1;
           nxt = pf_head(nx, ny, pf);
         }
         const uint32_t id =
@@ -436,28 +441,61 @@ __global__ void __launch_bounds__(512, 1) k_encode_wide(const EncodeArgs<T> a) {
   }
 }
 
-// The same steps in two phases per CTA iteration, so that the 64 rotated
-// values leave the registers before the search:
-//   phase 1  load, scale, sum of squares, butterflies, row norm, normalise;
-//            thread t writes its 32 points to pts[q][t] (its own column of the
-//            buffer: no barrier between the phases, conflict-free accesses);
-//   phase 2  a rolled loop over the 32 points: the list head of point q + 2 is
-//            fetched while point q is scored against the codewords (a plain
-//            (x, y) table, scores bitwise those of k_encode_wide), and the
-//            indices are packed through a 64-bit bit accumulator that emits
-//            each 32-bit word as it fills.
+// The same steps with the list heads in shared memory.  One CTA of R rows x C
+// chunk-threads (at most 512 threads, one CTA per SM).  Each row's C threads
+// synchronise on the row's own named barrier when C is a multiple of 32 (so
+// that rows drift apart and one row's search overlaps another's loads), else
+// on the CTA barrier.  Per row:
+//   load, scale, sum of squares, butterflies; the row norm (every warp of the
+//   row reduces the row's partial sums in one fixed order, so r is bitwise
+//   reproducible);
+//   then in two halves of 16 pairs: normalise into the thread's own column of
+//   the point buffer and search those points in a rolled loop (the list head of
+//   point q + 2 is fetched while point q is scored), packing the indices
+//   through a 64-bit bit accumulator that emits each 32-bit word as it fills.
+// List heads come from a shared copy of the central S x S cells of the table's
+// inner grid (filled by bulk copies while the other tables are built); points
+// outside it, or whose inner list is longer than a head, read the main table.
 // Shared memory: cb2 float2[K] | fT4 float4[16][C] | isg4 float4[8][C] |
-// pts float2[32][T] | part float[T] | rsum float[R].
+// part float[2][T] | rsum float[R] (padded) | pts float2[16][T] | hs uint2[S][S]
+// | bar uint64.
 template <int BITS, typename T, bool POLAR>
 __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const int C = a.d_in / kE, NT = blockDim.x;
+  const int C = a.d_in / kE, NT = blockDim.x, R = a.rows_per_cta;
   float2* cb2 = reinterpret_cast<float2*>(smem);
   float4* fT4 = reinterpret_cast<float4*>(smem + (((size_t)a.K * sizeof(float2) + 15) & ~15));
   float4* isg4 = fT4 + (kE / 4) * C;
-  float2* pts = reinterpret_cast<float2*>(isg4 + (kQ / 4) * C);
-  float* part = reinterpret_cast<float*>(pts + (size_t)kQ * NT);
-  float* rsum = part + NT;
+  float* part = reinterpret_cast<float*>(isg4 + (kQ / 4) * C);  // [2][NT]
+  float* rsum = part + 2 * NT;                                   // [R], padded to 16 bytes
+  float2* pts = reinterpret_cast<float2*>(rsum + ((R + 3) & ~3));  // [16][NT]
+  uint2* hs = reinterpret_cast<uint2*>(pts + (size_t)(kQ / 2) * NT);  // [S][S]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(hs + (size_t)a.hs_side * a.hs_side);
+
+  PrefilterView pf;
+  if (a.prefilter != nullptr) {
+    pf = prefilter_view(a.prefilter, a.K);
+  } else {
+    pf.G = 0;
+    pf.Gf = 0.f;
+    pf.R = 0.f;
+    pf.inv_h = 0.f;
+    pf.Gi = 0;
+  }
+  // the shared copy of the inner grid: its table must be the one the launch
+  // was sized for (a table for another codebook size reads as none)
+  const int S = (!POLAR && pf.G > 0 && pf.Gi == a.hs_gi) ? a.hs_side : 0;
+  const int c0 = (pf.Gi - S) / 2;
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (S > 0) {
+    if (threadIdx.x == 0) mbar_expect_tx(bar, (unsigned)(S * S * 8));
+    for (int r = threadIdx.x; r < S; r += NT)
+      bulk_g2s(hs + (size_t)r * S, pf.inner + (size_t)(c0 + r) * pf.Gi + c0, (unsigned)(S * 8), bar);
+  }
   constexpr int kBa = BITS / 2, kNa = 1 << kBa, kNp = 1 << (BITS - kBa);
   float* lev = reinterpret_cast<float*>(cb2);
   if constexpr (POLAR) {
@@ -471,38 +509,36 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
     return mask_negative(seed, (uint32_t)j) ? -v : v;
   });
   fill_quads<kQ>(isg4, a.sigma, a.d_in / 2, C, [](int, float v) { return 1.0f / v; });
-  PrefilterView pf;
-  if (a.prefilter != nullptr) {
-    pf = prefilter_view(a.prefilter, a.K);
-  } else {
-    pf.G = 0;
-    pf.Gf = 0.f;
-  }
   __syncthreads();
-
-  const int R = a.rows_per_cta;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = NT >> 5;
-  // W of row group r0 (R rows from r0, clipped to the matrix) into L2
-  auto prefetch_rows = [&](int64_t r0) {
-    if (threadIdx.x == 0 && r0 < a.d_out) {
-      const int64_t nr = min((int64_t)R, (int64_t)a.d_out - r0);
-      bulk_prefetch_l2(a.W + r0 * a.d_in, (unsigned)(nr * a.d_in * (int64_t)sizeof(T)));
+  int flags = 0;
+  if (S > 0) {
+    const bool ok = mbar_wait_bounded(bar, 0);
+    if (__syncthreads_or(!ok)) {  // the copies never landed: give up, after one more bounded wait
+      if (threadIdx.x == 0) mbar_wait_bounded(bar, 0);
+      raise_flag(a.status, QAMW_STATUS_TIMEOUT);
+      return;
     }
-  };
-  prefetch_rows((int64_t)blockIdx.x * R);
+  }
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = NT >> 5;
   const int rl = threadIdx.x / C, c = threadIdx.x - rl * C;
+  const bool per_row = (C % 32) == 0;  // a row is whole warps: it has its own barrier
   const int nb = min(a.block, kE), lanes = max(a.block / kE, 1);
   const float sqrt_b = sqrtf((float)a.block);
-  float2* mypts = pts + threadIdx.x;
-  int flags = 0;
-  unsigned scored = 0;
   const bool count = a.candidates != nullptr;
+  float2* mypts = pts + threadIdx.x;
+  unsigned scored = 0;
+  int buf = 0;
   for (int64_t r0 = (int64_t)blockIdx.x * R; r0 < a.d_out; r0 += (int64_t)gridDim.x * R) {
     const int64_t row = r0 + rl;
     const bool active = rl < R && row < a.d_out;
+    if (per_row && !active) continue;  // the row's threads all skip, barrier included
     float x[kE];
     float ss = 0.f;
     if (active) {
+      if (c == 0 && row + (int64_t)gridDim.x * R < a.d_out)  // this row's next one, into L2
+        bulk_prefetch_l2(a.W + (row + (int64_t)gridDim.x * R) * a.d_in,
+                         (unsigned)(a.d_in * (int64_t)sizeof(T)));
       load64(a.W + row * a.d_in + (int64_t)c * kE, x);
 #pragma unroll
       for (int i = 0; i < kE / 4; ++i) {
@@ -520,22 +556,34 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
 #pragma unroll
       for (int j = 0; j < kE; ++j) x[j] = 0.f;
     }
-    part[threadIdx.x] = ss;
+    float* pb = part + buf * NT;
+    buf ^= 1;
+    pb[threadIdx.x] = ss;
     fwht_reg<kE>(x, nb);
     fwht_lanes<kE>(x, lanes);
-    __syncthreads();
-    for (int q = warp; q < R; q += nwarps) {
+    float r;
+    if (per_row) {
+      // the row's partial sums: double-buffered, so one barrier per row suffices
+      asm volatile("bar.sync %0, %1;" ::"r"(1 + rl), "r"(C) : "memory");
       float t = 0.f;
-      for (int k = lane; k < C; k += 32) t += part[q * C + k];
+      for (int k = lane; k < C; k += 32) t += pb[rl * C + k];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-      if (lane == 0) rsum[q] = sqrtf(t);
+      r = sqrtf(t);
+    } else {
+      __syncthreads();
+      for (int q = warp; q < R; q += nwarps) {
+        float t = 0.f;
+        for (int k = lane; k < C; k += 32) t += pb[q * C + k];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        if (lane == 0) rsum[q] = sqrtf(t);
+      }
+      __syncthreads();
+      if (!active) continue;
+      r = rsum[rl];
     }
-    __syncthreads();
-    prefetch_rows(r0 + (int64_t)gridDim.x * R);  // the next row group, during the search
-    if (!active) continue;
 
-    const float r = rsum[rl];
     if (c == 0) {
       const __half h = __float2half_rn(r);
       a.rnorm[row] = h;
@@ -543,59 +591,34 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
       else if (isinf(__half2float(h))) flags |= QAMW_STATUS_RANGE;
     }
     uint32_t* dst = reinterpret_cast<uint32_t*>(a.packed + row * a.row_bytes) + (size_t)c * BITS;
-    if (!(r > 0.f)) {  // zero row: every index 0
+    if (!(r > 0.f) || !isfinite(r)) {  // zero row, or not finite (flagged): every index 0
 #pragma unroll
       for (int t = 0; t < BITS; ++t) dst[t] = 0u;
     } else {
       const float inv = 1.0f / (r * sqrt_b);
-#pragma unroll
-      for (int i = 0; i < kQ / 4; ++i) {
-        const float4 is = isg4[i * C + c];
-        mypts[(4 * i + 0) * NT] = make_float2((x[8 * i + 0] * inv) * is.x, (x[8 * i + 1] * inv) * is.x);
-        mypts[(4 * i + 1) * NT] = make_float2((x[8 * i + 2] * inv) * is.y, (x[8 * i + 3] * inv) * is.y);
-        mypts[(4 * i + 2) * NT] = make_float2((x[8 * i + 4] * inv) * is.z, (x[8 * i + 5] * inv) * is.z);
-        mypts[(4 * i + 3) * NT] = make_float2((x[8 * i + 6] * inv) * is.w, (x[8 * i + 7] * inv) * is.w);
-      }
       uint64_t acc = 0;
       int nbits = 0;
-      if constexpr (POLAR) {
-        const float np_over_2pi = (float)kNp * 0.159154943f;
-#pragma unroll 1
-        for (int q = 0; q < kQ; ++q) {
-          const float2 p = mypts[q * NT];
-          const uint32_t id = (uint32_t)polar_index(p.x, p.y, lev, kNa, kNp, np_over_2pi);
-          scored += kNa;
-          acc |= (uint64_t)id << nbits;
-          nbits += BITS;
-          if (nbits >= 32) {
-            *dst++ = (uint32_t)acc;
-            acc >>= 32;
-            nbits -= 32;
-          }
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        // normalise pairs 16 hf .. 16 hf + 15 into the point buffer
+#pragma unroll
+        for (int i = 0; i < kQ / 8; ++i) {
+          const float4 is = isg4[(hf * (kQ / 8) + i) * C + c];
+          const int q0 = hf * (kQ / 2) + 4 * i;
+          // p_k = z_k / sigma_k with z = y / (r sqrt(b)): one factor per pair
+          const float f0 = inv * is.x, f1 = inv * is.y, f2 = inv * is.z, f3 = inv * is.w;
+          mypts[(4 * i + 0) * NT] = make_float2(x[2 * q0 + 0] * f0, x[2 * q0 + 1] * f0);
+          mypts[(4 * i + 1) * NT] = make_float2(x[2 * q0 + 2] * f1, x[2 * q0 + 3] * f1);
+          mypts[(4 * i + 2) * NT] = make_float2(x[2 * q0 + 4] * f2, x[2 * q0 + 5] * f2);
+          mypts[(4 * i + 3) * NT] = make_float2(x[2 * q0 + 6] * f3, x[2 * q0 + 7] * f3);
         }
-      } else {
-        // list heads of kGrp points are fetched one group ahead of their
-        // scoring, so that the L2 latency of a head load is hidden
-        constexpr int kGrp = 4;
-        uint2 hc[kGrp], hn[kGrp];
-#pragma unroll
-        for (int k = 0; k < kGrp; ++k) {
-          const float2 p = mypts[k * NT];
-          hc[k] = pf_head(p.x, p.y, pf);
-        }
+        if constexpr (POLAR) {
+          const float np_over_2pi = (float)kNp * 0.159154943f;
 #pragma unroll 1
-        for (int g = 0; g < kQ / kGrp; ++g) {
-          if (g + 1 < kQ / kGrp) {
-#pragma unroll
-            for (int k = 0; k < kGrp; ++k) {
-              const float2 p = mypts[((g + 1) * kGrp + k) * NT];
-              hn[k] = pf_head(p.x, p.y, pf);
-            }
-          }
-#pragma unroll
-          for (int k = 0; k < kGrp; ++k) {
-            const float2 p = mypts[(g * kGrp + k) * NT];
-            const uint32_t id = (uint32_t)pf_finish2(hc[k], p.x, p.y, cb2, a.K, pf, scored, count);
+          for (int q = 0; q < kQ / 2; ++q) {
+            const float2 p = mypts[q * NT];
+            const uint32_t id = (uint32_t)polar_index(p.x, p.y, lev, kNa, kNp, np_over_2pi);
+            scored += kNa;
             acc |= (uint64_t)id << nbits;
             nbits += BITS;
             if (nbits >= 32) {
@@ -604,8 +627,27 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
               nbits -= 32;
             }
           }
-#pragma unroll
-          for (int k = 0; k < kGrp; ++k) hc[k] = hn[k];
+        } else {
+          float2 p = mypts[0];
+          uint2 h0 = pf_head_shared(p.x, p.y, pf, hs, S, c0);
+          p = mypts[NT];
+          uint2 h1 = pf_head_shared(p.x, p.y, pf, hs, S, c0);
+#pragma unroll 1
+          for (int q = 0; q < kQ / 2; ++q) {
+            p = mypts[min(q + 2, kQ / 2 - 1) * NT];
+            const uint2 h2 = pf_head_shared(p.x, p.y, pf, hs, S, c0);
+            p = mypts[q * NT];
+            const uint32_t id = (uint32_t)pf_finish2(h0, p.x, p.y, cb2, a.K, pf, scored, count);
+            acc |= (uint64_t)id << nbits;
+            nbits += BITS;
+            if (nbits >= 32) {
+              *dst++ = (uint32_t)acc;
+              acc >>= 32;
+              nbits -= 32;
+            }
+            h0 = h1;
+            h1 = h2;
+          }
         }
       }
     }
@@ -644,48 +686,39 @@ void encode_shape(int C, int* R_out, int* threads_out) {
   *threads_out = bestT;
 }
 
-size_t encode_staged_smem(int K, int d_in, int T, int R) {
-  return (((size_t)K * sizeof(float2) + 15) & ~(size_t)15) + (size_t)d_in * sizeof(float) +
-         (size_t)(d_in / 2) * sizeof(float) + (size_t)T * kQ * sizeof(float2) +
-         (size_t)T * sizeof(float) + (size_t)R * sizeof(float);
-}
-
-// k_encode's shape: the R (rows per CTA iteration, R * C <= 512 threads) that
-// keeps the most busy threads resident per SM (228 KB of shared memory, 512
-// threads at <= 128 registers); ties go to the smaller CTA.  Returns false when
-// not even one row fits.
-bool encode_staged_shape(int C, int K, int d_in, int* R_out, int* threads_out, size_t* smem_out) {
-  int bestR = 0, bestT = 0;
-  size_t bestS = 0;
-  long best = -1;
-  for (int R = 1; R * C <= 512; ++R) {
-    const int T = ((R * C + 31) / 32) * 32;
-    const size_t sm = encode_staged_smem(K, d_in, T, R);
-    if (sm > 227 * 1024) break;
-    const int by_smem = (int)((228 * 1024) / (sm + 1024));
-    const int ctas = std::min(by_smem, 512 / T);
-    const long busy = (long)ctas * R * C;
-    if (ctas >= 1 && busy > best) {
-      best = busy;
-      bestR = R;
-      bestT = T;
-      bestS = sm;
-    }
-  }
-  if (bestR == 0) return false;
-  *R_out = bestR;
-  *threads_out = bestT;
-  *smem_out = bestS;
+// k_encode's shape: R rows of C chunk-threads (at most 15 rows -- one named
+// barrier each -- and 512 threads, one CTA per SM) and the side S of the shared
+// copy of the inner grid, the largest multiple of 4 that fits next to the other
+// tables (at most the inner grid).  Returns false when the tables and the
+// point buffer alone do not fit (very wide rows: k_encode_wide).
+bool encode_shared_shape(int C, int K, int d_in, int gi, int* R_out, int* threads_out,
+                         int* side_out, size_t* smem_out) {
+  const int R = std::max(1, std::min(15, 512 / C));
+  const int T = ((R * C + 31) / 32) * 32;
+  const size_t base = (((size_t)K * sizeof(float2) + 15) & ~(size_t)15) +
+                      (size_t)d_in * sizeof(float) + (size_t)(d_in / 2) * sizeof(float) +
+                      2 * (size_t)T * sizeof(float) + (size_t)((R + 3) & ~3) * sizeof(float) +
+                      (size_t)(kQ / 2) * T * sizeof(float2) + sizeof(uint64_t);
+  const size_t cap = 227 * 1024;
+  if (R * C > 512 || base > cap) return false;
+  int S = (int)std::sqrt((double)(cap - base) / 8.0);
+  S = std::min(S, gi) & ~3;
+  if (S < 8) S = 0;
+  *R_out = R;
+  *threads_out = T;
+  *side_out = S;
+  *smem_out = base + (size_t)S * S * 8;
   return true;
 }
 
 template <int BITS, typename T, bool POLAR>
 cudaError_t run_encode(EncodeArgs<T> a, cudaStream_t stream) {
   const int C = a.d_in / kE;
-  int R, threads;
+  const int gi = (a.prefilter != nullptr && !POLAR) ? prefilter_inner(prefilter_grid(BITS)) : 0;
+  int R, threads, side = 0;
   size_t smem;
   const void* fn;
-  if (encode_staged_shape(C, a.K, a.d_in, &R, &threads, &smem)) {
+  if (encode_shared_shape(C, a.K, a.d_in, gi, &R, &threads, &side, &smem)) {
     fn = reinterpret_cast<const void*>(&k_encode<BITS, T, POLAR>);
   } else {
     encode_shape(C, &R, &threads);
@@ -695,6 +728,8 @@ cudaError_t run_encode(EncodeArgs<T> a, cudaStream_t stream) {
     fn = reinterpret_cast<const void*>(&k_encode_wide<BITS, T, POLAR>);
   }
   a.rows_per_cta = R;
+  a.hs_side = side;
+  a.hs_gi = gi;
   cudaError_t err = allow_smem(fn, smem);
   if (err != cudaSuccess) return err;
   const int grid = persistent_grid(fn, threads, smem, (a.d_out + R - 1) / R);
@@ -721,6 +756,8 @@ cudaError_t encode_rows_typed(const T* W, const qamw_matrix& m, int32_t* st,
   a.block = m.block;
   a.K = 1 << m.bits;
   a.rows_per_cta = 1;
+  a.hs_side = 0;
+  a.hs_gi = 0;
   a.seed = m.mask_seed;
   switch (m.bits) {
     case 1: return run_encode<1, T, POLAR>(a, stream);

@@ -50,6 +50,7 @@ __global__ void __launch_bounds__(1024) k_pf_header(const float2* __restrict__ c
     h.cap = kPfCap;
     h.K = K;
     h.NS = G > 0 ? kPfSectors : 0;
+    h.Gi = prefilter_inner(G);
     *hdr = h;
   }
 }
@@ -82,6 +83,51 @@ __device__ void write_list(void* table, size_t nlists, size_t n, bool overflow, 
     *reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(table) + prefilter_lists_offset() +
                               n * 8) = h;
   }
+}
+
+// Inner grid, one thread per cell: the ascending union of the four child
+// lists, or the "more" bit (more than 4 candidates, or an overflowed child).
+__global__ void __launch_bounds__(256) k_pf_inner(void* __restrict__ table) {
+  const PrefilterHeader hdr = *reinterpret_cast<const PrefilterHeader*>(table);
+  const int G = hdr.G, Gi = hdr.Gi;
+  const int cell = blockIdx.x * blockDim.x + threadIdx.x;
+  if (cell >= Gi * Gi) return;
+  const int ix = cell % Gi, iy = cell / Gi;
+  const size_t nlists = (size_t)G * G + hdr.NS;
+  const uint16_t* tails = reinterpret_cast<const uint16_t*>(
+      reinterpret_cast<const uint8_t*>(table) + prefilter_tails_offset(nlists));
+  uint32_t u[kPfHeadSlots];
+  int m = 0;
+  bool more = false;
+  for (int d = 0; d < 4 && !more; ++d) {
+    const size_t n = (size_t)(2 * iy + (d >> 1)) * G + (2 * ix + (d & 1));
+    const uint16_t* t = tails + n * kPfSlots;
+    const uint32_t cnt = t[0];
+    if (cnt == kPfOverflow || cnt == 0u) {
+      more = true;
+      break;
+    }
+    for (uint32_t k = 1; k <= cnt && !more; ++k) {
+      const uint32_t v = t[k];
+      int pos = 0;
+      while (pos < m && u[pos] < v) ++pos;
+      if (pos < m && u[pos] == v) continue;
+      if (m == kPfHeadSlots) {
+        more = true;
+        break;
+      }
+      for (int q = m; q > pos; --q) u[q] = u[q - 1];
+      u[pos] = v;
+      ++m;
+    }
+  }
+  uint32_t slot[kPfHeadSlots];
+  for (int t = 0; t < kPfHeadSlots; ++t) slot[t] = more ? 0u : ((t < m ? u[t] : u[0]) << 3) & 0x3fffu;
+  slot[0] |= (uint32_t)((more ? kPfHeadSlots : m) - 1) << 14;
+  if (more) slot[2] |= kPfMoreBit;
+  uint2* inner = reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(table) +
+                                          prefilter_inner_offset(nlists));
+  inner[cell] = make_uint2(slot[0] | (slot[1] << 16), slot[2] | (slot[3] << 16));
 }
 
 // One warp per cell.
@@ -322,6 +368,9 @@ cudaError_t launch_build_prefilter(const float* d_codebook, int bits, int G, voi
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   const int NS = prefilter_sectors(G);
   k_pf_sectors<<<(NS + kBuildWarps - 1) / kBuildWarps, kBuildWarps * 32, 0, stream>>>(cb, d_table);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  const int Gi = prefilter_inner(G);
+  if (Gi > 0) k_pf_inner<<<(Gi * Gi + 255) / 256, 256, 0, stream>>>(d_table);
   return cudaGetLastError();
 }
 

@@ -66,6 +66,8 @@ __global__ void __launch_bounds__(512) k_assign(const float2* __restrict__ sampl
   } else {
     pf.G = 0;
     pf.Gf = 0.f;
+    pf.R = 0.f;
+    pf.inv_h = 0.f;
   }
   __syncthreads();
   int flags = 0;
