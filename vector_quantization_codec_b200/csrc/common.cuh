@@ -226,16 +226,20 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 
 // Shared-memory loads at a 32-bit shared address (base + byte offset), so
 // that gathers need no 64-bit address arithmetic.  lds_f2_ge loads only when
-// n >= k (a predicated load), else keeps v.
+// n >= k (a predicated load).
 __device__ __forceinline__ float2 lds_f2(uint32_t addr) {
   float2 v;
-  asm("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
   return v;
 }
 
 template <int k>
-__device__ __forceinline__ float2 lds_f2_ge(uint32_t n, uint32_t addr, float2 v) {
-  asm("{\n .reg .pred q;\n setp.ge.u32 q, %2, %3;\n @q ld.shared.v2.f32 {%0, %1}, [%4];\n}"
+__device__ __forceinline__ float2 lds_f2_ge(uint32_t n, uint32_t addr) {
+  // a defined value for lanes that skip the load: a predicated write to an
+  // undefined register would keep that register live back to its first use
+  float2 v = make_float2(0.f, 0.f);
+  asm volatile(
+      "{\n .reg .pred q;\n setp.ge.u32 q, %2, %3;\n @q ld.shared.v2.f32 {%0, %1}, [%4];\n}"
       : "+f"(v.x), "+f"(v.y)
       : "r"(n), "n"(k), "r"(addr));
   return v;
@@ -456,15 +460,52 @@ __device__ __forceinline__ uint2 pf_head(float px, float py, const PrefilterView
   return n == kPfNoList ? make_uint2(0u, kPfNoListBit) : __ldg(pf.heads + n);
 }
 
-// Rare ends of pf_finish2: a list longer than the head (its tail continues
-// from slot 5 with the best of the head as the incumbent), an overflowed list
-// or a point without one (exhaustive search).
-__device__ __forceinline__ int pf_finish_rare(uint32_t hx, uint32_t hy, float px, float py,
-                                              float m2x, float m2y, const float2* cb, int K,
+// The four head slots of a list scored against p (m2 = -2 p): slot t is
+// loaded only when t < min(count, 4) (a predicated shared load: lanes with
+// short lists add no traffic) and otherwise scores +inf; the minimum is taken
+// as a tree in which the left operand wins ties (the slots hold ascending
+// indices).  Returns the best score and its byte offset.
+__device__ __forceinline__ void pf_score_head(uint2 h, float m2x, float m2y, uint32_t base,
+                                              float& ea, uint32_t& oa) {
+  const uint32_t hx = h.x, hy = h.y;
+  const uint32_t o0 = hx & 0x3fffu, o1 = hx >> 16, o2 = hy & 0x3fffu, o3 = hy >> 16;
+  const uint32_t n4 = (hx >> 14) & 3u;  // min(count, 4) - 1
+  const float e0 = score_cw(m2x, m2y, lds_f2(base + o0));
+  const float s1 = score_cw(m2x, m2y, lds_f2_ge<1>(n4, base + o1));
+  const float s2 = score_cw(m2x, m2y, lds_f2_ge<2>(n4, base + o2));
+  const float s3 = score_cw(m2x, m2y, lds_f2_ge<3>(n4, base + o3));
+  const float e1 = n4 >= 1u ? s1 : INFINITY;
+  const float e2 = n4 >= 2u ? s2 : INFINITY;
+  const float e3 = n4 >= 3u ? s3 : INFINITY;
+  float eb = e2;
+  uint32_t ob = o2;
+  ea = e0;
+  oa = o0;
+  if (e1 < ea) {
+    ea = e1;
+    oa = o1;
+  }
+  if (e3 < eb) {
+    eb = e3;
+    ob = o3;
+  }
+  if (eb < ea) {
+    ea = eb;
+    oa = ob;
+  }
+}
+
+// Rare ends of pf_finish2, for a head with the "more" or the no-list bit: a
+// list longer than the head continues in its tail (the point's list n,
+// recomputed) from slot 5 with the best of the head as the incumbent; an
+// overflowed list or a point without a list (no table, or not finite) is
+// searched exhaustively.
+__device__ __forceinline__ int pf_finish_rare(uint2 h, float px, float py, const float2* cb, int K,
                                               const PrefilterView& pf, float be, int bi,
                                               unsigned& scored, bool count) {
-  const uint32_t head_cnt = ((hx >> 14) & 3u) + 1u;
-  if (hy & kPfNoListBit) {
+  const float m2x = -2.f * px, m2y = -2.f * py;
+  const uint32_t head_cnt = ((h.x >> 14) & 3u) + 1u;
+  if (h.y & kPfNoListBit) {
     if (count) scored -= head_cnt;
     return nearest_all2(m2x, m2y, cb, K, scored);
   }
@@ -480,62 +521,48 @@ __device__ __forceinline__ int pf_finish_rare(uint32_t hx, uint32_t hy, float px
 }
 
 // Nearest codeword of p from its list head; the same index as nearest_all2.
-// Slot t of the head is scored when t < min(count, 4) -- a predicated shared
-// load, so that lanes with short lists add no traffic -- and the others score
-// +inf; the minimum of the four is taken as a tree in which the left operand
-// wins ties (the slots hold ascending indices).  With `count`, `scored`
-// accumulates the distinct candidates of each list.
+// With `count`, `scored` accumulates the distinct candidates of each list.
 __device__ __forceinline__ int pf_finish2(uint2 h, float px, float py, const float2* cb, int K,
                                           const PrefilterView& pf, unsigned& scored, bool count) {
-  const float m2x = -2.f * px, m2y = -2.f * py;
-  const uint32_t hx = h.x, hy = h.y;
-  const uint32_t o0 = hx & 0x3fffu, o1 = hx >> 16, o2 = hy & 0x3fffu, o3 = hy >> 16;
-  const uint32_t n4 = (hx >> 14) & 3u;  // min(count, 4) - 1
-  const uint32_t base = smem_u32(cb);
-  const float2 z = make_float2(0.f, 0.f);
-  const float2 c0 = lds_f2(base + o0);
-  const float2 c1 = lds_f2_ge<1>(n4, base + o1, z);
-  const float2 c2 = lds_f2_ge<2>(n4, base + o2, z);
-  const float2 c3 = lds_f2_ge<3>(n4, base + o3, z);
-  const float e0 = score_cw(m2x, m2y, c0);
-  const float e1 = n4 >= 1u ? score_cw(m2x, m2y, c1) : INFINITY;
-  const float e2 = n4 >= 2u ? score_cw(m2x, m2y, c2) : INFINITY;
-  const float e3 = n4 >= 3u ? score_cw(m2x, m2y, c3) : INFINITY;
-  float ea = e0, eb = e2;
-  uint32_t oa = o0, ob = o2;
-  if (e1 < ea) {
-    ea = e1;
-    oa = o1;
-  }
-  if (e3 < eb) {
-    eb = e3;
-    ob = o3;
-  }
-  if (eb < ea) {
-    ea = eb;
-    oa = ob;
-  }
-  if (count) scored += n4 + 1u;
-  if (!(hy & (kPfMoreBit | kPfNoListBit))) return (int)(oa >> 3);
-  return pf_finish_rare(hx, hy, px, py, m2x, m2y, cb, K, pf, ea, (int)(oa >> 3), scored, count);
+  float ea;
+  uint32_t oa;
+  pf_score_head(h, -2.f * px, -2.f * py, smem_u32(cb), ea, oa);
+  if (count) scored += ((h.x >> 14) & 3u) + 1u;
+  if (!(h.y & (kPfMoreBit | kPfNoListBit))) return (int)(oa >> 3);
+  return pf_finish_rare(h, px, py, cb, K, pf, ea, (int)(oa >> 3), scored, count);
+}
+
+// pf_finish2's common path alone: the index, or kPfRare when the head has the
+// "more" or the no-list bit (the caller then runs the full search apart from
+// its hot loop).  Counts only what it resolves.
+constexpr uint32_t kPfRare = 0xffffffffu;
+__device__ __forceinline__ uint32_t pf_finish_fast(uint2 h, float px, float py, uint32_t cb_s,
+                                                   unsigned& scored, bool count) {
+  float ea;
+  uint32_t oa;
+  pf_score_head(h, -2.f * px, -2.f * py, cb_s, ea, oa);
+  const bool rare = (h.y & (kPfMoreBit | kPfNoListBit)) != 0u;
+  if (count && !rare) scored += ((h.x >> 14) & 3u) + 1u;
+  return rare ? kPfRare : (oa >> 3);
 }
 
 // Head of p's list for a caller holding the inner-grid cells [c0, c0 + S)^2
 // in shared memory (hs, row-major S x S): that copy when p falls in it and the
-// union there fits the head, else the main table (a global load).  Both loads
-// are predicated; only points off the grid (or without a table) branch.
+// union there fits the head, else the main table (a predicated global load).
+// Without a branch: a point off the grid (or without a table, or not finite)
+// gets the no-list head, which the caller resolves with the full search.
 __device__ __forceinline__ uint2 pf_head_shared(float px, float py, const PrefilterView& pf,
                                                 const uint2* hs, int S, int c0) {
   const float gx = fmaf(px, pf.inv_h, pf.Rih);
   const float gy = fmaf(py, pf.inv_h, pf.Rih);
-  if (!(gx >= 0.f && gx < pf.Gf && gy >= 0.f && gy < pf.Gf))
-    return pf_head(px, py, pf);  // off the grid, without a table, or not finite
-  const int ix = (int)gx, iy = (int)gy;
+  const bool in_grid = (gx >= 0.f) & (gx < pf.Gf) & (gy >= 0.f) & (gy < pf.Gf);
+  const int ix = in_grid ? (int)gx : 0, iy = in_grid ? (int)gy : 0;
   const unsigned sx = (unsigned)((ix >> 1) - c0), sy = (unsigned)((iy >> 1) - c0);
+  const bool in_sq = in_grid & (sx < (unsigned)S) & (sy < (unsigned)S);
   uint2 h = make_uint2(0u, kPfMoreBit);
-  if (sx < (unsigned)S && sy < (unsigned)S) h = hs[sy * S + sx];
-  if (h.y & kPfMoreBit) h = __ldg(pf.heads + (iy * pf.G + ix));
-  return h;
+  if (in_sq) h = hs[sy * S + sx];
+  if (in_grid & ((h.y & kPfMoreBit) != 0u)) h = __ldg(pf.heads + (iy * pf.G + ix));
+  return in_grid ? h : make_uint2(0u, kPfNoListBit);
 }
 
 __device__ __forceinline__ int nearest_pf2(float px, float py, const float2* cb, int K,

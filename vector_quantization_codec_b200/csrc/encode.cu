@@ -596,8 +596,13 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
       for (int t = 0; t < BITS; ++t) dst[t] = 0u;
     } else {
       const float inv = 1.0f / (r * sqrt_b);
-      uint64_t acc = 0;
-      int nbits = 0;
+      // each index goes to the first word of its point's slot once the point
+      // has been read; the 16 indices of a half are then packed with fixed
+      // shifts (LSB first, index k at bits [k BITS, (k + 1) BITS))
+      uint32_t* myid = reinterpret_cast<uint32_t*>(mypts);
+      uint32_t w[BITS];
+#pragma unroll
+      for (int t = 0; t < BITS; ++t) w[t] = 0u;
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         // normalise pairs 16 hf .. 16 hf + 15 into the point buffer
@@ -614,42 +619,60 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
         }
         if constexpr (POLAR) {
           const float np_over_2pi = (float)kNp * 0.159154943f;
-#pragma unroll 1
+#pragma unroll 4
           for (int q = 0; q < kQ / 2; ++q) {
             const float2 p = mypts[q * NT];
-            const uint32_t id = (uint32_t)polar_index(p.x, p.y, lev, kNa, kNp, np_over_2pi);
+            myid[q * 2 * NT] = (uint32_t)polar_index(p.x, p.y, lev, kNa, kNp, np_over_2pi);
             scored += kNa;
-            acc |= (uint64_t)id << nbits;
-            nbits += BITS;
-            if (nbits >= 32) {
-              *dst++ = (uint32_t)acc;
-              acc >>= 32;
-              nbits -= 32;
-            }
           }
         } else {
+          // the list heads of points q + 2, q + 3 are fetched while q, q + 1
+          // are scored; a resolved point's slot becomes (index, ~0), a point
+          // that needs the full search keeps its slot and is found below
+          const uint32_t cb_s = smem_u32(cb2);
+          uint32_t rare = 0;
           float2 p = mypts[0];
-          uint2 h0 = pf_head_shared(p.x, p.y, pf, hs, S, c0);
+          uint2 ha = pf_head_shared(p.x, p.y, pf, hs, S, c0);
           p = mypts[NT];
-          uint2 h1 = pf_head_shared(p.x, p.y, pf, hs, S, c0);
+          uint2 hb = pf_head_shared(p.x, p.y, pf, hs, S, c0);
 #pragma unroll 1
-          for (int q = 0; q < kQ / 2; ++q) {
+          for (int q = 0; q < kQ / 2; q += 2) {
             p = mypts[min(q + 2, kQ / 2 - 1) * NT];
-            const uint2 h2 = pf_head_shared(p.x, p.y, pf, hs, S, c0);
+            const uint2 hc = pf_head_shared(p.x, p.y, pf, hs, S, c0);
+            p = mypts[min(q + 3, kQ / 2 - 1) * NT];
+            const uint2 hd = pf_head_shared(p.x, p.y, pf, hs, S, c0);
             p = mypts[q * NT];
-            const uint32_t id = (uint32_t)pf_finish2(h0, p.x, p.y, cb2, a.K, pf, scored, count);
-            acc |= (uint64_t)id << nbits;
-            nbits += BITS;
-            if (nbits >= 32) {
-              *dst++ = (uint32_t)acc;
-              acc >>= 32;
-              nbits -= 32;
+            uint32_t id = pf_finish_fast(ha, p.x, p.y, cb_s, scored, count);
+            rare |= id;
+            if (id != kPfRare) reinterpret_cast<uint2*>(mypts)[q * NT] = make_uint2(id, ~0u);
+            p = mypts[(q + 1) * NT];
+            id = pf_finish_fast(hb, p.x, p.y, cb_s, scored, count);
+            rare |= id;
+            if (id != kPfRare) reinterpret_cast<uint2*>(mypts)[(q + 1) * NT] = make_uint2(id, ~0u);
+            ha = hc;
+            hb = hd;
+          }
+          // points off the grid, lists longer than a head, or no list
+          if (__any_sync(__activemask(), (rare >> 31) != 0u)) {
+#pragma unroll 1
+            for (int k = 0; k < kQ / 2; ++k) {
+              const uint2 v = reinterpret_cast<const uint2*>(mypts)[k * NT];
+              if (v.y != ~0u)
+                myid[k * 2 * NT] = (uint32_t)nearest_pf2(__uint_as_float(v.x), __uint_as_float(v.y),
+                                                         cb2, a.K, pf, scored, count);
             }
-            h0 = h1;
-            h1 = h2;
           }
         }
+#pragma unroll
+        for (int k = 0; k < kQ / 2; ++k) {
+          const uint32_t id = myid[k * 2 * NT];
+          const int bit = (hf * (kQ / 2) + k) * BITS, wi = bit >> 5, sh = bit & 31;
+          w[wi] |= id << sh;
+          if (sh + BITS > 32) w[wi + 1] |= id >> (32 - sh);
+        }
       }
+#pragma unroll
+      for (int t = 0; t < BITS; ++t) dst[t] = w[t];
     }
     if (c == C - 1) {  // zero the row's padding words
       for (int64_t o = (int64_t)C * BITS * 4; o < a.row_bytes; o += 4)
