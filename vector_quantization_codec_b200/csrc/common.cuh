@@ -111,6 +111,23 @@ __device__ __forceinline__ uint32_t extract_idx(const uint32_t (&w)[BITS]) {
     return __funnelshift_r(w[wi], w[wi + 1], sh) & mask;
 }
 
+// Index Q of a chunk as a byte offset into a table of 8-byte entries
+// (8 x index): one shift and one mask (a funnel shift first when the index
+// straddles two words).
+template <int BITS, int Q>
+__device__ __forceinline__ uint32_t extract_off8(const uint32_t (&w)[BITS]) {
+  constexpr int bit = Q * BITS, wi = bit >> 5, sh = bit & 31;
+  constexpr uint32_t mask = ((1u << BITS) - 1u) << 3;
+  if constexpr (sh + BITS <= 32) {
+    if constexpr (sh >= 3)
+      return (w[wi] >> (sh - 3)) & mask;
+    else
+      return (w[wi] << (3 - sh)) & mask;
+  } else {
+    return (__funnelshift_r(w[wi], w[wi + 1], sh) << 3) & mask;
+  }
+}
+
 template <int BITS>
 __device__ __forceinline__ void pack32(const uint32_t (&idx)[kQ], uint32_t (&w)[BITS]) {
 #pragma unroll
@@ -287,7 +304,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity) {
   for (unsigned i = 0; i < kSpinLimit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    __nanosleep(256);
+    if (i >= 64) __nanosleep(256);  // poll at first: copies usually land within a few tries
   }
   return false;
 }

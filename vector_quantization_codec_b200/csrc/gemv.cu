@@ -26,7 +26,7 @@ namespace {
 
 // ------------------------------------------------------------------ batch 1
 
-constexpr int kGemvStages = 4;
+constexpr int kGemvStages = 3;
 
 struct Gemv1Args {
   const uint8_t* packed;
@@ -66,9 +66,13 @@ __device__ __forceinline__ void dot_pairs(const uint32_t (&w)[BITS], const uint3
       ...);
 }
 
+// Region 0: the fp16x2 codebook table [K][copies], then xbar [64][C] (chunk-
+// interleaved: D x / s first, then xbar in place).
+__host__ __device__ inline size_t gemv1_table_bytes(int K, int copies_log2) {
+  return align16((size_t)K * ((size_t)1 << copies_log2) * 4);
+}
 __host__ __device__ inline size_t gemv1_region0(int K, int copies_log2, int d_in) {
-  const size_t t = (size_t)K * ((size_t)1 << copies_log2) * 4, x = (size_t)d_in * 4;
-  return align16(t > x ? t : x);
+  return gemv1_table_bytes(K, copies_log2) + align16((size_t)d_in * 4);
 }
 
 __device__ __forceinline__ void issue_tile(const Gemv1Args& a, int tile, unsigned char* dst,
@@ -116,38 +120,32 @@ __global__ void __launch_bounds__(MAXT, 1) k_gemv1(const Gemv1Args a) {
       issued[s] = 1;
     }
   }
-  // D_j x_j / s_j for every column, spread over the whole CTA, chunk-interleaved
-  // in the table area (free until the table is written below)
-  float* xsT = reinterpret_cast<float*>(tab);
-  const __nv_bfloat16* xin = a.x;
+  // prologue, with its global loads issued together:
+  //   D_j x_j / s_j for every column into xsT [j][c] (8 columns per thread,
+  //   16-byte loads), and the fp16x2 codebook table with `copies` replicas of
+  //   each entry side by side, written in a lane-rotated order,
+  //   (r + lane) mod copies, so that a warp's stores spread over the banks;
+  //   then one warp per slice turns its chunks into xbar = sigma (.)
+  //   R_fwd(x / s) in place, and every warp loads its chunk's xbar.
+  float* xsT = reinterpret_cast<float*>(smem + gemv1_table_bytes(a.K, a.copies_log2));
   const uint64_t seed = a.seed;
   int flags = 0;
-  fill_interleaved<kE>(xsT, a.scale, a.d_in, C, [&](int j, float sv) {
-    const float xv = __bfloat162float(xin[j]);
-    if (!isfinite(xv)) flags = QAMW_STATUS_NONFINITE;
-    const float q = __fdiv_rn(xv, sv);
-    return mask_negative(seed, (uint32_t)j) ? -q : q;
-  });
-  __syncthreads();
-
-  // xbar of this lane's chunk c: sigma (.) R_fwd(x / s), in registers
-  const int sl = warp % a.S, kk = warp / a.S;
-  const int c = sl * 32 + lane;
-  const bool active = c < C;
-  float xr[kE];
-  float sg[kQ];
-  if (active) {
-    load_halves<kQ>(a.sigma + (int64_t)c * kQ, sg);
+  for (int j8 = tid * 8; j8 < a.d_in; j8 += blockDim.x * 8) {
+    const uint4 xv = __ldg(reinterpret_cast<const uint4*>(a.x + j8));
+    const uint4 sv = __ldg(reinterpret_cast<const uint4*>(a.scale + j8));
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+    const __half2* sh = reinterpret_cast<const __half2*>(&sv);
 #pragma unroll
-    for (int j = 0; j < kE; ++j) xr[j] = xsT[j * C + c];
-  } else {
-#pragma unroll
-    for (int j = 0; j < kE; ++j) xr[j] = 0.f;
+    for (int e = 0; e < 4; ++e) {
+      const float2 s2 = __half22float2(sh[e]);
+      const float x0 = __uint_as_float(xw[e] << 16), x1 = __uint_as_float(xw[e] & 0xffff0000u);
+      if (!isfinite(x0) || !isfinite(x1)) flags = QAMW_STATUS_NONFINITE;
+      const int j = j8 + 2 * e;
+      const float q0 = __fdiv_rn(x0, s2.x), q1 = __fdiv_rn(x1, s2.y);
+      xsT[(j % kE) * C + j / kE] = mask_negative(seed, (uint32_t)j) ? -q0 : q0;
+      xsT[((j + 1) % kE) * C + (j + 1) / kE] = mask_negative(seed, (uint32_t)(j + 1)) ? -q1 : q1;
+    }
   }
-  __syncthreads();
-  // fp16x2 codebook, `copies` replicas of each entry side by side: one load per
-  // codeword, then its replicas in a lane-rotated order, (r + lane) mod copies,
-  // so that a warp's stores spread over the banks (at most 2-way conflicts)
 #pragma unroll 4
   for (int j = tid; j < a.K; j += blockDim.x) {
     const float2 cw = __ldg(a.codebook + j);
@@ -157,16 +155,47 @@ __global__ void __launch_bounds__(MAXT, 1) k_gemv1(const Gemv1Args a) {
       tab[(j << a.copies_log2) + ((r + lane) & (copies - 1))] = u;
   }
   __syncthreads();
-  fwht_reg<kE>(xr, min(a.block, kE));
-  fwht_lanes<kE>(xr, max(a.block / kE, 1));
-  if (active) {
-    const float inv_sqrt_b = 1.0f / sqrtf((float)a.block);
+
+  const int sl = warp % a.S, kk = warp / a.S;
+  const int c = sl * 32 + lane;
+  const bool active = c < C;
+  float xr[kE];
+  if (kk == 0) {  // one warp per slice: xbar of its 32 chunks, in place
+    if (active) {
 #pragma unroll
-    for (int q = 0; q < kQ; ++q) {
-      const float f = sg[q] * inv_sqrt_b;
-      xr[2 * q] *= f;
-      xr[2 * q + 1] *= f;
+      for (int j = 0; j < kE; ++j) xr[j] = xsT[j * C + c];
+    } else {
+#pragma unroll
+      for (int j = 0; j < kE; ++j) xr[j] = 0.f;
     }
+    fwht_reg<kE>(xr, min(a.block, kE));
+    fwht_lanes<kE>(xr, max(a.block / kE, 1));
+    if (active) {
+      const float inv_sqrt_b = 1.0f / sqrtf((float)a.block);
+      const uint4* sg8 = reinterpret_cast<const uint4*>(a.sigma + (int64_t)c * kQ);
+#pragma unroll
+      for (int t = 0; t < kQ / 8; ++t) {  // sigma of pairs 8t .. 8t + 7
+        const uint4 v = __ldg(sg8 + t);
+        const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f2 = __half22float2(h[e]);
+          const int q = 8 * t + 2 * e;
+          xsT[(2 * q) * C + c] = xr[2 * q] * (f2.x * inv_sqrt_b);
+          xsT[(2 * q + 1) * C + c] = xr[2 * q + 1] * (f2.x * inv_sqrt_b);
+          xsT[(2 * q + 2) * C + c] = xr[2 * q + 2] * (f2.y * inv_sqrt_b);
+          xsT[(2 * q + 3) * C + c] = xr[2 * q + 3] * (f2.y * inv_sqrt_b);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (active) {
+#pragma unroll
+    for (int j = 0; j < kE; ++j) xr[j] = xsT[j * C + c];
+  } else {
+#pragma unroll
+    for (int j = 0; j < kE; ++j) xr[j] = 0.f;
   }
 
   const uint32_t copy = (uint32_t)lane & (uint32_t)(copies - 1);
@@ -257,7 +286,7 @@ cudaError_t run_gemv1(const qamw_matrix& m, const uint16_t* d_x, uint16_t* d_y,
   a.seed = m.mask_seed;
   const int C = m.d_in / kE;
   a.S = (C + 31) / 32;
-  a.k = a.S <= 8 ? 8 / a.S : 1;
+  a.k = a.S <= 16 ? 16 / a.S : 1;  // 16 warps (512 threads) per SM
   // ~20 KB of indices per stage, whole rows, a multiple of k rows
   int R = (int)(20480 / m.row_bytes);
   R = R < a.k ? a.k : (R / a.k) * a.k;
@@ -270,7 +299,7 @@ cudaError_t run_gemv1(const qamw_matrix& m, const uint16_t* d_x, uint16_t* d_y,
   const size_t smem = gemv1_smem(a.K, cl, a.stage_bytes, R, a.S, a.d_in);
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   const int threads = 32 * a.S * a.k;
-  // 256-thread bound (up to 255 registers) unless a row needs more than 8 slices
+  // 512 threads: at most 128 registers, 16 warps per SM
   const void* fn = threads <= 256 ? reinterpret_cast<const void*>(&k_gemv1<BITS, 256>)
                                   : reinterpret_cast<const void*>(&k_gemv1<BITS, 512>);
   cudaError_t err = allow_smem(fn, smem);
