@@ -45,6 +45,31 @@ L2_FLUSH_BYTES = 256 << 20
 FP32_LANES_PER_SM = 128
 SMS = 148
 
+# DRAM bytes (read + write) of one k_encode launch on this workload, from one
+# ncu capture (profiles/k_encode_4096x4096_k2048.md), valid while the encoder's
+# sources hash to the recorded sha256; otherwise the roofline reports traffic
+# null.
+ENCODE_TRAFFIC = {"bytes": 35314688 + 5376,
+                  "sha256": "9402c512c28228a9394bba9f21a92e7ad0a49e96eef64f6045c2e3c6bcf70790"}
+ENCODE_SOURCES = ("vector_quantization_codec_b200/csrc/encode.cu",
+                  "vector_quantization_codec_b200/csrc/common.cuh",
+                  "vector_quantization_codec_b200/csrc/launch.cuh")
+
+
+def sources_sha256(paths) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def encode_traffic():
+    if ENCODE_TRAFFIC["bytes"] is None:
+        return None
+    return ENCODE_TRAFFIC["bytes"] if sources_sha256(ENCODE_SOURCES) == ENCODE_TRAFFIC["sha256"] else None
+
 
 # ------------------------------------------------------------------ host logic
 
@@ -233,21 +258,19 @@ def run_gpu(args) -> dict | None:
 
     stages = ["scales", "calibrate", "encode", "decode", "gemv"]
 
-    def step(ev=None):
-        def mark(i):
-            if ev is not None:
-                ev[i].record(stream)
-        mark(0)
-        qamw.qamw_channel_scales(D_IN, act, ALPHA, m.chan_scale, status=status, stream=stream)
-        mark(1)
-        qamw.qamw_calibrate_sigma(W, m, workspace=ws_cal, status=status, stream=stream)
-        mark(2)
-        qamw.qamw_encode_rows(W, m, status=status, stream=stream)
-        mark(3)
-        qamw.qamw_decode(m, W_hat, status=status, stream=stream)
-        mark(4)
-        qamw.qamw_decode_gemv(m, x, y, workspace=ws_gemv, status=status, stream=stream)
-        mark(5)
+    # one step: the five C-ABI calls, each on the current stream (the capture
+    # stream while a graph is recorded)
+    stage_calls = [
+        lambda: qamw.qamw_channel_scales(D_IN, act, ALPHA, m.chan_scale, status=status),
+        lambda: qamw.qamw_calibrate_sigma(W, m, workspace=ws_cal, status=status),
+        lambda: qamw.qamw_encode_rows(W, m, status=status),
+        lambda: qamw.qamw_decode(m, W_hat, status=status),
+        lambda: qamw.qamw_decode_gemv(m, x, y, workspace=ws_gemv, status=status),
+    ]
+
+    def step():
+        for call in stage_calls:
+            call()
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
@@ -262,7 +285,25 @@ def run_gpu(args) -> dict | None:
     torch.cuda.synchronize()
     candidates = int(cand.item())
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    # the step and each stage as CUDA graphs of the same C-ABI calls (device
+    # time; the host only replays); the L2 flush stays outside the events
+    torch.cuda.synchronize()
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step):
+        step()
+    g_stage = []
+    for call in stage_calls:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            call()
+        g_stage.append(g)
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        g_step.replay()
+    torch.cuda.synchronize()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -270,19 +311,27 @@ def run_gpu(args) -> dict | None:
         wall0 = time.perf_counter()
         for k in range(args.steps):
             flush.fill_(1.0)
-            step(events[k])
+            ev[k][0].record(stream)
+            g_step.replay()
+            ev[k][1].record(stream)
         torch.cuda.synchronize()
         wall1 = time.perf_counter()
     if world > 1:
         dist.barrier()
-    stage_ms = {s: [] for s in stages}
-    for ev in events:
-        for i, s in enumerate(stages):
-            stage_ms[s].append(ev[i].elapsed_time(ev[i + 1]))
-    step_ms = [sum(stage_ms[s][k] for s in stages) for k in range(args.steps)]
+    step_ms = [a.elapsed_time(b) for a, b in ev]
     mean_step = sum(step_ms) / len(step_ms)
-    mean_stage = {s: sum(v) / len(v) for s, v in stage_ms.items()}
     mean_step_max = max_over_ranks(mean_step, world, dev)
+    # each stage alone (after the same flush), for the breakdown
+    stage_ms = {s: [] for s in stages}
+    for s, g in zip(stages, g_stage):
+        for k in range(args.steps):
+            flush.fill_(1.0)
+            ev[k][0].record(stream)
+            g.replay()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        stage_ms[s] = [a.elapsed_time(b) for a, b in ev]
+    mean_stage = {s: sum(v) / len(v) for s, v in stage_ms.items()}
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(args, W_np, act_np, x_np, m, ws_cal, ws_gemv, W_hat, y, status, stream, world, dev)
@@ -325,11 +374,23 @@ def run_gpu(args) -> dict | None:
     }
     dominant = max(["calibrate", "encode", "decode", "gemv"], key=lambda s: mean_stage[s])
     if dominant == "encode":
-        achieved = flops / (mean_stage["encode"] * 1e-3) / 1e12
-        peak = fp32_peak_tflops(sm_mhz)
-        roofline = dict(bound="alu", kernel="k_encode (qamw_encode_rows)", achieved=achieved,
-                        peak=peak, unit="TFLOP/s", frac=achieved / peak, traffic=None,
-                        peak_source=f"148 SM x 128 FP32 lanes x 2 x {sm_mhz:.0f} MHz (run clock)")
+        # the encoder's bound is the larger of bytes / HBM and algorithmic
+        # flops / FP32 peak; for this workload the bytes (see components)
+        t_bytes = ab["encode"] / (hbm * 1e9)
+        t_flops = flops / (fp32_peak_tflops(sm_mhz) * 1e12)
+        if t_bytes >= t_flops:
+            achieved = ab["encode"] / (mean_stage["encode"] * 1e-3) / 1e9
+            roofline = dict(bound="hbm", kernel="k_encode (qamw_encode_rows)", achieved=achieved,
+                            peak=hbm, unit="GB/s", frac=achieved / hbm,
+                            traffic=encode_traffic(),
+                            peak_source=peaks["source"] + " MEASURED_PEAKS.json hbm_gbs")
+        else:
+            achieved = flops / (mean_stage["encode"] * 1e-3) / 1e12
+            peak = fp32_peak_tflops(sm_mhz)
+            roofline = dict(bound="alu", kernel="k_encode (qamw_encode_rows)", achieved=achieved,
+                            peak=peak, unit="TFLOP/s", frac=achieved / peak,
+                            traffic=encode_traffic(),
+                            peak_source=f"148 SM x 128 FP32 lanes x 2 x {sm_mhz:.0f} MHz (run clock)")
     else:
         key = {"decode": "decode", "gemv": "gemv", "calibrate": "encode"}[dominant]
         achieved = ab[key] / (mean_stage[dominant] * 1e-3) / 1e9
@@ -354,6 +415,7 @@ def run_gpu(args) -> dict | None:
                    "block": BLOCK, "alpha": ALPHA, "gemv_batch": GEMV_BATCH,
                    "step": "scales+calibrate+encode_rows+decode+decode_gemv",
                    "l2": "flushed (256 MB write) before every step, outside the timed events",
+                   "timing": "CUDA events around a CUDA-graph replay of the step's five C-ABI calls",
                    "parallelism": f"{world} independent matrices (one per GPU)"},
         "components": comp,
         "roofline": roofline,
@@ -369,9 +431,9 @@ def run_gpu(args) -> dict | None:
     return out
 
 
-# kernels one step launches: scales 1, calibrate 4 (row norms, selection,
-# partial sums, finish), encode 1, decode 1, decode-GEMV 2 (rotate, gemv)
-LAUNCHES_PER_STEP = 9
+# kernels one step launches: scales 1, calibrate 3 (rows, extension, finish),
+# encode 1, decode 1, decode-GEMV 1 (batch 1)
+LAUNCHES_PER_STEP = 7
 
 
 def run_e2e(args, W_np, act_np, x_np, m, ws_cal, ws_gemv, W_hat, y, status, stream, world, dev):

@@ -47,9 +47,27 @@ __global__ void __launch_bounds__(256) k_scales(const float* __restrict__ a, int
     const float v = a[j];
     __half h;
     if (v > 0.f && isfinite(v)) {
-      h = __double2half(pow((double)v / mean, (double)alpha));
-      const float hf = __half2float(h);
-      if (isinf(hf) || hf == 0.f) range = 1;
+      // binary16(pow(v / mean, alpha)) of the fp64 power: an fp32 evaluation
+      // decides unless it lies within its error bound (log2f 1 ulp, exp2f 2
+      // ulp, the ratio 2^-24: under (2 + |t| + |alpha|) 2^-23 relative for
+      // t = alpha log2 r; a 2x margin taken) of a binary16 rounding midpoint -- the
+      // midpoints between h and its neighbours are exact in fp32 -- or
+      // outside the normal/subnormal range; there the fp64 pow decides
+      const float t = alpha * log2f((float)((double)v / mean));
+      const float y = exp2f(t);
+      h = __float2half_rn(y);
+      const uint16_t hb = __half_as_ushort(h);
+      bool exact = y > 0.f && hb > 0u && hb < 0x7bffu;
+      if (exact) {
+        const float hf = __half2float(h);
+        const float up = __half2float(__ushort_as_half((uint16_t)(hb + 1)));
+        const float dn = __half2float(__ushort_as_half((uint16_t)(hb - 1)));
+        const float tol = y * (2.0f + fabsf(t) + fabsf(alpha)) * 2.4e-7f;
+        exact = fabsf(y - 0.5f * (hf + up)) > tol && fabsf(y - 0.5f * (hf + dn)) > tol;
+      }
+      if (!exact) h = __double2half(pow((double)v / mean, (double)alpha));
+      const float hf2 = __half2float(h);
+      if (isinf(hf2) || hf2 == 0.f) range = 1;
     } else {
       h = __float2half(1.0f);
     }
@@ -184,10 +202,12 @@ __global__ void __launch_bounds__(512) k_calib_ext(const T* __restrict__ W,
   const int C = d_in / kE;
   const int c = threadIdx.x;
   const bool active_c = c < C;
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < 32) {  // the non-zero rows found among the first 1024 (integer sum)
     int n = 0;
-    for (int b = 0; b < nparts; ++b) n += nonzero[b];
-    total = n;
+    for (int b = threadIdx.x; b < nparts; b += 32) n += nonzero[b];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+    if (threadIdx.x == 0) total = n;
   }
   float acc[kQ];
 #pragma unroll
