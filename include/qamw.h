@@ -218,6 +218,22 @@ QAMW_API int qamw_calibrate_sigma(const void *d_W, int dtype, const qamw_matrix 
 QAMW_API int qamw_encode_rows(const void *d_W, int dtype, const qamw_matrix *m,
                               uint64_t *d_candidates, int32_t *d_status, void *stream);
 
+/* qamw_normalised_pairs: the normalised points p_k = z_k / sigma_k (section
+ *   3.1 steps 1-4 with the given m->chan_scale and m->sigma: the points the
+ *   encoder searches, bitwise) of rows [row0, row0 + nrows), written to
+ *   d_points as float pairs, row-major [nrows][d_in / 2][2] (caller-owned,
+ *   16-byte aligned, nrows * d_in * 4 bytes).  Rows whose norm is zero or not
+ *   finite give NaN points (qamw_train_codebook skips and flags them).  This is
+ *   the input of a per-checkpoint codebook: the explainer page's "Significance
+ *   and Claims" names training on the empirical normalised pairs instead of
+ *   the unit circular Gaussian as a possible gain; qamw_train_codebook on
+ *   these points does that.  m->packed and m->row_norm are not touched.
+ *   Errors: QAMW_ERR_SHAPE for a row range outside [0, d_out).  Flags:
+ *   NONFINITE. */
+QAMW_API int qamw_normalised_pairs(const void *d_W, int dtype, const qamw_matrix *m, int64_t row0,
+                                   int64_t nrows, float *d_points, int32_t *d_status,
+                                   void *stream);
+
 /* Section 3.5, the polar baseline: the amplitude |z_k|/sigma_k is quantised
  * with an N_a-level Lloyd-Max codebook of the unit Rayleigh density
  * r exp(-r^2/2) and the phase arg z_k is rounded to one of N_p uniform bins;

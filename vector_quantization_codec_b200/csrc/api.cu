@@ -286,6 +286,19 @@ int qamw_encode_rows(const void* d_W, int dtype, const qamw_matrix* m, uint64_t*
                                     static_cast<cudaStream_t>(stream)));
 }
 
+int qamw_normalised_pairs(const void* d_W, int dtype, const qamw_matrix* m, int64_t row0,
+                          int64_t nrows, float* d_points, int32_t* d_status, void* stream) {
+  int rc = check_matrix(m, false);
+  if (rc != QAMW_OK) return rc;
+  if (dtype != QAMW_DTYPE_F32 && dtype != QAMW_DTYPE_BF16) return QAMW_ERR_INVALID;
+  if (row0 < 0 || nrows < 0 || row0 + nrows > m->d_out) return QAMW_ERR_SHAPE;
+  if (nrows == 0) return QAMW_OK;
+  if (!d_W || !d_points || !m->sigma || !m->chan_scale) return QAMW_ERR_INVALID;
+  if (!aligned16(d_W) || !aligned16(d_points)) return QAMW_ERR_ALIGN;
+  return cuda_rc(launch_points(d_W, dtype, *m, row0, nrows, d_points, d_status,
+                               static_cast<cudaStream_t>(stream)));
+}
+
 int qamw_encode_rows_polar(const void* d_W, int dtype, const qamw_matrix* m, int32_t* d_status,
                            void* stream) {
   int rc = check_matrix(m, true);

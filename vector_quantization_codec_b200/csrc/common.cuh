@@ -37,6 +37,20 @@ __device__ __forceinline__ bool mask_negative(uint64_t seed, uint32_t j) {
   return (mix64((seed << 32) + j) >> 63) != 0;
 }
 
+// Programmatic dependent launch.  The kernels of the encode / decode / GEMV
+// path are launched so that each may start while the kernel ahead of it in the
+// stream is finishing.  pdl_wait() returns once that kernel has completed and
+// its writes are visible (at once when there is no such kernel); every read of
+// data another path kernel writes (s, sigma, calibration partials, indices,
+// r_hat) and every global write come after it.  Before it a kernel reads only
+// data no path kernel writes (W, x, the statistic, the codebook, the search
+// table).  pdl_trigger(), called after pdl_wait(), lets the next kernel start:
+// when kernel N starts, every kernel before N - 1 has completed.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void raise_flag(int32_t* status, int flag) {
   if (flag && status) atomicOr(status, flag);
 }

@@ -134,18 +134,11 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
     ipos.advance(sdr, sdc, C);
   };
   if (threadIdx.x == 0) {
-    const int64_t b0 = (int64_t)blockIdx.x * blockDim.x;
-    ipos.r = b0 / C;
-    ipos.c = (int)(b0 - ipos.r * C);
     for (int s = 0; s < kDecStages; ++s) {
       mbar_init(&bar[s], 1);
       issued[s] = 0;
     }
     fence_mbar_init();
-    for (int s = 0; s < kDecStages; ++s) {
-      if (b0 + s * stride >= V) break;
-      issue(s, b0 + s * stride);
-    }
   }
   // table fills: unrolled so that each thread's loads are in flight together;
   // the codewords as (x + y, x - y) when the block is at least 2 (the first
@@ -155,6 +148,18 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
   for (int i = threadIdx.x; i < a.K; i += blockDim.x) {
     const float2 cw = a.codebook[i];
     cb[i] = fold ? make_float2(cw.x + cw.y, cw.x - cw.y) : cw;
+  }
+  // the indices, r_hat, sigma and s below come from the kernels ahead
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x == 0) {
+    const int64_t b0 = (int64_t)blockIdx.x * blockDim.x;
+    ipos.r = b0 / C;
+    ipos.c = (int)(b0 - ipos.r * C);
+    for (int s = 0; s < kDecStages; ++s) {
+      if (b0 + s * stride >= V) break;
+      issue(s, b0 + s * stride);
+    }
   }
   fill_quads<kQ>(sg4, a.sigma, P, C, [](int, float v) { return v; });
   const float inv_sqrt_b = 1.0f / sqrtf((float)a.block);
@@ -263,8 +268,7 @@ cudaError_t run_decode(const DecodeArgs& a, cudaStream_t stream) {
   if (err != cudaSuccess) return err;
   const int64_t V = (int64_t)a.d_out * (a.d_in / kE);
   const int grid = persistent_grid(fn, threads, smem, (V + threads - 1) / threads);
-  k_decode<BITS><<<grid, threads, smem, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(k_decode<BITS>, dim3(grid), dim3(threads), smem, stream, a);
 }
 
 }  // namespace

@@ -18,33 +18,52 @@ namespace {
 
 // ------------------------------------------------------------------ scales
 
-// Every CTA sums the whole statistic in the same fixed order (fp64), so all
-// CTAs see the identical mean; each then rounds its slice of scales.
-__global__ void __launch_bounds__(256) k_scales(const float* __restrict__ a, int d_in,
-                                                float alpha, __half* __restrict__ s,
-                                                int32_t* status) {
-  __shared__ double red[8];
+// One CTA of 1024 threads: thread t holds the statistic of channels t + 1024 i
+// (i < 32, d_in <= 32768) in registers, so the statistic is read once; the
+// fp64 sum is reduced in a fixed order (per-thread ascending i, a shuffle tree
+// per warp, then the 32 warp sums by the same tree), so the mean is bitwise
+// reproducible; each thread then rounds its own channels' scales.
+constexpr int kScaleThreads = 1024;
+__global__ void __launch_bounds__(kScaleThreads) k_scales(const float* __restrict__ a, int d_in,
+                                                          float alpha, __half* __restrict__ s,
+                                                          int32_t* status) {
+  __shared__ double red[32];
+  __shared__ double mean_s;
+  constexpr int kPer = kMaxDin / kScaleThreads;
+  float vals[kPer];
   double sum = 0.0;
   int bad = 0;
-#pragma unroll 8
-  for (int j = threadIdx.x; j < d_in; j += blockDim.x) {
-    const float v = a[j];
-    if (v > 0.f && isfinite(v))
-      sum += (double)v;
-    else
-      bad = 1;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int j = threadIdx.x + i * kScaleThreads;
+    vals[i] = j < d_in ? a[j] : 1.f;
+    if (j < d_in) {
+      if (vals[i] > 0.f && isfinite(vals[i]))
+        sum += (double)vals[i];
+      else
+        bad = 1;
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sum;
   __syncthreads();
-  double total = 0.0;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) total += red[w];
-  const double mean = total / (double)d_in;
+  if (threadIdx.x < 32) {
+    double t = red[threadIdx.x];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (threadIdx.x == 0) mean_s = t / (double)d_in;
+  }
+  bad = __syncthreads_or(bad);
+  const double mean = mean_s;
+  pdl_wait();  // s may still be read by the kernel ahead
+  pdl_trigger();
   int range = 0;
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j < d_in) {
-    const float v = a[j];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int j = threadIdx.x + i * kScaleThreads;
+    if (j >= d_in) break;
+    const float v = vals[i];
     __half h;
     if (v > 0.f && isfinite(v)) {
       // binary16(pow(v / mean, alpha)) of the fp64 power: an fp32 evaluation
@@ -73,8 +92,7 @@ __global__ void __launch_bounds__(256) k_scales(const float* __restrict__ a, int
     }
     s[j] = h;
   }
-  if (blockIdx.x == 0) bad = __syncthreads_or(bad);
-  raise_flag(status, ((blockIdx.x == 0 && bad) ? QAMW_STATUS_BAD_STAT : 0) |
+  raise_flag(status, ((threadIdx.x == 0 && bad) ? QAMW_STATUS_BAD_STAT : 0) |
                          (range ? QAMW_STATUS_RANGE : 0));
 }
 
@@ -104,6 +122,8 @@ __global__ void __launch_bounds__(MAXT) k_calib_rows(const T* __restrict__ W,
                                                      int32_t* __restrict__ nonzero,
                                                      int32_t* status) {
   extern __shared__ __align__(16) float sm[];
+  pdl_wait();
+  pdl_trigger();
   const int C = d_in / kE, P = d_in / 2;
   float* fT = sm;                     // [j][c]: D * s of column 64c + j
   float* red = sm + d_in;             // [g][q][c]
@@ -199,6 +219,8 @@ __global__ void __launch_bounds__(512) k_calib_ext(const T* __restrict__ W,
   __shared__ float part[512];
   __shared__ float rtot;
   __shared__ int total;
+  pdl_wait();
+  pdl_trigger();
   const int C = d_in / kE;
   const int c = threadIdx.x;
   const bool active_c = c < C;
@@ -274,6 +296,8 @@ __global__ void __launch_bounds__(256) k_calib_finish(const float* __restrict__ 
                                                       const int32_t* __restrict__ n_cal_p, int P,
                                                       __half* __restrict__ sigma,
                                                       int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   const int g = blockIdx.x * (blockDim.x / 16) + threadIdx.x / 16, i = threadIdx.x & 15;
   const int k = min(g, P - 1);
   double sum = 0.0;
@@ -322,6 +346,8 @@ struct EncodeArgs {
 template <int BITS, typename T, bool POLAR>
 __global__ void __launch_bounds__(512, 1) k_encode_wide(const EncodeArgs<T> a) {
   extern __shared__ __align__(16) unsigned char smem[];
+  pdl_wait();
+  pdl_trigger();
   float2* cb2 = reinterpret_cast<float2*>(smem);
   // per-column tables transposed, [position in chunk][chunk], so that the lanes
   // of a warp (consecutive chunks) read consecutive words
@@ -524,6 +550,8 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
 #pragma unroll 4
     for (int i = threadIdx.x; i < a.K; i += NT) cb2[i] = a.codebook[i];
   }
+  pdl_wait();  // s and sigma below, W, and the outputs, after the kernel ahead
+  pdl_trigger();
   const uint64_t seed = a.seed;
   fill_quads<kE>(fT4, a.scale, a.d_in, C, [=](int j, float v) {
     return mask_negative(seed, (uint32_t)j) ? -v : v;
@@ -531,14 +559,11 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
   fill_quads<kQ>(isg4, a.sigma, a.d_in / 2, C, [](int, float v) { return 1.0f / v; });
   __syncthreads();
   int flags = 0;
-  if (S > 0) {
-    const bool ok = mbar_wait_bounded(bar, 0);
-    if (__syncthreads_or(!ok)) {  // the copies never landed: give up, after one more bounded wait
-      if (threadIdx.x == 0) mbar_wait_bounded(bar, 0);
-      raise_flag(a.status, QAMW_STATUS_TIMEOUT);
-      return;
-    }
-  }
+  // the head copy is waited for just before a thread's first search, so that it
+  // overlaps the first row's loads and butterflies; a thread whose wait runs out
+  // searches the main table instead (same results) and flags TIMEOUT
+  int S_eff = S;
+  bool hs_pending = S > 0;
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = NT >> 5;
   const int rl = threadIdx.x / C, c = threadIdx.x - rl * C;
@@ -549,16 +574,18 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
   float2* mypts = pts + threadIdx.x;
   unsigned scored = 0;
   int buf = 0;
-  for (int64_t r0 = (int64_t)blockIdx.x * R; r0 < a.d_out; r0 += (int64_t)gridDim.x * R) {
+  // this CTA's rows: a contiguous block of floor or ceil(d_out / grid)
+  const int64_t row_lo = (int64_t)blockIdx.x * a.d_out / gridDim.x;
+  const int64_t row_hi = ((int64_t)blockIdx.x + 1) * a.d_out / gridDim.x;
+  for (int64_t r0 = row_lo; r0 < row_hi; r0 += R) {
     const int64_t row = r0 + rl;
-    const bool active = rl < R && row < a.d_out;
+    const bool active = rl < R && row < row_hi;
     if (per_row && !active) continue;  // the row's threads all skip, barrier included
     float x[kE];
     float ss = 0.f;
     if (active) {
-      if (c == 0 && row + (int64_t)gridDim.x * R < a.d_out)  // this row's next one, into L2
-        bulk_prefetch_l2(a.W + (row + (int64_t)gridDim.x * R) * a.d_in,
-                         (unsigned)(a.d_in * (int64_t)sizeof(T)));
+      if (c == 0 && row + R < row_hi)  // this thread group's next row, into L2
+        bulk_prefetch_l2(a.W + (row + R) * a.d_in, (unsigned)(a.d_in * (int64_t)sizeof(T)));
       load64(a.W + row * a.d_in + (int64_t)c * kE, x);
 #pragma unroll
       for (int i = 0; i < kE / 4; ++i) {
@@ -615,6 +642,13 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
 #pragma unroll
       for (int t = 0; t < BITS; ++t) dst[t] = 0u;
     } else {
+      if (hs_pending) {
+        hs_pending = false;
+        if (!mbar_wait_bounded(bar, 0)) {
+          S_eff = 0;
+          flags |= QAMW_STATUS_TIMEOUT;
+        }
+      }
       const float inv = 1.0f / (r * sqrt_b);
       // each index goes to the first word of its point's slot once the point
       // has been read; the 16 indices of a half are then packed with fixed
@@ -652,15 +686,15 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
           const uint32_t cb_s = smem_u32(cb2);
           uint32_t rare = 0;
           float2 p = mypts[0];
-          uint2 ha = pf_head_shared(p.x, p.y, pf, hs, S, c0);
+          uint2 ha = pf_head_shared(p.x, p.y, pf, hs, S_eff, c0);
           p = mypts[NT];
-          uint2 hb = pf_head_shared(p.x, p.y, pf, hs, S, c0);
+          uint2 hb = pf_head_shared(p.x, p.y, pf, hs, S_eff, c0);
 #pragma unroll 1
           for (int q = 0; q < kQ / 2; q += 2) {
             p = mypts[min(q + 2, kQ / 2 - 1) * NT];
-            const uint2 hc = pf_head_shared(p.x, p.y, pf, hs, S, c0);
+            const uint2 hc = pf_head_shared(p.x, p.y, pf, hs, S_eff, c0);
             p = mypts[min(q + 3, kQ / 2 - 1) * NT];
-            const uint2 hd = pf_head_shared(p.x, p.y, pf, hs, S, c0);
+            const uint2 hd = pf_head_shared(p.x, p.y, pf, hs, S_eff, c0);
             p = mypts[q * NT];
             uint32_t id = pf_finish_fast(ha, p.x, p.y, cb_s, scored, count);
             rare |= id;
@@ -699,6 +733,7 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
         *reinterpret_cast<uint32_t*>(a.packed + row * a.row_bytes + o) = 0u;
     }
   }
+  if (S > 0 && threadIdx.x == 0) mbar_wait_bounded(bar, 0);  // no copy in flight at exit
   raise_flag(a.status, flags);
   if (a.candidates != nullptr) {
     unsigned long long v = scored;
@@ -706,6 +741,76 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (lane == 0) atomicAdd(a.candidates, v);
   }
+}
+
+// The normalised points p_k = z_k / sigma_k of rows [row0, row0 + nrows)
+// (section 3.1 steps 1-4): the encoder's first phase, with the same fixed-order
+// row-norm reduction and the same p = y (1 / (r sqrt(b)) (1 / sigma_k)), so the
+// points are bitwise those the encoder searches.  Rows whose norm is zero or
+// not finite give NaN points.  out: float2 [nrows][d_in / 2].
+template <typename T>
+__global__ void __launch_bounds__(512) k_points(const EncodeArgs<T> a, int64_t row0,
+                                                int64_t nrows, float2* __restrict__ out) {
+  extern __shared__ __align__(16) float psm[];
+  const int P = a.d_in >> 1, C = a.d_in / kE, R = a.rows_per_cta;
+  float* fT = psm;          // [j][c]: D * s of column 64c + j
+  float* isgT = fT + a.d_in;  // [q][c]: 1 / sigma of pair 32c + q
+  float* part = isgT + P;   // [blockDim]
+  float* rsum = part + blockDim.x;
+  const uint64_t seed = a.seed;
+  fill_interleaved<kE>(fT, a.scale, a.d_in, C, [=](int j, float v) {
+    return mask_negative(seed, (uint32_t)j) ? -v : v;
+  });
+  fill_interleaved<kQ>(isgT, a.sigma, P, C, [](int, float v) { return 1.0f / v; });
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int rl = threadIdx.x / C, c = threadIdx.x - rl * C;
+  const int nb = min(a.block, kE), lanes = max(a.block / kE, 1);
+  const float sqrt_b = sqrtf((float)a.block);
+  int flags = 0;
+  for (int64_t g0 = (int64_t)blockIdx.x * R; g0 < nrows; g0 += (int64_t)gridDim.x * R) {
+    const int64_t g = g0 + rl;  // row within the range
+    const bool active = rl < R && g < nrows;
+    float x[kE];
+    float ss = 0.f;
+    if (active) {
+      load64(a.W + (row0 + g) * a.d_in + (int64_t)c * kE, x);
+#pragma unroll
+      for (int j = 0; j < kE; ++j) {
+        x[j] *= fT[j * C + c];
+        ss = fmaf(x[j], x[j], ss);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < kE; ++j) x[j] = 0.f;
+    }
+    part[threadIdx.x] = ss;
+    fwht_reg<kE>(x, nb);
+    fwht_lanes<kE>(x, lanes);
+    __syncthreads();
+    for (int q = warp; q < R; q += nwarps) {
+      float t = 0.f;
+      for (int k = lane; k < C; k += 32) t += part[q * C + k];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      if (lane == 0) rsum[q] = sqrtf(t);
+    }
+    __syncthreads();
+    if (!active) continue;
+    const float r = rsum[rl];
+    if (!isfinite(r)) flags |= QAMW_STATUS_NONFINITE;
+    const bool none = !(r > 0.f) || !isfinite(r);
+    const float inv = 1.0f / (r * sqrt_b);
+    float4* dst = reinterpret_cast<float4*>(out + g * P + (int64_t)c * kQ);
+#pragma unroll
+    for (int q = 0; q < kQ; q += 2) {
+      const float f0 = inv * isgT[q * C + c], f1 = inv * isgT[(q + 1) * C + c];
+      dst[q / 2] = none ? make_float4(NAN, NAN, NAN, NAN)
+                        : make_float4(x[2 * q] * f0, x[2 * q + 1] * f0, x[2 * q + 2] * f1,
+                                      x[2 * q + 3] * f1);
+    }
+  }
+  raise_flag(a.status, flags);
 }
 
 // Rows per CTA iteration and the CTA size for k_encode_wide: R whole rows of C
@@ -777,7 +882,7 @@ cudaError_t run_encode(EncodeArgs<T> a, cudaStream_t stream) {
   if (err != cudaSuccess) return err;
   const int grid = persistent_grid(fn, threads, smem, (a.d_out + R - 1) / R);
   void* args[] = {&a};
-  return cudaLaunchKernel(fn, dim3(grid), dim3(threads), args, smem, stream);
+  return launch_pdl_ptr(fn, dim3(grid), dim3(threads), smem, stream, args);
 }
 
 template <typename T, bool POLAR>
@@ -843,27 +948,24 @@ cudaError_t calibrate_typed(const T* W, const qamw_matrix& m, const EncodeWorksp
                                : reinterpret_cast<const void*>(&k_calib_rows<T, 512>);
   if ((err = allow_smem(fn, smem)) != cudaSuccess) return err;
   if (maxt == 256)
-    k_calib_rows<T, 256><<<kCalCtas, threads, smem, stream>>>(W, s, d_out, d_in, m.block,
-                                                              m.mask_seed, RPC, ws.cal_partial,
-                                                              ws.cal_nonzero, st);
+    err = launch_pdl(k_calib_rows<T, 256>, dim3(kCalCtas), dim3(threads), smem, stream, W, s,
+                     d_out, d_in, m.block, m.mask_seed, RPC, ws.cal_partial, ws.cal_nonzero, st);
   else
-    k_calib_rows<T, 512><<<kCalCtas, threads, smem, stream>>>(W, s, d_out, d_in, m.block,
-                                                              m.mask_seed, RPC, ws.cal_partial,
-                                                              ws.cal_nonzero, st);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    err = launch_pdl(k_calib_rows<T, 512>, dim3(kCalCtas), dim3(threads), smem, stream, W, s,
+                     d_out, d_in, m.block, m.mask_seed, RPC, ws.cal_partial, ws.cal_nonzero, st);
+  if (err != cudaSuccess) return err;
   {
     const int et = ((C + 31) / 32) * 32;
     const size_t esmem = (size_t)d_in * sizeof(float);
     const void* efn = reinterpret_cast<const void*>(&k_calib_ext<T>);
     if ((err = allow_smem(efn, esmem)) != cudaSuccess) return err;
-    k_calib_ext<T><<<1, et, esmem, stream>>>(W, s, d_out, d_in, m.block, m.mask_seed,
-                                             ws.cal_nonzero, kCalCtas, ws.cal_ext, ws.n_cal);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    err = launch_pdl(k_calib_ext<T>, dim3(1), dim3(et), esmem, stream, W, s, d_out, d_in, m.block,
+                     m.mask_seed, ws.cal_nonzero, kCalCtas, ws.cal_ext, ws.n_cal);
+    if (err != cudaSuccess) return err;
   }
-  k_calib_finish<<<(P + 15) / 16, 256, 0, stream>>>(ws.cal_partial, kCalCtas, ws.cal_ext,
-                                                    ws.n_cal, P,
-                                                    reinterpret_cast<__half*>(m.sigma), st);
-  return cudaGetLastError();
+  return launch_pdl(k_calib_finish, dim3((P + 15) / 16), dim3(256), 0, stream,
+                    (const float*)ws.cal_partial, kCalCtas, (const float*)ws.cal_ext,
+                    (const int32_t*)ws.n_cal, P, reinterpret_cast<__half*>(m.sigma), st);
 }
 
 // Section 3.5: Lloyd-Max levels of the unit Rayleigh density on one warp (lane
@@ -939,7 +1041,8 @@ cudaError_t launch_channel_scales(const float* d_act_stat, int d_in, float alpha
                                   int32_t* d_status, cudaStream_t stream) {
   __half* s = reinterpret_cast<__half*>(d_scale);
   if (d_act_stat != nullptr && alpha != 0.0f)
-    k_scales<<<(d_in + 255) / 256, 256, 0, stream>>>(d_act_stat, d_in, alpha, s, d_status);
+    return launch_pdl(k_scales, dim3(1), dim3(kScaleThreads), 0, stream, d_act_stat, d_in, alpha, s,
+                      d_status);
   else
     k_fill_half<<<(d_in + 255) / 256, 256, 0, stream>>>(s, d_in, 1.0f);
   return cudaGetLastError();
@@ -951,6 +1054,41 @@ cudaError_t launch_calibrate(const void* d_W, int dtype, const qamw_matrix& m,
     return calibrate_typed<float>(static_cast<const float*>(d_W), m, ws, d_status, stream);
   return calibrate_typed<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(d_W), m, ws, d_status,
                                         stream);
+}
+
+template <typename T>
+cudaError_t points_typed(const T* W, const qamw_matrix& m, int64_t row0, int64_t nrows,
+                         float2* out, int32_t* st, cudaStream_t stream) {
+  EncodeArgs<T> a{};
+  a.W = W;
+  a.scale = reinterpret_cast<const __half*>(m.chan_scale);
+  a.sigma = reinterpret_cast<const __half*>(m.sigma);
+  a.status = st;
+  a.d_out = m.d_out;
+  a.d_in = m.d_in;
+  a.block = m.block;
+  a.seed = m.mask_seed;
+  const int C = m.d_in / kE;
+  const int R = std::max(1, 256 / C);
+  a.rows_per_cta = R;
+  const int threads = ((R * C + 31) / 32) * 32;
+  const size_t smem = (size_t)m.d_in * 4 + (size_t)(m.d_in / 2) * 4 + (size_t)threads * 4 +
+                      (size_t)R * 4;
+  const void* fn = reinterpret_cast<const void*>(&k_points<T>);
+  cudaError_t err = allow_smem(fn, smem);
+  if (err != cudaSuccess) return err;
+  const int grid = persistent_grid(fn, threads, smem, (nrows + R - 1) / R);
+  k_points<T><<<grid, threads, smem, stream>>>(a, row0, nrows, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_points(const void* d_W, int dtype, const qamw_matrix& m, int64_t row0,
+                          int64_t nrows, float* d_points, int32_t* d_status, cudaStream_t stream) {
+  float2* out = reinterpret_cast<float2*>(d_points);
+  if (dtype == QAMW_DTYPE_BF16)
+    return points_typed(static_cast<const __nv_bfloat16*>(d_W), m, row0, nrows, out, d_status,
+                        stream);
+  return points_typed(static_cast<const float*>(d_W), m, row0, nrows, out, d_status, stream);
 }
 
 cudaError_t launch_encode_rows(const void* d_W, int dtype, const qamw_matrix& m, int32_t* d_status,

@@ -112,7 +112,23 @@ __global__ void __launch_bounds__(MAXT, 1) k_gemv1(const Gemv1Args a) {
       issued[s] = 0;
     }
     fence_mbar_init();
-    // first tiles in flight while xbar and the codebook table are prepared
+  }
+  // the fp16x2 codebook table needs nothing from the kernels ahead: `copies`
+  // replicas of each entry side by side, written in a lane-rotated order,
+  // (r + lane) mod copies, so that a warp's stores spread over the banks
+#pragma unroll 4
+  for (int j = tid; j < a.K; j += blockDim.x) {
+    const float2 cw = __ldg(a.codebook + j);
+    const __half2 h = __floats2half2_rn(cw.x, cw.y);
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(&h);
+    for (int r = 0; r < copies; ++r)
+      tab[(j << a.copies_log2) + ((r + lane) & (copies - 1))] = u;
+  }
+  // the indices, r_hat, sigma and s come from the kernels ahead
+  pdl_wait();
+  pdl_trigger();
+  if (tid == 0) {
+    // first tiles in flight while xbar is prepared
     for (int s = 0; s < kGemvStages; ++s) {
       const int tile = blockIdx.x + s * gridDim.x;
       if (tile >= a.ntiles) break;
@@ -120,13 +136,9 @@ __global__ void __launch_bounds__(MAXT, 1) k_gemv1(const Gemv1Args a) {
       issued[s] = 1;
     }
   }
-  // prologue, with its global loads issued together:
-  //   D_j x_j / s_j for every column into xsT [j][c] (8 columns per thread,
-  //   16-byte loads), and the fp16x2 codebook table with `copies` replicas of
-  //   each entry side by side, written in a lane-rotated order,
-  //   (r + lane) mod copies, so that a warp's stores spread over the banks;
-  //   then one warp per slice turns its chunks into xbar = sigma (.)
-  //   R_fwd(x / s) in place, and every warp loads its chunk's xbar.
+  // D_j x_j / s_j for every column into xsT [j][c] (8 columns per thread,
+  // 16-byte loads); then one warp per slice turns its chunks into xbar =
+  // sigma (.) R_fwd(x / s) in place, and every warp loads its chunk's xbar.
   float* xsT = reinterpret_cast<float*>(smem + gemv1_table_bytes(a.K, a.copies_log2));
   const uint64_t seed = a.seed;
   int flags = 0;
@@ -145,14 +157,6 @@ __global__ void __launch_bounds__(MAXT, 1) k_gemv1(const Gemv1Args a) {
       xsT[(j % kE) * C + j / kE] = mask_negative(seed, (uint32_t)j) ? -q0 : q0;
       xsT[((j + 1) % kE) * C + (j + 1) / kE] = mask_negative(seed, (uint32_t)(j + 1)) ? -q1 : q1;
     }
-  }
-#pragma unroll 4
-  for (int j = tid; j < a.K; j += blockDim.x) {
-    const float2 cw = __ldg(a.codebook + j);
-    const __half2 h = __floats2half2_rn(cw.x, cw.y);
-    const uint32_t u = *reinterpret_cast<const uint32_t*>(&h);
-    for (int r = 0; r < copies; ++r)
-      tab[(j << a.copies_log2) + ((r + lane) & (copies - 1))] = u;
   }
   __syncthreads();
 
@@ -306,10 +310,8 @@ cudaError_t run_gemv1(const qamw_matrix& m, const uint16_t* d_x, uint16_t* d_y,
   if (err != cudaSuccess) return err;
   const int grid = a.ntiles < sm_count() ? a.ntiles : sm_count();
   if (threads <= 256)
-    k_gemv1<BITS, 256><<<grid, threads, smem, stream>>>(a);
-  else
-    k_gemv1<BITS, 512><<<grid, threads, smem, stream>>>(a);
-  return cudaGetLastError();
+    return launch_pdl(k_gemv1<BITS, 256>, dim3(grid), dim3(threads), smem, stream, a);
+  return launch_pdl(k_gemv1<BITS, 512>, dim3(grid), dim3(threads), smem, stream, a);
 }
 
 // ------------------------------------------------------------- batch 2..16

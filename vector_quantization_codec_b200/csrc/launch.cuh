@@ -21,6 +21,41 @@ int persistent_grid(const void* kernel, int threads, size_t smem, int64_t work_c
 // Opt a kernel into more than 48 KB of dynamic shared memory.
 cudaError_t allow_smem(const void* kernel, size_t smem);
 
+// Launch of a path kernel with programmatic stream serialisation: it may start
+// while the kernel ahead of it in the stream finishes (the kernel itself waits,
+// with pdl_wait, before it touches that kernel's results).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// The same for a kernel chosen at run time (args: pointers to its arguments).
+inline cudaError_t launch_pdl_ptr(const void* kernel, dim3 grid, dim3 block, size_t smem,
+                                  cudaStream_t stream, void** args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, kernel, args);
+}
+
 // Workspace carve-up of qamw_encode.
 struct EncodeWorkspace {
   int32_t* cal_nonzero;  // [kCalCtas] non-zero rows each CTA found among rows 0..1023
@@ -43,6 +78,9 @@ cudaError_t launch_channel_scales(const float* d_act_stat, int d_in, float alpha
                                   int32_t* d_status, cudaStream_t stream);
 cudaError_t launch_calibrate(const void* d_W, int dtype, const qamw_matrix& m,
                              const EncodeWorkspace& ws, int32_t* d_status, cudaStream_t stream);
+// Normalised points of rows [row0, row0 + nrows) as float2 [nrows][d_in / 2].
+cudaError_t launch_points(const void* d_W, int dtype, const qamw_matrix& m, int64_t row0,
+                          int64_t nrows, float* d_points, int32_t* d_status, cudaStream_t stream);
 cudaError_t launch_encode_rows(const void* d_W, int dtype, const qamw_matrix& m, int32_t* d_status,
                                unsigned long long* d_candidates, bool polar, cudaStream_t stream);
 cudaError_t launch_polar_codebook(int bits, float* d_codebook, cudaStream_t stream);

@@ -45,7 +45,8 @@ EXPORTS = ("qamw_row_bytes", "qamw_default_block", "qamw_bits_per_weight",
            "qamw_workspace_bytes", "qamw_prefilter_bytes", "qamw_status_string",
            "qamw_train_codebook", "qamw_build_prefilter", "qamw_encode", "qamw_channel_scales",
            "qamw_calibrate_sigma", "qamw_encode_rows", "qamw_decode", "qamw_decode_gemv",
-           "qamw_decode_gemv_noalloc", "qamw_polar_codebook", "qamw_encode_rows_polar")
+           "qamw_decode_gemv_noalloc", "qamw_polar_codebook", "qamw_encode_rows_polar",
+           "qamw_normalised_pairs")
 
 
 class QamwError(RuntimeError):
@@ -85,6 +86,7 @@ def _load() -> C.CDLL:
         "qamw_decode_gemv_noalloc": (I, [C.POINTER(qamw_matrix), V, I, V, V, V]),
         "qamw_polar_codebook": (I, [I, V, V]),
         "qamw_encode_rows_polar": (I, [V, I, C.POINTER(qamw_matrix), V, V]),
+        "qamw_normalised_pairs": (I, [V, I, C.POINTER(qamw_matrix), I64, I64, V, V, V]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -283,6 +285,23 @@ def qamw_encode_rows_polar(W: torch.Tensor, m: EncodedMatrix, status: torch.Tens
     rc = _lib.qamw_encode_rows_polar(_p(W), _dtype_code(W), C.byref(st), _p(status), _s(stream))
     _check("qamw_encode_rows_polar", rc)
     return m
+
+
+def qamw_normalised_pairs(W: torch.Tensor, m: EncodedMatrix, row0: int = 0,
+                          nrows: int | None = None, out: torch.Tensor | None = None,
+                          status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The normalised points z_k / sigma_k of rows [row0, row0 + nrows) as a float32
+    [nrows, d_in / 2, 2] tensor (the encoder's points, bitwise; NaN for rows whose
+    norm is zero or not finite): samples for a per-checkpoint codebook."""
+    if nrows is None:
+        nrows = m.d_out - row0
+    if out is None:
+        out = torch.empty((nrows, m.d_in // 2, 2), dtype=torch.float32, device=W.device)
+    st = m.struct()
+    rc = _lib.qamw_normalised_pairs(_p(W), _dtype_code(W), C.byref(st), row0, nrows, _p(out),
+                                    _p(status), _s(stream))
+    _check("qamw_normalised_pairs", rc)
+    return out
 
 
 def qamw_decode(m: EncodedMatrix, out: torch.Tensor | None = None,
