@@ -131,6 +131,18 @@ QAMW_API size_t qamw_prefilter_bytes(int bits);
 /* Human-readable text for a QAMW_OK / QAMW_ERR_* code or a status flag word. */
 QAMW_API const char *qamw_status_string(int code);
 
+/* qamw_selftest_wait_timeout: a check of the failure path of the bounded waits
+ *   (no counterpart in the paper).  One CTA waits, with the wait the kernels
+ *   use on their bulk-copy rings, on an mbarrier that nothing arrives on, for
+ *   `tries` polls (1 .. the kernels' own limit, 2^18: about 1 s), then ORs
+ *   QAMW_STATUS_TIMEOUT into *d_status and stores the wait's clock cycles in
+ *   *d_cycles (nullable, device).  The kernels give up after 2^18 polls in the
+ *   same way: they flag TIMEOUT, let their copies in flight land and return,
+ *   and the CUDA context stays usable.  Errors: QAMW_ERR_INVALID for tries out
+ *   of range or a null status. */
+QAMW_API int qamw_selftest_wait_timeout(unsigned tries, int32_t *d_status, long long *d_cycles,
+                                        void *stream);
+
 /* ------------------------------------------------------------------ calls */
 
 /* Section 3.6 eq. (2): Lloyd iterations for the joint 2D codebook.

@@ -147,6 +147,15 @@ def test_gemv_and_train_argument_errors():
              None, None) == qamw.QAMW_ERR_WORKSPACE
     assert L.qamw_build_prefilter(C.c_void_p(FAKE), 11, C.c_void_p(FAKE), 10, None) == \
         qamw.QAMW_ERR_WORKSPACE
+    # the bounded-wait check takes 1 .. 2^18 polls and a status word
+    S = L.qamw_selftest_wait_timeout
+    assert S(0, C.c_void_p(FAKE), None, None) == qamw.QAMW_ERR_INVALID
+    assert S((1 << 18) + 1, C.c_void_p(FAKE), None, None) == qamw.QAMW_ERR_INVALID
+    assert S(16, None, None, None) == qamw.QAMW_ERR_INVALID
+    # the row range of the point export must lie inside the matrix
+    P = L.qamw_normalised_pairs
+    assert P(C.c_void_p(FAKE), qamw.QAMW_DTYPE_BF16, C.byref(m), 90, 20, C.c_void_p(FAKE), None,
+             None) == qamw.QAMW_ERR_SHAPE
 
 
 def test_status_strings():

@@ -247,9 +247,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 // ------------------------------------------------------- async bulk copies
 // cp.async.bulk global -> shared with mbarrier completion (TMA, no tensor map,
-// never multicast).  Every wait is bounded: kSpinLimit tries with a short sleep
-// between them (well under a second in total) before the caller gives up.
-constexpr unsigned kSpinLimit = 1u << 20;
+// never multicast).  Every wait is bounded: kSpinLimit polls, each a
+// potentially suspending try_wait followed (after the first 64) by a 256 ns
+// sleep -- about 8,000 cycles a poll measured on B200, so about a second in all
+// -- before the caller gives up.  A copy that lands takes a few polls.
+constexpr unsigned kSpinLimit = 1u << 18;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -315,8 +317,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
   return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity) {
-  for (unsigned i = 0; i < kSpinLimit; ++i) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity,
+                                                  unsigned limit = kSpinLimit) {
+  for (unsigned i = 0; i < limit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if (i >= 64) __nanosleep(256);  // poll at first: copies usually land within a few tries
   }

@@ -46,7 +46,7 @@ EXPORTS = ("qamw_row_bytes", "qamw_default_block", "qamw_bits_per_weight",
            "qamw_train_codebook", "qamw_build_prefilter", "qamw_encode", "qamw_channel_scales",
            "qamw_calibrate_sigma", "qamw_encode_rows", "qamw_decode", "qamw_decode_gemv",
            "qamw_decode_gemv_noalloc", "qamw_polar_codebook", "qamw_encode_rows_polar",
-           "qamw_normalised_pairs")
+           "qamw_normalised_pairs", "qamw_selftest_wait_timeout")
 
 
 class QamwError(RuntimeError):
@@ -87,6 +87,7 @@ def _load() -> C.CDLL:
         "qamw_polar_codebook": (I, [I, V, V]),
         "qamw_encode_rows_polar": (I, [V, I, C.POINTER(qamw_matrix), V, V]),
         "qamw_normalised_pairs": (I, [V, I, C.POINTER(qamw_matrix), I64, I64, V, V, V]),
+        "qamw_selftest_wait_timeout": (I, [C.c_uint, V, V, V]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -302,6 +303,14 @@ def qamw_normalised_pairs(W: torch.Tensor, m: EncodedMatrix, row0: int = 0,
                                     _p(status), _s(stream))
     _check("qamw_normalised_pairs", rc)
     return out
+
+
+def qamw_selftest_wait_timeout(tries: int, status: torch.Tensor, cycles: torch.Tensor | None = None,
+                               stream=None) -> None:
+    """Bounded-wait failure check: a wait that nothing completes gives up after
+    `tries` polls and flags QAMW_STATUS_TIMEOUT in `status`."""
+    _check("qamw_selftest_wait_timeout",
+           _lib.qamw_selftest_wait_timeout(tries, _p(status), _p(cycles), _s(stream)))
 
 
 def qamw_decode(m: EncodedMatrix, out: torch.Tensor | None = None,
