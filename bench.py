@@ -50,8 +50,8 @@ SMS = 148
 # ncu capture (profiles/k_encode_4096x4096_k2048.md), valid while the encoder's
 # sources hash to the recorded sha256; otherwise the roofline reports traffic
 # null.
-ENCODE_TRAFFIC = {"bytes": 35314688 + 5376,
-                  "sha256": "9402c512c28228a9394bba9f21a92e7ad0a49e96eef64f6045c2e3c6bcf70790"}
+ENCODE_TRAFFIC = {"bytes": 35311360 + 2048,
+                  "sha256": "fdfeb5b74f11795a602577e0d7a255ea69705b2d5734fcd09137a9b0cbb576b0"}
 ENCODE_SOURCES = ("vector_quantization_codec_b200/csrc/encode.cu",
                   "vector_quantization_codec_b200/csrc/common.cuh",
                   "vector_quantization_codec_b200/csrc/launch.cuh")
