@@ -50,8 +50,8 @@ SMS = 148
 # ncu capture (profiles/k_encode_4096x4096_k2048.md), valid while the encoder's
 # sources hash to the recorded sha256; otherwise the roofline reports traffic
 # null.
-ENCODE_TRAFFIC = {"bytes": 35311360 + 2048,
-                  "sha256": "fdfeb5b74f11795a602577e0d7a255ea69705b2d5734fcd09137a9b0cbb576b0"}
+ENCODE_TRAFFIC = {"bytes": 35311616 + 4608,
+                  "sha256": "1f7e056fda94e64066c0105216993430be7fcc058e375719dcb48c9b4913154f"}
 ENCODE_SOURCES = ("vector_quantization_codec_b200/csrc/encode.cu",
                   "vector_quantization_codec_b200/csrc/common.cuh",
                   "vector_quantization_codec_b200/csrc/launch.cuh")

@@ -583,14 +583,16 @@ __device__ __forceinline__ uint32_t pf_finish_fast(uint2 h, float px, float py, 
 // Head of p's list for a caller holding the inner-grid cells [c0, c0 + S)^2
 // in shared memory (hs, row-major S x S): that copy when p falls in it and the
 // union there fits the head, else the main table (a predicated global load).
-// Without a branch: a point off the grid (or without a table, or not finite)
-// gets the no-list head, which the caller resolves with the full search.
+// Without a branch: a point off the grid (or without a table) gets the no-list
+// head, which the caller resolves with the full search.  p must be finite
+// (the encoder stores rows whose points would not be as zero rows); the grid
+// test on floor(g) is then the float test 0 <= g < G of pf_list, with G a power
+// of two.
 __device__ __forceinline__ uint2 pf_head_shared(float px, float py, const PrefilterView& pf,
                                                 const uint2* hs, int S, int c0) {
-  const float gx = fmaf(px, pf.inv_h, pf.Rih);
-  const float gy = fmaf(py, pf.inv_h, pf.Rih);
-  const bool in_grid = (gx >= 0.f) & (gx < pf.Gf) & (gy >= 0.f) & (gy < pf.Gf);
-  const int ix = in_grid ? (int)gx : 0, iy = in_grid ? (int)gy : 0;
+  const int ix = __float2int_rd(fmaf(px, pf.inv_h, pf.Rih));
+  const int iy = __float2int_rd(fmaf(py, pf.inv_h, pf.Rih));
+  const bool in_grid = ((unsigned)(ix | iy)) < (unsigned)pf.G;
   const unsigned sx = (unsigned)((ix >> 1) - c0), sy = (unsigned)((iy >> 1) - c0);
   const bool in_sq = in_grid & (sx < (unsigned)S) & (sy < (unsigned)S);
   uint2 h = make_uint2(0u, kPfMoreBit);

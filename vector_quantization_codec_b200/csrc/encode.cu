@@ -638,7 +638,10 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
       else if (isinf(__half2float(h))) flags |= QAMW_STATUS_RANGE;
     }
     uint32_t* dst = reinterpret_cast<uint32_t*>(a.packed + row * a.row_bytes) + (size_t)c * BITS;
-    if (!(r > 0.f) || !isfinite(r)) {  // zero row, or not finite (flagged): every index 0
+    const float inv = 1.0f / (r * sqrt_b);
+    // zero row, not finite (flagged), or a norm so small that 1 / (r sqrt(b))
+    // overflows (points that would not be finite): every index 0
+    if (!(r > 0.f) || !isfinite(r) || !isfinite(inv)) {
 #pragma unroll
       for (int t = 0; t < BITS; ++t) dst[t] = 0u;
     } else {
@@ -649,7 +652,6 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
           flags |= QAMW_STATUS_TIMEOUT;
         }
       }
-      const float inv = 1.0f / (r * sqrt_b);
       // each index goes to the first word of its point's slot once the point
       // has been read; the 16 indices of a half are then packed with fixed
       // shifts (LSB first, index k at bits [k BITS, (k + 1) BITS))
