@@ -129,7 +129,9 @@ def test_decode_matches_oracle(case):
 
 GEMV_CASES = [(256, 512, 64, 8, 1), (300, 1024, 128, 11, 4), (97, 4096, 1024, 7, 16),
               (64, 192, 64, 3, 3), (24, 11008, 128, 11, 13), (33, 640, 128, 9, 8),
-              (17, 128, 1, 1, 1), (16, 20480, 128, 11, 1), (10, 20480, 256, 8, 5)]
+              (17, 128, 1, 1, 1), (16, 20480, 128, 11, 1), (10, 20480, 256, 8, 5),
+              (40, 2048, 128, 11, 9), (12, 16384, 128, 11, 2), (20, 6144, 128, 11, 3),
+              (21, 6144, 128, 11, 6)]
 
 
 @pytest.mark.parametrize("case", GEMV_CASES, ids=lambda c: f"{c[0]}x{c[1]}_b{c[2]}_B{c[3]}_n{c[4]}")

@@ -13,9 +13,12 @@
 //   come from an fp16x2 copy of the codebook replicated so that a warp's 32
 //   random lookups hit at most 2 lanes per bank.  Per-slice partial dot
 //   products are summed in a fixed order (bitwise reproducible).
-// batch 2..16 (k_rotate + k_gemv): xbar for all columns is written once to the
-//   workspace (chunk-interleaved so that lanes read consecutive words), then
-//   one warp per row accumulates all batch columns.
+// batch 2..16 (k_rotate + k_gemv_s): xbar for all columns is written once to
+//   the workspace (chunk-interleaved so that lanes read consecutive words).
+//   Each CTA stages 4 or 8 of its columns in shared memory beside a replicated
+//   fp16x2 codebook, and a warp sums two rows at a time (batch 9..16: two
+//   column passes).  Where that does not fit (long rows), k_gemv reads xbar
+//   from the workspace with one warp per row.
 #include <utility>
 
 #include "common.cuh"
@@ -432,10 +435,149 @@ cudaError_t run_gemv(const qamw_matrix& m, int batch, const float2* xbar, uint16
   return cudaGetLastError();
 }
 
+// The same product with B batch columns of xbar (columns t0 .. t0 + B - 1 of
+// the workspace) staged in shared memory once per CTA.  A warp sums R
+// consecutive rows at once, lanes over the rows' chunks, so that each xbar
+// value read from shared memory serves R rows.  Codewords come from an fp16x2
+// table with 2^cl replicas of each entry, lane l reading replica l mod 2^cl, as
+// in the batch-1 kernel.  Used when B columns of xbar and the table fit in
+// shared memory.
+template <int BITS, int B, int R>
+__global__ void __launch_bounds__(512, 1) k_gemv_s(const uint8_t* __restrict__ packed,
+                                                   int64_t row_bytes, const __half* __restrict__ rnorm,
+                                                   const float2* __restrict__ codebook, int K,
+                                                   int cl, const float2* __restrict__ xbarT,
+                                                   int t0, int d_out, int d_in, int batch,
+                                                   __nv_bfloat16* __restrict__ y) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint32_t* tab = reinterpret_cast<uint32_t*>(smem);
+  float2* xs = reinterpret_cast<float2*>(smem + gemv1_table_bytes(K, cl));  // [B][P]
+  const int C = d_in / kE, P = d_in / 2;
+  const int lane = threadIdx.x & 31;
+  const int copies = 1 << cl;
+#pragma unroll 4
+  for (int j = threadIdx.x; j < K; j += blockDim.x) {
+    const float2 cw = __ldg(codebook + j);
+    const __half2 h = __floats2half2_rn(cw.x, cw.y);
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(&h);
+    for (int r = 0; r < copies; ++r) tab[(j << cl) + ((r + lane) & (copies - 1))] = u;
+  }
+  const uint32_t copy = (uint32_t)lane & (uint32_t)(copies - 1);
+  {
+    const float4* src = reinterpret_cast<const float4*>(xbarT + (int64_t)t0 * P);
+    float4* dst = reinterpret_cast<float4*>(xs);
+    const int n4 = B * P / 2;
+#pragma unroll 4
+    for (int i = threadIdx.x; i < n4; i += blockDim.x) dst[i] = __ldg(src + i);
+  }
+  __syncthreads();
+  const int warps = (gridDim.x * blockDim.x) >> 5;
+  const int nt = min(B, batch - t0);
+  for (int row = ((blockIdx.x * blockDim.x + threadIdx.x) >> 5) * R; row < d_out;
+       row += warps * R) {
+    float acc[R][B];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int t = 0; t < B; ++t) acc[r][t] = 0.f;
+    for (int c = lane; c < C; c += 32) {
+      uint32_t idx[R][kQ];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        // rows past the end read index 0 and are not written
+        uint32_t w[BITS];
+        const bool ok = row + r < d_out;
+        const uint32_t* src =
+            reinterpret_cast<const uint32_t*>(packed + (int64_t)(ok ? row + r : row) * row_bytes);
+#pragma unroll
+        for (int t = 0; t < BITS; ++t) w[t] = ok ? __ldg(src + (size_t)c * BITS + t) : 0u;
+        unpack32<BITS>(w, idx[r]);
+      }
+#pragma unroll
+      for (int q = 0; q < kQ; ++q) {
+        float2 cw[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const uint32_t h = tab[(idx[r][q] << cl) | copy];
+          cw[r] = __half22float2(*reinterpret_cast<const __half2*>(&h));
+        }
+#pragma unroll
+        for (int t = 0; t < B; ++t) {
+          const float2 xb = xs[t * P + q * C + c];
+#pragma unroll
+          for (int r = 0; r < R; ++r)
+            acc[r][t] = fmaf(xb.x, cw[r].x, fmaf(xb.y, cw[r].y, acc[r][t]));
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int t = 0; t < B; ++t) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[r][t] += __shfl_xor_sync(0xffffffffu, acc[r][t], o);
+      }
+    if (lane == 0) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        if (row + r >= d_out) break;
+        const float rn = __half2float(rnorm[row + r]);
+#pragma unroll
+        for (int t = 0; t < B; ++t)
+          if (t < nt) y[(int64_t)(t0 + t) * d_out + row + r] = __float2bfloat16_rn(acc[r][t] * rn);
+      }
+    }
+  }
+}
+
+constexpr size_t kGemvSmemCap = 200 * 1024;
+constexpr int kGemvRows = 2;  // rows per warp in k_gemv_s
+
+size_t gemv_s_smem(int K, int cl, int B, int d_in) {
+  return gemv1_table_bytes(K, cl) + (size_t)B * (d_in / 2) * sizeof(float2);
+}
+
+// Most codebook replicas (up to 16, 32 for K <= 1024) with which the table and
+// B columns of xbar fit in shared memory; -1 if not even one copy does.
+int gemv_s_copies_log2(int K, int B, int d_in) {
+  for (int cl = K <= 1024 ? 5 : 4; cl >= 0; --cl)
+    if (gemv_s_smem(K, cl, B, d_in) <= kGemvSmemCap) return cl;
+  return -1;
+}
+
+template <int BITS, int B, int R>
+cudaError_t run_gemv_s(const qamw_matrix& m, int batch, int t0, int cl, const float2* xbar,
+                       uint16_t* d_y, cudaStream_t stream) {
+  const int threads = 512, K = 1 << m.bits;
+  const size_t smem = gemv_s_smem(K, cl, B, m.d_in);
+  const void* fn = reinterpret_cast<const void*>(&k_gemv_s<BITS, B, R>);
+  cudaError_t err = allow_smem(fn, smem);
+  if (err != cudaSuccess) return err;
+  const int64_t warps = (m.d_out + R - 1) / R;
+  const int grid = persistent_grid(fn, threads, smem, (warps * 32 + threads - 1) / threads);
+  k_gemv_s<BITS, B, R><<<grid, threads, smem, stream>>>(
+      m.packed, m.row_bytes, reinterpret_cast<const __half*>(m.row_norm),
+      reinterpret_cast<const float2*>(m.codebook), K, cl, xbar, t0, m.d_out, m.d_in, batch,
+      reinterpret_cast<__nv_bfloat16*>(d_y));
+  return cudaGetLastError();
+}
+
 template <int BITS>
 cudaError_t gemv_bits(const qamw_matrix& m, const uint16_t* d_x, int batch, const float2* xbar,
                       uint16_t* d_y, int32_t* d_status, cudaStream_t stream) {
   if (batch == 1) return run_gemv1<BITS>(m, d_x, d_y, d_status, stream);
+  const int K = 1 << m.bits;
+  const int cl4 = gemv_s_copies_log2(K, 4, m.d_in), cl8 = gemv_s_copies_log2(K, 8, m.d_in);
+  if (batch <= 4 && cl4 >= 0)
+    return run_gemv_s<BITS, 4, kGemvRows>(m, batch, 0, cl4, xbar, d_y, stream);
+  if (cl8 >= 0) {  // column passes of 8
+    for (int t0 = 0; t0 < batch; t0 += 8) {
+      const cudaError_t err =
+          run_gemv_s<BITS, 8, kGemvRows>(m, batch, t0, cl8, xbar, d_y, stream);
+      if (err != cudaSuccess) return err;
+    }
+    return cudaSuccess;
+  }
   if (batch <= 4) return run_gemv<BITS, 4>(m, batch, xbar, d_y, stream);
   if (batch <= 8) return run_gemv<BITS, 8>(m, batch, xbar, d_y, stream);
   return run_gemv<BITS, 16>(m, batch, xbar, d_y, stream);
