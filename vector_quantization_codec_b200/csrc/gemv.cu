@@ -320,52 +320,65 @@ cudaError_t run_gemv1(const qamw_matrix& m, const uint16_t* d_x, uint16_t* d_y,
 // ------------------------------------------------------------- batch 2..16
 
 // xbarT[t][q][c] (float2) = pair 32c+q of xbar_t, for t < batch; zeros for
-// batch <= t < bpad; one thread per (t, chunk c).
-__global__ void __launch_bounds__(256) k_rotate(const __nv_bfloat16* __restrict__ x, int batch,
-                                                int bpad, int d_in, int block, uint64_t seed,
-                                                const __half* __restrict__ s,
-                                                const __half* __restrict__ sigma,
-                                                float2* __restrict__ xbarT, int32_t* status) {
+// batch <= t < bpad.  A CTA takes 32 consecutive (t, chunk c) items: all its
+// threads form D x / s element by element into shared memory, then one warp
+// rotates the 32 chunks from there (lane = item), so that the per-element
+// divisions and sign hashes are spread over the whole CTA.
+constexpr int kRotItems = 32;
+constexpr int kRotThreads = 256;
+
+__global__ void __launch_bounds__(kRotThreads) k_rotate(const __nv_bfloat16* __restrict__ x,
+                                                        int batch, int bpad, int d_in, int block,
+                                                        uint64_t seed,
+                                                        const __half* __restrict__ s,
+                                                        const __half* __restrict__ sigma,
+                                                        float2* __restrict__ xbarT,
+                                                        int32_t* status) {
+  __shared__ float buf[kRotItems][kE + 1];  // +1: conflict-free rows and columns
   const int C = d_in / kE, P = d_in / 2;
   const int64_t V = (int64_t)bpad * C;
   const int nb = min(block, kE), lanes = max(block / kE, 1);
   const float inv_sqrt_b = 1.0f / sqrtf((float)block);
   int flags = 0;
-  for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < V;
-       base += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t v = base + threadIdx.x;
-    const bool active = v < V;
-    const int64_t t = active ? v / C : 0;
-    const int c = active ? (int)(v - t * C) : 0;
-    const bool real = active && t < batch;
-    float xv[kE];
-    if (real) {
-      float sc[kE];
-      load64(x + t * d_in + (int64_t)c * kE, xv);
-      load_halves<kE>(s + (int64_t)c * kE, sc);
-#pragma unroll
-      for (int j = 0; j < kE; ++j) {
-        const int col = c * kE + j;
-        if (!isfinite(xv[j])) flags = QAMW_STATUS_NONFINITE;
-        const float q = __fdiv_rn(xv[j], sc[j]);
-        xv[j] = mask_negative(seed, (uint32_t)col) ? -q : q;
+  for (int64_t base = (int64_t)blockIdx.x * kRotItems; base < V;
+       base += (int64_t)gridDim.x * kRotItems) {
+    for (int e = threadIdx.x; e < kRotItems * kE; e += kRotThreads) {
+      const int i = e / kE, j = e - i * kE;
+      const int64_t v = base + i;
+      const int64_t t = v < V ? v / C : bpad;
+      float val = 0.f;
+      if (t < batch) {
+        const int col = (int)(v - t * C) * kE + j;
+        const float xv = __bfloat162float(x[t * d_in + col]);
+        if (!isfinite(xv)) flags = QAMW_STATUS_NONFINITE;
+        const float q = __fdiv_rn(xv, __half2float(s[col]));
+        val = mask_negative(seed, (uint32_t)col) ? -q : q;
       }
-    } else {
-#pragma unroll
-      for (int j = 0; j < kE; ++j) xv[j] = 0.f;
+      buf[i][j] = val;
     }
-    fwht_reg<kE>(xv, nb);
-    fwht_lanes<kE>(xv, lanes);
-    if (active) {
-      float sg[kQ];
-      load_halves<kQ>(sigma + (int64_t)c * kQ, sg);
-      float2* dst = xbarT + t * P + c;
+    __syncthreads();
+    if (threadIdx.x < 32) {  // one whole warp: the lane shuffles need all 32
+      const int64_t v = base + threadIdx.x;
+      const bool active = v < V;
+      const int64_t t = active ? v / C : 0;
+      const int c = active ? (int)(v - t * C) : 0;
+      float xv[kE];
 #pragma unroll
-      for (int q = 0; q < kQ; ++q) {
-        const float f = sg[q] * inv_sqrt_b;
-        dst[(size_t)q * C] = make_float2(xv[2 * q] * f, xv[2 * q + 1] * f);
+      for (int j = 0; j < kE; ++j) xv[j] = buf[threadIdx.x][j];
+      fwht_reg<kE>(xv, nb);
+      fwht_lanes<kE>(xv, lanes);
+      if (active) {
+        float sg[kQ];
+        load_halves<kQ>(sigma + (int64_t)c * kQ, sg);
+        float2* dst = xbarT + t * P + c;
+#pragma unroll
+        for (int q = 0; q < kQ; ++q) {
+          const float f = sg[q] * inv_sqrt_b;
+          dst[(size_t)q * C] = make_float2(xv[2 * q] * f, xv[2 * q + 1] * f);
+        }
       }
     }
+    __syncthreads();
   }
   raise_flag(status, flags);
 }
@@ -597,11 +610,10 @@ cudaError_t launch_decode_gemv(const qamw_matrix& m, const uint16_t* d_x, int ba
   float2* xbar = static_cast<float2*>(d_ws);
   if (batch > 1) {
     const int bpad = batch <= 4 ? 4 : (batch <= 8 ? 8 : 16);
-    const int threads = 256;
     const int64_t V = (int64_t)bpad * (m.d_in / kE);
     const void* fn = reinterpret_cast<const void*>(&k_rotate);
-    const int grid = persistent_grid(fn, threads, 0, (V + threads - 1) / threads);
-    k_rotate<<<grid, threads, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(d_x), batch,
+    const int grid = persistent_grid(fn, kRotThreads, 0, (V + kRotItems - 1) / kRotItems);
+    k_rotate<<<grid, kRotThreads, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(d_x), batch,
                                            bpad, m.d_in, m.block, m.mask_seed,
                                            reinterpret_cast<const __half*>(m.chan_scale),
                                            reinterpret_cast<const __half*>(m.sigma), xbar,
