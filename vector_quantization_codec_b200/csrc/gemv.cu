@@ -340,6 +340,9 @@ __global__ void __launch_bounds__(kRotThreads) k_rotate(const __nv_bfloat16* __r
   const int nb = min(block, kE), lanes = max(block / kE, 1);
   const float inv_sqrt_b = 1.0f / sqrtf((float)block);
   int flags = 0;
+  // s and sigma may come from the kernels ahead
+  pdl_wait();
+  pdl_trigger();
   for (int64_t base = (int64_t)blockIdx.x * kRotItems; base < V;
        base += (int64_t)gridDim.x * kRotItems) {
     for (int e = threadIdx.x; e < kRotItems * kE; e += kRotThreads) {
@@ -390,7 +393,7 @@ __global__ void __launch_bounds__(256) k_gemv(const uint8_t* __restrict__ packed
                                               const float2* __restrict__ codebook, int K,
                                               const float2* __restrict__ xbarT, int d_out, int d_in,
                                               int batch, __nv_bfloat16* __restrict__ y) {
-  extern __shared__ __align__(16) unsigned char smem[];
+  extern __shared__ __align__(128) unsigned char smem[];
   float2* cb = reinterpret_cast<float2*>(smem);
   for (int i = threadIdx.x; i < K; i += blockDim.x) cb[i] = codebook[i];
   __syncthreads();
@@ -462,7 +465,7 @@ __global__ void __launch_bounds__(512, 1) k_gemv_s(const uint8_t* __restrict__ p
                                                    int cl, const float2* __restrict__ xbarT,
                                                    int t0, int d_out, int d_in, int batch,
                                                    __nv_bfloat16* __restrict__ y) {
-  extern __shared__ __align__(16) unsigned char smem[];
+  extern __shared__ __align__(128) unsigned char smem[];
   uint32_t* tab = reinterpret_cast<uint32_t*>(smem);
   float2* xs = reinterpret_cast<float2*>(smem + gemv1_table_bytes(K, cl));  // [B][P]
   const int C = d_in / kE, P = d_in / 2;
@@ -476,6 +479,10 @@ __global__ void __launch_bounds__(512, 1) k_gemv_s(const uint8_t* __restrict__ p
     for (int r = 0; r < copies; ++r) tab[(j << cl) + ((r + lane) & (copies - 1))] = u;
   }
   const uint32_t copy = (uint32_t)lane & (uint32_t)(copies - 1);
+  // xbar, the indices and r_hat come from the kernels ahead; the table build
+  // above overlaps their end
+  pdl_wait();
+  pdl_trigger();
   {
     const float4* src = reinterpret_cast<const float4*>(xbarT + (int64_t)t0 * P);
     float4* dst = reinterpret_cast<float4*>(xs);
@@ -568,11 +575,11 @@ cudaError_t run_gemv_s(const qamw_matrix& m, int batch, int t0, int cl, const fl
   if (err != cudaSuccess) return err;
   const int64_t warps = (m.d_out + R - 1) / R;
   const int grid = persistent_grid(fn, threads, smem, (warps * 32 + threads - 1) / threads);
-  k_gemv_s<BITS, B, R><<<grid, threads, smem, stream>>>(
-      m.packed, m.row_bytes, reinterpret_cast<const __half*>(m.row_norm),
-      reinterpret_cast<const float2*>(m.codebook), K, cl, xbar, t0, m.d_out, m.d_in, batch,
-      reinterpret_cast<__nv_bfloat16*>(d_y));
-  return cudaGetLastError();
+  return launch_pdl(k_gemv_s<BITS, B, R>, dim3(grid), dim3(threads), smem, stream, m.packed,
+                    m.row_bytes, reinterpret_cast<const __half*>(m.row_norm),
+                    reinterpret_cast<const float2*>(m.codebook), K, cl,
+                    static_cast<const float2*>(xbar), t0, m.d_out, m.d_in, batch,
+                    reinterpret_cast<__nv_bfloat16*>(d_y));
 }
 
 template <int BITS>
@@ -613,12 +620,11 @@ cudaError_t launch_decode_gemv(const qamw_matrix& m, const uint16_t* d_x, int ba
     const int64_t V = (int64_t)bpad * (m.d_in / kE);
     const void* fn = reinterpret_cast<const void*>(&k_rotate);
     const int grid = persistent_grid(fn, kRotThreads, 0, (V + kRotItems - 1) / kRotItems);
-    k_rotate<<<grid, kRotThreads, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(d_x), batch,
-                                           bpad, m.d_in, m.block, m.mask_seed,
-                                           reinterpret_cast<const __half*>(m.chan_scale),
-                                           reinterpret_cast<const __half*>(m.sigma), xbar,
-                                           d_status);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err = launch_pdl(k_rotate, dim3(grid), dim3(kRotThreads), 0, stream,
+                                 reinterpret_cast<const __nv_bfloat16*>(d_x), batch, bpad,
+                                 m.d_in, m.block, m.mask_seed,
+                                 reinterpret_cast<const __half*>(m.chan_scale),
+                                 reinterpret_cast<const __half*>(m.sigma), xbar, d_status);
     if (err != cudaSuccess) return err;
   }
   // The batch 2..16 kernels run B = 4/8/16 columns; columns batch..B-1 read
