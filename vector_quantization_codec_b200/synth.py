@@ -104,5 +104,59 @@ def llama2_7b_layer_shapes() -> list[tuple[str, int, int]]:
 
 
 def llama_13b_layer_shapes() -> list[tuple[str, int, int]]:
+    """(name, d_out, d_in) of the seven linear weights of one 13B-shaped layer."""
     return [("q", 5120, 5120), ("k", 5120, 5120), ("v", 5120, 5120), ("o", 5120, 5120),
             ("gate", 13824, 5120), ("up", 13824, 5120), ("down", 5120, 13824)]
+
+
+# The input each linear weight of a transformer layer sees: q/k/v share the
+# attention input, gate/up share the MLP input, o and down see their own.  One
+# activation statistic is drawn per (layer, input).
+LAYER_INPUT = {"q": 0, "k": 0, "v": 0, "o": 1, "gate": 2, "up": 2, "down": 3}
+
+
+def layer_matrices(shapes: list[tuple[str, int, int]], layers: int, workload: int) -> list[dict]:
+    """Every linear weight of `layers` layers in order (layer-major), each with
+    the seeds of its weights and of its activation statistic."""
+    out = []
+    for layer in range(layers):
+        for t, (name, d_out, d_in) in enumerate(shapes):
+            out.append(dict(layer=layer, name=name, d_out=d_out, d_in=d_in,
+                            w_seed=(workload, layer, t),
+                            act_seed=(workload, layer, 100 + LAYER_INPUT[name])))
+    return out
+
+
+def act_stat_for(key: tuple, d_in: int) -> np.ndarray:
+    """act_stat_lognormal seeded by a (workload, layer, input) key."""
+    g = rng(*key, T_ACT)
+    a = g.lognormal(0.0, 1.0, size=d_in)
+    n_out = int(round(0.01 * d_in))
+    if n_out:
+        a[g.choice(d_in, size=n_out, replace=False)] *= 20.0
+    return a.astype(np.float32)
+
+
+def student_t_weights_device(d_out: int, d_in: int, key: tuple, device, out=None,
+                             scale: float = 0.02, nu: int = 5):
+    """Student-t(nu) * scale weights drawn on a CUDA device by torch's Philox
+    generator (for workloads too large to draw on the host): t = Z / sqrt(V / nu)
+    with V the sum of nu squared standard normals.  Returns bf16 [d_out, d_in]
+    (written into `out` when given).  Seeded by `key`; the values differ from
+    student_t_weights' (another generator) but follow the same distribution."""
+    import torch
+    seed = int(np.random.SeedSequence([int(k) for k in key]).generate_state(1, np.uint64)[0] >> 1)
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    if out is None:
+        out = torch.empty((d_out, d_in), dtype=torch.bfloat16, device=device)
+    rows = max(1, (1 << 26) // d_in)  # bounded temporaries
+    for r0 in range(0, d_out, rows):
+        n = min(rows, d_out - r0)
+        z = torch.randn((n, d_in), generator=g, device=device)
+        v = torch.zeros_like(z)
+        for _ in range(nu):
+            e = torch.randn((n, d_in), generator=g, device=device)
+            v.addcmul_(e, e)
+        out[r0:r0 + n] = (z * torch.rsqrt(v / nu) * scale).to(torch.bfloat16)
+    return out
