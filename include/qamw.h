@@ -271,6 +271,19 @@ QAMW_API int qamw_encode_rows_polar(const void *d_W, int dtype, const qamw_matri
  * Needs no workspace. */
 QAMW_API int qamw_decode(const qamw_matrix *m, uint16_t *d_W_out, int32_t *d_status, void *stream);
 
+/* qamw_decode for n matrices in one call: matrix i is decoded into
+ * d_W_out[i] (a host array of n device pointers, each [ms[i].d_out][ms[i].d_in]
+ * bf16, 16B-aligned; ms is a host array of n descriptors).  The result equals n
+ * qamw_decode calls.  Matrices that share bits, codebook and the class of the
+ * Hadamard block (1, or >= 2) -- consecutive in ms -- go through one kernel
+ * launch (up to 64 at a time), so the per-launch set-up (the codeword table)
+ * is paid once for the run and the tail of one matrix overlaps the next.
+ * Shapes, blocks and seeds may differ.  Errors: those of qamw_decode for any
+ * matrix (nothing is enqueued then); QAMW_ERR_INVALID for n < 0 or null
+ * arrays.  Needs no workspace. */
+QAMW_API int qamw_decode_many(const qamw_matrix *ms, int n, uint16_t *const *d_W_out,
+                              int32_t *d_status, void *stream);
+
 /* y = x * W_hat^T without forming W_hat: since R_inv = R_fwd^T,
  * y[t][i] = r_i * sum_k < xbar_t[k], c[index_ik] > with
  * xbar_t = sigma (.) R_fwd(x_t / s) (pair k = coordinates 2k, 2k+1).

@@ -326,6 +326,20 @@ int qamw_decode(const qamw_matrix* m, uint16_t* d_W_out, int32_t* d_status, void
   return cuda_rc(launch_decode(*m, d_W_out, d_status, static_cast<cudaStream_t>(stream)));
 }
 
+int qamw_decode_many(const qamw_matrix* ms, int n, uint16_t* const* d_W_out, int32_t* d_status,
+                     void* stream) {
+  if (n < 0 || (n > 0 && (!ms || !d_W_out))) return QAMW_ERR_INVALID;
+  for (int i = 0; i < n; ++i) {
+    const int rc = check_matrix(&ms[i], false);
+    if (rc != QAMW_OK) return rc;
+    if (ms[i].d_out == 0) continue;
+    if (!d_W_out[i]) return QAMW_ERR_INVALID;
+    if (!aligned16(d_W_out[i])) return QAMW_ERR_ALIGN;
+  }
+  if (n == 0) return QAMW_OK;
+  return cuda_rc(launch_decode_many(ms, n, d_W_out, d_status, static_cast<cudaStream_t>(stream)));
+}
+
 int qamw_decode_gemv(const qamw_matrix* m, const uint16_t* d_x, int batch, uint16_t* d_y,
                      void* d_workspace, size_t ws_bytes, int32_t* d_status, void* stream) {
   int rc = check_matrix(m, false);

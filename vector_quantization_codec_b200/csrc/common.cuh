@@ -51,6 +51,64 @@ __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Packed fp32x2 arithmetic (sm_100): one instruction for two lanes of a
+// float2, each rounded exactly like the scalar operation (round to nearest
+// even), so a packed butterfly gives bitwise the scalar butterfly's results.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+// a - b as fma(b, -1, a): the exact difference rounded once, as a subtraction.
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  return __ffma2_rn(b, make_float2(-1.f, -1.f), a);
+}
+
+// Sylvester butterflies of element span 2 H2 .. 32 over 64 values held as 32
+// float2 (v[i] = elements 2i, 2i + 1), the stages of span < nb only; the span-1
+// stage (within a float2) is the caller's.  Stage order and operand order are
+// those of fwht_reg, so the results are bitwise the same.
+template <int H2>
+__device__ __forceinline__ void fwht2_stage(float2 (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 2 * H2) {
+#pragma unroll
+    for (int j = i; j < i + H2; ++j) {
+      const float2 a = v[j], b = v[j + H2];
+      v[j] = add2(a, b);
+      v[j + H2] = sub2(a, b);
+    }
+  }
+}
+
+__device__ __forceinline__ void fwht2_reg(float2 (&v)[32], int nb) {
+  if (2 < nb) fwht2_stage<1>(v);
+  if (4 < nb) fwht2_stage<2>(v);
+  if (8 < nb) fwht2_stage<4>(v);
+  if (16 < nb) fwht2_stage<8>(v);
+  if (32 < nb) fwht2_stage<16>(v);
+}
+
+// fwht_lanes on float2 registers: the same fma with a +-1 factor per element.
+__device__ __forceinline__ void fwht2_lanes(float2 (&v)[32], int lanes) {
+  const unsigned lane = threadIdx.x & 31u;
+  for (int s = 1; s < lanes; s <<= 1) {
+    const float sg = (lane & (unsigned)s) ? -1.f : 1.f;
+    const float2 sg2 = make_float2(sg, sg);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      float2 o;
+      o.x = __shfl_xor_sync(0xffffffffu, v[j].x, s);
+      o.y = __shfl_xor_sync(0xffffffffu, v[j].y, s);
+      v[j] = fma2(sg2, v[j], o);
+    }
+  }
+}
+
+// Generic-proxy accesses to shared memory before this fence are ordered before
+// later asynchronous-proxy (bulk copy) accesses of the issuing thread.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void raise_flag(int32_t* status, int flag) {
   if (flag && status) atomicOr(status, flag);
 }

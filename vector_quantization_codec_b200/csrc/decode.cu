@@ -1,15 +1,36 @@
 // decode.cu -- QAM-W decoder (paper section 3.2): packed indices -> BF16 rows.
 //
-// One thread decodes one chunk of 64 columns (32 pairs) of one row:
-//   unpack its 32 indices from `bits` 32-bit words (the chunk's bit range is
-//   word aligned: 32 * bits bits), look each codeword up in shared memory,
-//   scale pair k by sigma_k, run the inverse Hadamard butterflies (in
-//   registers, then across the lanes of the block for b > 64), multiply column
-//   j by r_hat * D_j / (sqrt(b) * s_j), round to BF16; the warp then writes its
-//   4 KB of output with coalesced 16-byte stores.
-// The kernel is bound by HBM: it reads bits/16 bytes and writes 2 bytes per
-// weight.
+// Per pair k of a row: look up codeword c[idx_k], scale by sigma_k and the row
+// norm r_hat, apply R_inv = diag(D) blockdiag(H_b) / sqrt(b), divide column j by
+// the channel scale s_j, round to BF16.  The kernel is bound by HBM: it reads
+// bits/16 bytes and writes 2 bytes per weight.
+//
+// Work: a row is cut into slices of 32 chunks (2048 columns); one warp decodes
+// one (row, slice) tile at a time, lane = chunk, 64 columns per lane.  A CTA
+// (12 warps, one per SM) takes a contiguous run of tiles of one (matrix, slice)
+// -- a segment -- so the per-column factors its lanes need (sigma of 32 pairs
+// in registers, D / (sqrt(b) s) of the slice's 2048 columns in a shared table)
+// are set up once per segment, and runs of tiles of many matrices go through
+// one launch (qamw_decode_many).
+//   - each warp streams its tiles' packed words through its own 2-stage ring of
+//     cp.async.bulk copies (mbarrier completion, bounded waits), so warps never
+//     wait on one another inside a segment;
+//   - codewords come from a shared table of binary16 pairs holding (x + y,
+//     x - y) -- the first butterfly stage folded in -- with 16 (K = 2048) or
+//     32 (K <= 1024) replicas of every entry, lane l reading replica
+//     l mod replicas, so a warp's 32 random lookups rarely collide;
+//   - the other butterflies run on float2 registers with packed fp32x2
+//     arithmetic (two lanes of work per instruction, rounded as the scalar
+//     operations);
+//   - the warp's 4 KB output tile is staged in shared memory in the 128-byte
+//     swizzled layout (no bank conflicts) and written by one TMA tensor store
+//     per tile.
+#include <algorithm>
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <type_traits>
 #include <utility>
+#include <vector>
 
 #include "common.cuh"
 #include "launch.cuh"
@@ -17,292 +38,439 @@
 namespace qamw {
 namespace {
 
-struct DecodeArgs {
+constexpr int kDecWarps = 12;
+constexpr int kDecThreads = 32 * kDecWarps;
+constexpr int kDecStages = 2;
+constexpr int kSliceChunks = 32;                    // chunks of a slice (one per lane)
+constexpr int kSliceCols = kSliceChunks * kE;       // 2048
+constexpr size_t kTileBytes = 4096;                 // BF16 output of one tile
+
+// Codeword replicas (log2): 16 for K = 2048, 32 below, so that the table of
+// binary16 pairs takes at most 128 KB (lanes l and l + 16 may collide).
+constexpr int rep_log2(int bits) { return bits >= 11 ? 4 : 5; }
+
+struct DecodeMat {
   const uint8_t* packed;
   const __half* rnorm;
   const __half* sigma;
   const __half* scale;
-  const float2* codebook;
-  __nv_bfloat16* out;
-  int32_t* status;
   int64_t row_bytes;
-  int d_out, d_in, block, K;
+  int64_t item0;  // first tile of this matrix in the launch (tiles: slice-major)
+  int d_out, d_in, block;
   uint64_t seed;
 };
 
-constexpr int kDecThreads = 256;
+template <int MAXM>
+struct DecodeLaunch {
+  CUtensorMap out[MAXM];  // BF16 output of matrix i as [d_out][d_in / 64][64]
+  DecodeMat m[MAXM];
+  const float2* codebook;
+  int32_t* status;
+  int K;
+  int fold;        // table holds (x + y, x - y): every matrix has block >= 2
+  int n;           // matrices
+  int64_t items;   // tiles in all
+};
 
-// x[2q], x[2q+1] = f_q * (table entry of index q), f_q = sigma_q * r_hat; the
-// table holds (c.x + c.y, c.x - c.y) when the Hadamard block is at least 2
-// (the first butterfly stage, which pairs x[2q] with x[2q + 1]), else c.
+__host__ __device__ inline int slices_of(int d_in) {
+  return (d_in / kE + kSliceChunks - 1) / kSliceChunks;
+}
+
+__host__ __device__ inline size_t align1024(size_t v) { return (v + 1023) & ~(size_t)1023; }
+
+// Index Q of a chunk as a byte offset into a table of entries 2^SH bytes apart.
+template <int BITS, int Q, int SH>
+__device__ __forceinline__ uint32_t extract_off(const uint32_t (&w)[BITS]) {
+  constexpr int bit = Q * BITS, wi = bit >> 5, sh = bit & 31;
+  constexpr uint32_t mask = ((1u << BITS) - 1u) << SH;
+  if constexpr (sh + BITS <= 32) {
+    if constexpr (sh >= SH)
+      return (w[wi] >> (sh - SH)) & mask;
+    else
+      return (w[wi] << (SH - sh)) & mask;
+  } else {
+    return (__funnelshift_r(w[wi], w[wi + 1], sh) << SH) & mask;
+  }
+}
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+// v[q] = f_q * (table entry of index q), f_q = sigma_q * r_hat.
 template <int BITS, int... Q>
-__device__ __forceinline__ void gather_pairs(const uint32_t (&w)[BITS], uint32_t cb_s,
-                                             const float4* sg4, int C, float rn, float (&x)[kE],
-                                             std::integer_sequence<int, Q...>) {
+__device__ __forceinline__ void gather2(const uint32_t (&w)[BITS], uint32_t tab_s, uint32_t rep4,
+                                        const __half2 (&sg)[16], float rn, float2 (&v)[32],
+                                        std::integer_sequence<int, Q...>) {
+  constexpr int SH = rep_log2(BITS) + 2;
   (
       [&] {
-        const float2 cw = lds_f2(cb_s + extract_off8<BITS, Q>(w));
-        const float4 s4 = sg4[(Q / 4) * C];
-        const float sq = (Q % 4 == 0) ? s4.x : (Q % 4 == 1) ? s4.y : (Q % 4 == 2) ? s4.z : s4.w;
-        const float f = sq * rn;
-        x[2 * Q] = cw.x * f;
-        x[2 * Q + 1] = cw.y * f;
+        const uint32_t h = lds_u32(tab_s + (extract_off<BITS, Q, SH>(w) | rep4));
+        const float2 cw = __half22float2(*reinterpret_cast<const __half2*>(&h));
+        const float f = ((Q & 1) ? __high2float(sg[Q >> 1]) : __low2float(sg[Q >> 1])) * rn;
+        v[Q] = mul2(cw, make_float2(f, f));
       }(),
       ...);
 }
 
-constexpr int kDecStages = 2;
+constexpr unsigned stage_bytes(int bits) { return 128u * (unsigned)bits; }
 
-// Bytes of the input stage of one CTA iteration: its T chunks' words, the row
-// padding between them, and 16-byte alignment at both ends.
-__host__ __device__ inline unsigned decode_stage_bytes(int threads, int bits) {
-  return (unsigned)(((size_t)threads * (bits * 4 + 16) + 32 + 15) & ~(size_t)15);
+// Shared memory (from a 1024-byte aligned base): table uint32 [K][replicas]
+// (padded to 1 KB) | out tiles [12 warps][4 KB] | rings [12][2][128 bits] |
+// gtab float4 [16][32] | bars [12][2] (+ 1 KB of alignment slack).
+size_t decode_smem(int K, int bits) {
+  return 1024 + align1024((size_t)K << (rep_log2(bits) + 2)) + kDecWarps * kTileBytes +
+         (size_t)kDecWarps * kDecStages * stage_bytes(bits) + 16 * 32 * 16 +
+         kDecWarps * kDecStages * 8;
 }
 
-// Position (row, chunk) of a virtual thread v = row C + chunk, advanced by a
-// fixed step without a 64-bit division.
-struct ChunkPos {
-  int64_t r;
-  int c;
-  __device__ __forceinline__ void advance(int64_t dr, int dc, int C) {
-    r += dr;
-    c += dc;
-    if (c >= C) {
-      c -= C;
-      ++r;
-    }
+__device__ __forceinline__ void tma_store_tile(const CUtensorMap* map, uint32_t src, int x, int y,
+                                               int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(x), "r"(y), "r"(z), "r"(src)
+      : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Until the bulk stores of this thread have read their shared-memory source.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Until the bulk stores of this thread are complete.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+template <int BITS, int MAXM>
+__global__ void __launch_bounds__(kDecThreads, 1) k_decode(const __grid_constant__ DecodeLaunch<MAXM> a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  constexpr int RL = rep_log2(BITS);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // the 128-byte swizzle of the output tiles is a function of address bits
+  // 4..9: tiles start on 1024-byte boundaries
+  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const size_t tab_bytes = align1024((size_t)a.K << (RL + 2));
+  uint32_t* tab = reinterpret_cast<uint32_t*>(smem);
+  uint4* ostage = reinterpret_cast<uint4*>(smem + tab_bytes + warp * kTileBytes);
+  unsigned char* rings = smem + tab_bytes + kDecWarps * kTileBytes;
+  unsigned char* ring = rings + (size_t)warp * kDecStages * stage_bytes(BITS);
+  float4* gtab = reinterpret_cast<float4*>(rings + (size_t)kDecWarps * kDecStages * stage_bytes(BITS));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gtab + 16 * 32) + warp * kDecStages;
+
+  // the codeword table needs nothing from the kernels ahead: replica r of entry
+  // j at [j][r], written in a lane-rotated order so that a warp's stores spread
+  // over the banks
+  for (int j = tid; j < a.K; j += kDecThreads) {
+    const float2 c = __ldg(a.codebook + j);
+    const __half2 h = a.fold ? __floats2half2_rn(c.x + c.y, c.x - c.y) : __floats2half2_rn(c.x, c.y);
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(&h);
+#pragma unroll
+    for (int r = 0; r < (1 << RL); ++r) tab[(j << RL) + ((r + lane) & ((1 << RL) - 1))] = u;
   }
-};
-
-// First byte (16-byte aligned down) and length (16-byte multiple) of the packed
-// words of the virtual threads from position p0 to position p1 inclusive.
-__device__ __forceinline__ void chunk_span(const DecodeArgs& a, int BITS, const ChunkPos& p0,
-                                           const ChunkPos& p1, int64_t& start16,
-                                           unsigned& bytes) {
-  const int64_t s = p0.r * a.row_bytes + (int64_t)p0.c * BITS * 4;
-  const int64_t e = p1.r * a.row_bytes + (int64_t)(p1.c + 1) * BITS * 4;
-  start16 = s & ~(int64_t)15;
-  bytes = (unsigned)(((e + 15) & ~(int64_t)15) - start16);
-}
-
-// Per-column factors live transposed in shared memory, [position in chunk][chunk],
-// so that the 32 lanes of a warp (32 consecutive chunks) read 32 consecutive
-// words.  The packed words of each grid-stride iteration -- one contiguous byte
-// range, since consecutive virtual threads own consecutive chunks -- arrive by
-// cp.async.bulk into a 2-stage ring ahead of use (two CTAs fit on an SM).  Each warp's output -- 32
-// chunks of 64 BF16 = 4 KB, contiguous in W_hat because virtual thread v owns
-// bytes [128 v, 128 v + 128) -- is staged in a swizzled shared tile (16-byte
-// unit t of lane l at slot t ^ (l & 7), no bank conflicts on either side) and
-// written back with 512-byte coalesced stores.
-template <int BITS>
-__global__ void __launch_bounds__(kDecThreads, 2) k_decode(const DecodeArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  uint4* stage = reinterpret_cast<uint4*>(smem);  // [warps][32 lanes][8] output tile
-  const unsigned in_bytes = decode_stage_bytes(blockDim.x, BITS);
-  unsigned char* in = smem + (size_t)blockDim.x * 128;  // [kDecStages][in_bytes]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(in + (size_t)kDecStages * in_bytes);
-  int64_t* sstart = reinterpret_cast<int64_t*>(bar + kDecStages);  // first byte of each stage
-  int* issued = reinterpret_cast<int*>(sstart + kDecStages);
-  float2* cb = reinterpret_cast<float2*>(bar + 2 * kDecStages + 2);
-  const int P = a.d_in >> 1, C = a.d_in / kE;
-  float4* sg4 = reinterpret_cast<float4*>(cb + a.K);  // [q/4][c]: sigma of pairs 32c + q
-  float4* g4 = sg4 + (kQ / 4) * C;                    // [j/4][c]: D/(sqrt(b) s), column 64c + j
-  const int64_t V = (int64_t)a.d_out * C;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  // grid-stride and in-CTA steps as (rows, chunks)
-  const int64_t sdr = stride / C;
-  const int sdc = (int)(stride - sdr * C);
-  const int bdr = (int)((blockDim.x - 1) / C), bdc = (int)((blockDim.x - 1) % C);
-  const ChunkPos last{(int64_t)a.d_out - 1, C - 1};
-
-  // thread 0 issues the stage copies: ipos is the first virtual thread of the
-  // next stage to issue
-  ChunkPos ipos{0, 0};
-  auto issue = [&](int s, int64_t b0) {
-    ChunkPos p1 = ipos;
-    if (b0 + blockDim.x >= V)
-      p1 = last;
-    else
-      p1.advance(bdr, bdc, C);
-    int64_t st16;
-    unsigned nb;
-    chunk_span(a, BITS, ipos, p1, st16, nb);
-    sstart[s] = st16;
-    mbar_expect_tx(&bar[s], nb);
-    bulk_g2s(in + (size_t)s * in_bytes, a.packed + st16, nb, &bar[s]);
-    ++issued[s];
-    ipos.advance(sdr, sdc, C);
-  };
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kDecStages; ++s) {
-      mbar_init(&bar[s], 1);
-      issued[s] = 0;
-    }
+  if (lane == 0) {
+    for (int s = 0; s < kDecStages; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
   }
-  // table fills: unrolled so that each thread's loads are in flight together;
-  // the codewords as (x + y, x - y) when the block is at least 2 (the first
-  // butterfly stage, folded into the table)
-  const bool fold = a.block >= 2;
-#pragma unroll 4
-  for (int i = threadIdx.x; i < a.K; i += blockDim.x) {
-    const float2 cw = a.codebook[i];
-    cb[i] = fold ? make_float2(cw.x + cw.y, cw.x - cw.y) : cw;
-  }
-  // the indices, r_hat, sigma and s below come from the kernels ahead
+  __syncwarp();
+  // the indices, r_hat, sigma and s come from the kernels ahead
   pdl_wait();
   pdl_trigger();
-  if (threadIdx.x == 0) {
-    const int64_t b0 = (int64_t)blockIdx.x * blockDim.x;
-    ipos.r = b0 / C;
-    ipos.c = (int)(b0 - ipos.r * C);
-    for (int s = 0; s < kDecStages; ++s) {
-      if (b0 + s * stride >= V) break;
-      issue(s, b0 + s * stride);
-    }
-  }
-  fill_quads<kQ>(sg4, a.sigma, P, C, [](int, float v) { return v; });
-  const float inv_sqrt_b = 1.0f / sqrtf((float)a.block);
-  const uint64_t seed = a.seed;
-  fill_quads<kE>(g4, a.scale, a.d_in, C, [=](int j, float sv) {
-    const float v = inv_sqrt_b / sv;
-    return mask_negative(seed, (uint32_t)j) ? -v : v;
-  });
-  __syncthreads();
 
-  const int lane = threadIdx.x & 31;
-  const uint32_t cb_s = smem_u32(cb);
-  uint4* wstage = stage + (threadIdx.x >> 5) * 256;
-  const int nb = min(a.block, kE);
-  const int lanes = max(a.block / kE, 1);
-  uint4* out16 = reinterpret_cast<uint4*>(a.out);
+  const uint32_t tab_s = smem_u32(tab);
+  const uint32_t rep4 = (uint32_t)(lane & ((1 << RL) - 1)) << 2;  // this lane's replica
+  const uint32_t ostage_s = smem_u32(ostage);
+  const int64_t lo = (int64_t)blockIdx.x * a.items / gridDim.x;
+  const int64_t hi = ((int64_t)blockIdx.x + 1) * a.items / gridDim.x;
+  int mi = 0;
+  while (mi + 1 < a.n && a.m[mi + 1].item0 <= lo) ++mi;
+  unsigned it = 0;  // this warp's tiles so far (ring position)
+  // lane 0: bit s = stage s has had a copy; bit 8 + s = phase parity of its last copy
+  unsigned issued = 0;
   int flags = 0;
-  int it = 0;
-  ChunkPos pos;  // this thread's virtual thread
-  {
-    const int64_t v0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    pos.r = v0 / C;
-    pos.c = (int)(v0 - pos.r * C);
-  }
-  // r_hat of this thread's row, loaded one iteration ahead
-  __half rn_next = (int64_t)blockIdx.x * blockDim.x + threadIdx.x < V ? a.rnorm[pos.r]
-                                                                      : __float2half(0.f);
-  for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < V;
-       base += stride, ++it, pos.advance(sdr, sdc, C)) {
-    const int stg = it % kDecStages;
-    const bool active = base + threadIdx.x < V;
-    const int64_t row = active ? pos.r : 0;
-    const int c = active ? pos.c : 0;
-    const float rn = __half2float(rn_next);
+  bool abort = false;
+  for (int64_t i = lo; i < hi;) {
+    const DecodeMat& M = a.m[mi];
+    const int S = slices_of(M.d_in);
+    const int64_t end_m = M.item0 + (int64_t)S * M.d_out;
+    if (i >= end_m) {
+      ++mi;
+      continue;
+    }
+    const int64_t rel = i - M.item0;
+    const int g = (int)(rel / M.d_out);
+    const int row_a = (int)(rel - (int64_t)g * M.d_out);
+    const int64_t seg_end = min(hi, M.item0 + (int64_t)(g + 1) * M.d_out);
+    const int row_b = row_a + (int)(seg_end - i);
+    i = seg_end;
+    const int C = M.d_in / kE;
+    const int nch = min(kSliceChunks, C - g * kSliceChunks);
+    const int ntiles = row_b - row_a > warp ? (row_b - row_a - warp + kDecWarps - 1) / kDecWarps : 0;
+    const unsigned bytes = (unsigned)((nch * BITS * 4 + 15) & ~15);
+    const uint8_t* src0 = M.packed + (int64_t)g * kSliceChunks * BITS * 4;
+    const unsigned it0 = it;  // ring position of this segment's first tile
+    auto issue = [&](int k) {  // tile k of this warp in this segment
+      const unsigned st = (it0 + (unsigned)k) % kDecStages;
+      const int row = row_a + warp + k * kDecWarps;
+      mbar_expect_tx(&bars[st], bytes);
+      bulk_g2s(ring + st * stage_bytes(BITS), src0 + (int64_t)row * M.row_bytes, bytes, &bars[st]);
+      // parity of this copy's phase = (number of copies into st so far) & 1
+      issued = (issued & (1u << st)) ? (issued ^ (1u << (8 + st))) : (issued | (1u << st));
+    };
+    if (lane == 0 && !abort)
+      for (int k = 0; k < min(kDecStages, ntiles); ++k) issue(k);
+    // the slice's output factors g_j = D_j / (sqrt(b) s_j), shared by the CTA
+    if (__syncthreads_or(abort)) break;  // every warp is done with the last segment's table
     {
-      ChunkPos nxt = pos;
-      nxt.advance(sdr, sdc, C);
-      rn_next = base + stride + threadIdx.x < V ? a.rnorm[nxt.r] : __float2half(0.f);
+      const float inv_sqrt_b = 1.0f / sqrtf((float)M.block);
+      const int col0 = g * kSliceCols;
+      for (int t = tid; t < nch * 16; t += kDecThreads) {  // gtab[(j/4)][c] = g of column 64c + j
+        const int c = t % nch, j4 = t / nch;
+        const int col = col0 + c * kE + 4 * j4;
+        const uint2 sv = __ldg(reinterpret_cast<const uint2*>(M.scale + col));
+        const float2 lo2 = __half22float2(*reinterpret_cast<const __half2*>(&sv.x));
+        const float2 hi2 = __half22float2(*reinterpret_cast<const __half2*>(&sv.y));
+        const float sv4[4] = {lo2.x, lo2.y, hi2.x, hi2.y};
+        float gv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float v = inv_sqrt_b / sv4[e];
+          gv[e] = mask_negative(M.seed, (uint32_t)(col + e)) ? -v : v;
+        }
+        gtab[j4 * 32 + c] = make_float4(gv[0], gv[1], gv[2], gv[3]);
+      }
     }
-    const bool ok = mbar_wait_bounded(&bar[stg], (unsigned)(it / kDecStages) & 1u);
-    if (__syncthreads_or(!ok)) {
-      flags |= QAMW_STATUS_TIMEOUT;
-      break;
-    }
-
-    uint32_t w[BITS];
+    // sigma of this lane's 32 pairs (binary16, as stored), into registers
+    const bool active = lane < nch;
+    __half2 sg[16];
     {
-      const int64_t off = active ? row * a.row_bytes + (int64_t)c * BITS * 4 - sstart[stg] : 0;
-      const uint32_t* src = reinterpret_cast<const uint32_t*>(in + (size_t)stg * in_bytes + off);
+      const uint4* sp = reinterpret_cast<const uint4*>(M.sigma + (int64_t)(g * kSliceChunks + lane) * kQ);
 #pragma unroll
-      for (int t = 0; t < BITS; ++t) w[t] = active ? src[t] : 0u;
-    }
-    __syncthreads();  // every thread has its words: the stage can be refilled
-    if (threadIdx.x == 0) {
-      const int64_t b2 = base + (int64_t)kDecStages * stride;
-      if (b2 < V) issue(stg, b2);
-    }
-
-    float x[kE];
-    gather_pairs<BITS>(w, cb_s, sg4 + c, C, rn, x, std::make_integer_sequence<int, kQ>{});
-    fwht_reg<kE, 2>(x, nb);  // stage 1 is in the table
-    fwht_lanes<kE>(x, lanes);
+      for (int t = 0; t < 4; ++t) {
+        const uint4 u = active ? __ldg(sp + t) : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int t = 0; t < kE / 8; ++t) {
-      const float4 g0 = g4[(2 * t) * C + c], g1 = g4[(2 * t + 1) * C + c];
-      const int j = 8 * t;
-      wstage[lane * 8 + (t ^ (lane & 7))] =
-          make_uint4(pack_bf16x2(x[j] * g0.x, x[j + 1] * g0.y), pack_bf16x2(x[j + 2] * g0.z, x[j + 3] * g0.w),
-                     pack_bf16x2(x[j + 4] * g1.x, x[j + 5] * g1.y), pack_bf16x2(x[j + 6] * g1.z, x[j + 7] * g1.w));
+        for (int e = 0; e < 4; ++e) sg[4 * t + e] = *reinterpret_cast<const __half2*>(&uu[e]);
+      }
     }
-    __syncwarp();
-    // unit uu = 32 i + lane of this warp's 4 KB belongs to lane uu / 8, slot uu % 8
-    const int64_t wbase = base + (threadIdx.x & ~31);
+    __syncthreads();
+    const int nb = min(M.block, kE);
+    const int lanes = max(M.block / kE, 1);
+    const CUtensorMap* omap = &a.out[mi];
+    // the tiles of this segment; the in-register butterfly stages are
+    // straight-line code when the block spans at least a whole chunk (a run-time
+    // test per stage would make the compiler move every value back into fixed
+    // registers after each stage)
+    auto tiles = [&](auto full) {
+      constexpr bool FULL = decltype(full)::value;
+      for (int k = 0; k < ntiles && !abort; ++k, ++it) {
+        const unsigned st = it % kDecStages;
+        const int row = row_a + warp + k * kDecWarps;
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars[st], (it / kDecStages) & 1u))) {
+          flags |= QAMW_STATUS_TIMEOUT;
+          abort = true;
+          break;
+        }
+        uint32_t w[BITS];
+        {
+          const uint32_t* src = reinterpret_cast<const uint32_t*>(ring + st * stage_bytes(BITS)) + lane * BITS;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int uu = 32 * i + lane, owner = uu >> 3, t = uu & 7;
-      if (wbase + owner < V) out16[(wbase + owner) * 8 + t] = wstage[owner * 8 + (t ^ (owner & 7))];
-    }
-    __syncwarp();
+          for (int t = 0; t < BITS; ++t) w[t] = active ? src[t] : 0u;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && k + kDecStages < ntiles) issue(k + kDecStages);
+        const float rn = __half2float(M.rnorm[row]);
+        float2 v[32];
+        gather2<BITS>(w, tab_s, rep4, sg, rn, v, std::make_integer_sequence<int, 32>{});
+        // the span-1 stage is in the table
+        if constexpr (FULL) {  // block >= 64: every in-register stage, straight-line
+          fwht2_stage<1>(v);
+          fwht2_stage<2>(v);
+          fwht2_stage<4>(v);
+          fwht2_stage<8>(v);
+          fwht2_stage<16>(v);
+        } else {
+          fwht2_reg(v, nb);
+        }
+        fwht2_lanes(v, lanes);
+        // the previous tile's store has read its source: the stage can be refilled
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const float4 g0 = gtab[(2 * t) * 32 + lane], g1 = gtab[(2 * t + 1) * 32 + lane];
+          const float2 p0 = mul2(v[4 * t], make_float2(g0.x, g0.y));
+          const float2 p1 = mul2(v[4 * t + 1], make_float2(g0.z, g0.w));
+          const float2 p2 = mul2(v[4 * t + 2], make_float2(g1.x, g1.y));
+          const float2 p3 = mul2(v[4 * t + 3], make_float2(g1.z, g1.w));
+          ostage[lane * 8 + (t ^ (lane & 7))] =
+              make_uint4(pack_bf16x2(p0.x, p0.y), pack_bf16x2(p1.x, p1.y), pack_bf16x2(p2.x, p2.y),
+                         pack_bf16x2(p3.x, p3.y));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        // chunks past the row's end (a ragged last slice) fall outside the
+        // tensor and are not written
+        if (lane == 0) tma_store_tile(omap, ostage_s, 0, g * kSliceChunks, row);
+      }
+    };
+    if (nb == kE)
+      tiles(std::true_type{});
+    else
+      tiles(std::false_type{});
   }
-  // after a timeout: let the copies still in flight land before this CTA's
-  // shared memory goes away
-  __syncthreads();
-  if (threadIdx.x == 0) {
+  // copies still in flight (after a timeout) land before the CTA's shared
+  // memory goes away; the output stores complete
+  if (lane == 0) {
     for (int s = 0; s < kDecStages; ++s)
-      if (issued[s] > 0) mbar_wait_bounded(&bar[s], (unsigned)(issued[s] - 1) & 1u);
+      if (issued & (1u << s)) mbar_wait_bounded(&bars[s], (issued >> (8 + s)) & 1u);
+    bulk_wait_all();
   }
   raise_flag(a.status, flags);
 }
 
-size_t decode_smem(int threads, const DecodeArgs& a, int bits) {
-  return (size_t)threads * 128 + (size_t)kDecStages * decode_stage_bytes(threads, bits) +
-         (2 * kDecStages + 2) * sizeof(uint64_t) + (size_t)a.K * sizeof(float2) +
-         (size_t)(a.d_in / 2) * sizeof(float) + (size_t)a.d_in * sizeof(float);
+// cuTensorMapEncodeTiled from the driver, looked up once.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
 }
 
-template <int BITS>
-cudaError_t run_decode(const DecodeArgs& a, cudaStream_t stream) {
-  // 256 threads, or 128 when the per-column tables of a very wide matrix leave
-  // no room for a 32 KB staging tile within the 227 KB a CTA may use
-  const int threads =
-      decode_smem(kDecThreads, a, BITS) <= 227 * 1024 ? kDecThreads : kDecThreads / 2;
-  const size_t smem = decode_smem(threads, a, BITS);
-  const void* fn = reinterpret_cast<const void*>(&k_decode<BITS>);
+// BF16 [d_out][d_in] seen as [d_out][d_in / 64][64] for tile stores of
+// {64 columns, 32 chunks, 1 row} in the 128-byte swizzled layout.
+bool encode_out_map(CUtensorMap* map, void* out, int d_out, int d_in) {
+  const auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)kE, (cuuint64_t)(d_in / kE), (cuuint64_t)d_out};
+  const cuuint64_t strides[2] = {(cuuint64_t)kE * 2, (cuuint64_t)d_in * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)kE, (cuuint32_t)kSliceChunks, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, out, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MAXM>
+bool fill_launch(DecodeLaunch<MAXM>& L, const qamw_matrix* const* ms, int n, uint16_t* const* outs,
+                 int32_t* d_status) {
+  L.codebook = reinterpret_cast<const float2*>(ms[0]->codebook);
+  L.status = d_status;
+  L.K = 1 << ms[0]->bits;
+  L.fold = ms[0]->block >= 2;
+  L.n = n;
+  int64_t item = 0;
+  for (int i = 0; i < n; ++i) {
+    const qamw_matrix& m = *ms[i];
+    DecodeMat& d = L.m[i];
+    d.packed = m.packed;
+    d.rnorm = reinterpret_cast<const __half*>(m.row_norm);
+    d.sigma = reinterpret_cast<const __half*>(m.sigma);
+    d.scale = reinterpret_cast<const __half*>(m.chan_scale);
+    d.row_bytes = m.row_bytes;
+    d.item0 = item;
+    d.d_out = m.d_out;
+    d.d_in = m.d_in;
+    d.block = m.block;
+    d.seed = m.mask_seed;
+    if (!encode_out_map(&L.out[i], outs[i], m.d_out, m.d_in)) return false;
+    item += (int64_t)slices_of(m.d_in) * m.d_out;
+  }
+  L.items = item;
+  return true;
+}
+
+template <int BITS, int MAXM>
+cudaError_t run_decode(const qamw_matrix* const* ms, int n, uint16_t* const* outs, int32_t* d_status,
+                       cudaStream_t stream) {
+  static_assert(sizeof(DecodeLaunch<MAXM>) <= 32000, "kernel parameters");
+  DecodeLaunch<MAXM> L;
+  if (!fill_launch<MAXM>(L, ms, n, outs, d_status)) return cudaErrorInvalidValue;
+  if (L.items == 0) return cudaSuccess;
+  const size_t smem = decode_smem(L.K, BITS);
+  const void* fn = reinterpret_cast<const void*>(&k_decode<BITS, MAXM>);
   cudaError_t err = allow_smem(fn, smem);
   if (err != cudaSuccess) return err;
-  const int64_t V = (int64_t)a.d_out * (a.d_in / kE);
-  const int grid = persistent_grid(fn, threads, smem, (V + threads - 1) / threads);
-  return launch_pdl(k_decode<BITS>, dim3(grid), dim3(threads), smem, stream, a);
+  // one CTA per SM; at least a few tiles per warp
+  int64_t grid = (L.items + 4 * kDecWarps - 1) / (4 * kDecWarps);
+  grid = std::min<int64_t>(std::max<int64_t>(grid, 1), sm_count());
+  return launch_pdl(k_decode<BITS, MAXM>, dim3((unsigned)grid), dim3(kDecThreads), smem, stream, L);
+}
+
+constexpr int kManyMax = 64;  // matrices per launch of qamw_decode_many
+
+template <int BITS>
+cudaError_t decode_bits(const qamw_matrix* const* ms, int n, uint16_t* const* outs,
+                        int32_t* d_status, cudaStream_t stream) {
+  if (n == 1) return run_decode<BITS, 1>(ms, 1, outs, d_status, stream);
+  for (int i = 0; i < n; i += kManyMax) {
+    const cudaError_t err =
+        run_decode<BITS, kManyMax>(ms + i, std::min(kManyMax, n - i), outs + i, d_status, stream);
+    if (err != cudaSuccess) return err;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t decode_group(const qamw_matrix* const* ms, int n, uint16_t* const* outs,
+                         int32_t* d_status, cudaStream_t stream) {
+  switch (ms[0]->bits) {
+    case 1: return decode_bits<1>(ms, n, outs, d_status, stream);
+    case 2: return decode_bits<2>(ms, n, outs, d_status, stream);
+    case 3: return decode_bits<3>(ms, n, outs, d_status, stream);
+    case 4: return decode_bits<4>(ms, n, outs, d_status, stream);
+    case 5: return decode_bits<5>(ms, n, outs, d_status, stream);
+    case 6: return decode_bits<6>(ms, n, outs, d_status, stream);
+    case 7: return decode_bits<7>(ms, n, outs, d_status, stream);
+    case 8: return decode_bits<8>(ms, n, outs, d_status, stream);
+    case 9: return decode_bits<9>(ms, n, outs, d_status, stream);
+    case 10: return decode_bits<10>(ms, n, outs, d_status, stream);
+    case 11: return decode_bits<11>(ms, n, outs, d_status, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const qamw_matrix& m, uint16_t* d_out, int32_t* d_status,
                           cudaStream_t stream) {
-  DecodeArgs a;
-  a.status = d_status;
-  a.packed = m.packed;
-  a.rnorm = reinterpret_cast<const __half*>(m.row_norm);
-  a.sigma = reinterpret_cast<const __half*>(m.sigma);
-  a.scale = reinterpret_cast<const __half*>(m.chan_scale);
-  a.codebook = reinterpret_cast<const float2*>(m.codebook);
-  a.out = reinterpret_cast<__nv_bfloat16*>(d_out);
-  a.row_bytes = m.row_bytes;
-  a.d_out = m.d_out;
-  a.d_in = m.d_in;
-  a.block = m.block;
-  a.K = 1 << m.bits;
-  a.seed = m.mask_seed;
-  switch (m.bits) {
-    case 1: return run_decode<1>(a, stream);
-    case 2: return run_decode<2>(a, stream);
-    case 3: return run_decode<3>(a, stream);
-    case 4: return run_decode<4>(a, stream);
-    case 5: return run_decode<5>(a, stream);
-    case 6: return run_decode<6>(a, stream);
-    case 7: return run_decode<7>(a, stream);
-    case 8: return run_decode<8>(a, stream);
-    case 9: return run_decode<9>(a, stream);
-    case 10: return run_decode<10>(a, stream);
-    case 11: return run_decode<11>(a, stream);
-    default: return cudaErrorInvalidValue;
+  const qamw_matrix* p = &m;
+  return decode_group(&p, 1, &d_out, d_status, stream);
+}
+
+cudaError_t launch_decode_many(const qamw_matrix* ms, int n, uint16_t* const* d_outs,
+                               int32_t* d_status, cudaStream_t stream) {
+  // one launch per run of up to kManyMax matrices with the same table: same
+  // bits and codebook, and the first butterfly folded (block >= 2) or not
+  std::vector<const qamw_matrix*> group;
+  std::vector<uint16_t*> gout;
+  auto flush = [&]() -> cudaError_t {
+    if (group.empty()) return cudaSuccess;
+    const cudaError_t e = decode_group(group.data(), (int)group.size(), gout.data(), d_status, stream);
+    group.clear();
+    gout.clear();
+    return e;
+  };
+  for (int i = 0; i < n; ++i) {
+    if (ms[i].d_out == 0) continue;
+    if (!group.empty()) {
+      const qamw_matrix& f = *group[0];
+      if (f.bits != ms[i].bits || f.codebook != ms[i].codebook || (f.block >= 2) != (ms[i].block >= 2)) {
+        const cudaError_t e = flush();
+        if (e != cudaSuccess) return e;
+      }
+    }
+    group.push_back(&ms[i]);
+    gout.push_back(d_outs[i]);
   }
+  return flush();
 }
 
 }  // namespace qamw

@@ -74,6 +74,8 @@ size_t gemv_workspace_bytes(int d_in, int batch);
 
 cudaError_t launch_decode(const qamw_matrix& m, uint16_t* d_out_bf16, int32_t* d_status,
                           cudaStream_t stream);
+cudaError_t launch_decode_many(const qamw_matrix* ms, int n, uint16_t* const* d_outs,
+                               int32_t* d_status, cudaStream_t stream);
 cudaError_t launch_channel_scales(const float* d_act_stat, int d_in, float alpha, uint16_t* d_scale,
                                   int32_t* d_status, cudaStream_t stream);
 cudaError_t launch_calibrate(const void* d_W, int dtype, const qamw_matrix& m,

@@ -44,7 +44,8 @@ QAMW_OP_CALIBRATE = 3
 EXPORTS = ("qamw_row_bytes", "qamw_default_block", "qamw_bits_per_weight",
            "qamw_workspace_bytes", "qamw_prefilter_bytes", "qamw_status_string",
            "qamw_train_codebook", "qamw_build_prefilter", "qamw_encode", "qamw_channel_scales",
-           "qamw_calibrate_sigma", "qamw_encode_rows", "qamw_decode", "qamw_decode_gemv",
+           "qamw_calibrate_sigma", "qamw_encode_rows", "qamw_decode", "qamw_decode_many",
+           "qamw_decode_gemv",
            "qamw_decode_gemv_noalloc", "qamw_polar_codebook", "qamw_encode_rows_polar",
            "qamw_normalised_pairs", "qamw_selftest_wait_timeout")
 
@@ -82,6 +83,7 @@ def _load() -> C.CDLL:
         "qamw_calibrate_sigma": (I, [V, I, C.POINTER(qamw_matrix), V, SZ, V, V]),
         "qamw_encode_rows": (I, [V, I, C.POINTER(qamw_matrix), V, V, V]),
         "qamw_decode": (I, [C.POINTER(qamw_matrix), V, V, V]),
+        "qamw_decode_many": (I, [C.POINTER(qamw_matrix), I, C.POINTER(C.c_void_p), V, V]),
         "qamw_decode_gemv": (I, [C.POINTER(qamw_matrix), V, I, V, V, SZ, V, V]),
         "qamw_decode_gemv_noalloc": (I, [C.POINTER(qamw_matrix), V, I, V, V, V]),
         "qamw_polar_codebook": (I, [I, V, V]),
@@ -322,6 +324,20 @@ def qamw_decode(m: EncodedMatrix, out: torch.Tensor | None = None,
     rc = _lib.qamw_decode(C.byref(st), _p(out), _p(status), _s(stream))
     _check("qamw_decode", rc)
     return out
+
+
+def qamw_decode_many(ms: list, outs: list | None = None, status: torch.Tensor | None = None,
+                     stream=None) -> list:
+    """qamw_decode of every matrix of `ms` in one call (bf16 [d_out, d_in] each)."""
+    if outs is None:
+        outs = [torch.empty((m.d_out, m.d_in), dtype=torch.bfloat16, device=m.packed.device)
+                for m in ms]
+    n = len(ms)
+    arr = (qamw_matrix * max(n, 1))(*[m.struct() for m in ms])
+    ptrs = (C.c_void_p * max(n, 1))(*[o.data_ptr() for o in outs])
+    rc = _lib.qamw_decode_many(arr, n, ptrs, _p(status), _s(stream))
+    _check("qamw_decode_many", rc)
+    return outs
 
 
 def qamw_decode_gemv(m: EncodedMatrix, x: torch.Tensor, y: torch.Tensor | None = None,
