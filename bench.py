@@ -307,9 +307,8 @@ class Workload:
                                         torch.empty_like(m.packed), torch.empty_like(m.row_norm),
                                         m.sigma, m.chan_scale, polar_codebook, None)
                 self.m_polar.append(mp)
-        cal = max(qamw.qamw_workspace_bytes(qamw.QAMW_OP_CALIBRATE, d["d_out"], d["d_in"], bits)
-                  for d in mats)
-        self.ws_cal = torch.empty(cal, dtype=torch.uint8, device=dev)
+        self.ws_cal = torch.empty(qamw.qamw_calibrate_many_workspace_bytes(self.m), dtype=torch.uint8,
+                                  device=dev)
         gw = max(qamw.qamw_workspace_bytes(qamw.QAMW_OP_GEMV, d["d_out"], d["d_in"], bits, 16)
                  for d in mats)
         self.ws_gemv = torch.empty(gw, dtype=torch.uint8, device=dev)
@@ -319,12 +318,12 @@ class Workload:
     def weights(self) -> int:
         return sum(d["d_out"] * d["d_in"] for d in self.mats)
 
-    # one C-ABI call per matrix per stage, on the current stream
+    # the calls of each stage, on the current stream
     def calibrate(self, stream=None):
+        # channel scales and eq. (1) of every matrix in one call
         from vector_quantization_codec_b200 import qamw
-        for W, a, m in zip(self.W, self.act, self.m):
-            qamw.qamw_channel_scales(m.d_in, a, ALPHA, m.chan_scale, status=self.status, stream=stream)
-            qamw.qamw_calibrate_sigma(W, m, workspace=self.ws_cal, status=self.status, stream=stream)
+        qamw.qamw_calibrate_many(self.W, self.m, self.act, ALPHA, workspace=self.ws_cal,
+                                 status=self.status, stream=stream)
 
     def encode(self, stream=None, candidates=None):
         from vector_quantization_codec_b200 import qamw
@@ -485,8 +484,9 @@ def run_gpu(args) -> dict | None:
     enc_ms, dec_ms, gemv_ms = phase_ms["encode"], phase_ms["decode"], phase_ms["gemv"]
     enc_roof = encoder_roofline(ab["encode"], flops, enc_ms, hbm, sm_mhz)
     comp = {
-        "calibrate": dict(ms=phase_ms["calibrate"], launches=nm * 4,
-                          note="channel scales + eq.(1) over the first 1024 rows, per matrix"),
+        "calibrate": dict(ms=phase_ms["calibrate"], launches=4 * ((nm + 63) // 64),
+                          note="channel scales + eq.(1) over the first 1024 rows of every matrix "
+                               "(qamw_calibrate_many)"),
         "encode": dict(ms=enc_ms, Mweights_per_s=weights / (enc_ms * 1e-3) / 1e6,
                        fp32_tflops=flops / (enc_ms * 1e-3) / 1e12,
                        frac_fp32_at_run_clock=flops / (enc_ms * 1e-3) / 1e12 / fp32_peak_tflops(sm_mhz),
@@ -549,14 +549,14 @@ def run_gpu(args) -> dict | None:
     return out
 
 
-# kernels one matrix launches per step: scales 1, calibrate 3 (rows, extension,
-# finish), encode 1, decode-GEMV 1 (batch 1); the decode phase is one
-# qamw_decode_many call, one launch per 64 matrices
-LAUNCHES_PER_MATRIX = 6
+# kernels of one step: per matrix, encode 1 and decode-GEMV 1 (batch 1); per
+# group of 64 matrices, calibration 4 (scales, rows, extension, finish) and
+# decode 1
+LAUNCHES_PER_MATRIX = 2
 
 
 def launches_per_step(n_matrices: int) -> int:
-    return n_matrices * LAUNCHES_PER_MATRIX + (n_matrices + 63) // 64
+    return n_matrices * LAUNCHES_PER_MATRIX + 5 * ((n_matrices + 63) // 64)
 
 
 def run_gemv_lines(args, wl, dev, stream, hbm) -> dict:

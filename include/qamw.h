@@ -219,6 +219,26 @@ QAMW_API int qamw_calibrate_sigma(const void *d_W, int dtype, const qamw_matrix 
                                   void *d_workspace, size_t ws_bytes, int32_t *d_status,
                                   void *stream);
 
+/* qamw_calibrate_many: qamw_channel_scales followed by qamw_calibrate_sigma
+ *   for each of n matrices, in four kernel launches per 64 matrices instead of
+ *   four per matrix (the results are bitwise those of the single calls).
+ *   d_W[i]: matrix i's weights (dtype as for qamw_encode, 16B-aligned);
+ *   d_act_stat: NULL, or n statistic pointers (each nullable: s = 1); alpha
+ *   applies to all; ms[i]: shape, block, mask_seed and the chan_scale and
+ *   sigma arrays written (packed and row_norm are not touched).  d_W,
+ *   d_act_stat and ms are host arrays of n entries.  Shapes may differ;
+ *   every d_out must be positive.
+ *   d_workspace: qamw_calibrate_many_workspace_bytes(ms, n) bytes (16B-aligned).
+ *   Errors: those of qamw_calibrate_sigma for any matrix (nothing is enqueued
+ *   then).  Flags: BAD_STAT, RANGE, NONFINITE. */
+QAMW_API int qamw_calibrate_many(const void *const *d_W, int dtype, const float *const *d_act_stat,
+                                 float alpha, const qamw_matrix *ms, int n, void *d_workspace,
+                                 size_t ws_bytes, int32_t *d_status, void *stream);
+
+/* Bytes of d_workspace qamw_calibrate_many needs for these n matrices (0 for
+ * invalid arguments). */
+QAMW_API size_t qamw_calibrate_many_workspace_bytes(const qamw_matrix *ms, int n);
+
 /* qamw_encode_rows: section 3.1 steps 1-6 for every row with the given
  *   m->chan_scale and m->sigma; writes m->packed and m->row_norm.  One kernel,
  *   no workspace.  m->prefilter may be NULL (exhaustive search; same result,

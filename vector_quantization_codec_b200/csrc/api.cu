@@ -272,6 +272,34 @@ int qamw_calibrate_sigma(const void* d_W, int dtype, const qamw_matrix* m, void*
   return cuda_rc(launch_calibrate(d_W, dtype, *m, ws, d_status, static_cast<cudaStream_t>(stream)));
 }
 
+size_t qamw_calibrate_many_workspace_bytes(const qamw_matrix* ms, int n) {
+  if (n <= 0 || !ms) return 0;
+  for (int i = 0; i < n; ++i)
+    if (ms[i].d_in <= 0 || ms[i].d_in % kE || ms[i].d_in > kMaxDin) return 0;
+  return calibrate_many_workspace_bytes(ms, n);
+}
+
+int qamw_calibrate_many(const void* const* d_W, int dtype, const float* const* d_act_stat,
+                        float alpha, const qamw_matrix* ms, int n, void* d_workspace,
+                        size_t ws_bytes, int32_t* d_status, void* stream) {
+  if (n < 0 || (n > 0 && (!ms || !d_W))) return QAMW_ERR_INVALID;
+  if (dtype != QAMW_DTYPE_F32 && dtype != QAMW_DTYPE_BF16) return QAMW_ERR_INVALID;
+  if (!std::isfinite(alpha)) return QAMW_ERR_INVALID;
+  if (n == 0) return QAMW_OK;
+  for (int i = 0; i < n; ++i) {
+    const int rc = check_matrix(&ms[i], true);
+    if (rc != QAMW_OK) return rc;
+    if (ms[i].d_out == 0) return QAMW_ERR_SHAPE;
+    if (!d_W[i]) return QAMW_ERR_INVALID;
+    if (!aligned16(d_W[i])) return QAMW_ERR_ALIGN;
+  }
+  const size_t need = calibrate_many_workspace_bytes(ms, n);
+  if (!d_workspace || ws_bytes < need) return QAMW_ERR_WORKSPACE;
+  if (!aligned16(d_workspace)) return QAMW_ERR_ALIGN;
+  return cuda_rc(launch_calibrate_many(d_W, dtype, d_act_stat, alpha, ms, n, d_workspace, d_status,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
 int qamw_encode_rows(const void* d_W, int dtype, const qamw_matrix* m, uint64_t* d_candidates,
                      int32_t* d_status, void* stream) {
   int rc = check_matrix(m, true);

@@ -15,10 +15,10 @@
 //   - each warp streams its tiles' packed words through its own 2-stage ring of
 //     cp.async.bulk copies (mbarrier completion, bounded waits), so warps never
 //     wait on one another inside a segment;
-//   - codewords come from a shared table of binary16 pairs holding (x + y,
-//     x - y) -- the first butterfly stage folded in -- with 16 (K = 2048) or
-//     32 (K <= 1024) replicas of every entry, lane l reading replica
-//     l mod replicas, so a warp's 32 random lookups rarely collide;
+//   - codewords come from a shared table of fp32 pairs holding (x + y, x - y)
+//     -- the first butterfly stage folded in -- with 8 (K = 2048), 16
+//     (K = 1024) or 32 (K <= 512) replicas of every entry, lane l reading
+//     replica l mod replicas, so a warp's 32 random lookups rarely collide;
 //   - the other butterflies run on float2 registers with packed fp32x2
 //     arithmetic (two lanes of work per instruction, rounded as the scalar
 //     operations);
@@ -45,9 +45,11 @@ constexpr int kSliceChunks = 32;                    // chunks of a slice (one pe
 constexpr int kSliceCols = kSliceChunks * kE;       // 2048
 constexpr size_t kTileBytes = 4096;                 // BF16 output of one tile
 
-// Codeword replicas (log2): 16 for K = 2048, 32 below, so that the table of
-// binary16 pairs takes at most 128 KB (lanes l and l + 16 may collide).
-constexpr int rep_log2(int bits) { return bits >= 11 ? 4 : 5; }
+// Codeword replicas (log2): 8 for K = 2048, 16 for K = 1024, 32 below, so that
+// the table of fp32 pairs takes at most 128 KB.  (A binary16 table would halve
+// it, but its rounding alone uses ~70% of the 1e-2 elementwise tolerance on
+// columns with small channel scales.)
+constexpr int rep_log2(int bits) { return bits >= 11 ? 3 : (bits == 10 ? 4 : 5); }
 
 struct DecodeMat {
   const uint8_t* packed;
@@ -93,22 +95,15 @@ __device__ __forceinline__ uint32_t extract_off(const uint32_t (&w)[BITS]) {
   }
 }
 
-__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-  return v;
-}
-
 // v[q] = f_q * (table entry of index q), f_q = sigma_q * r_hat.
 template <int BITS, int... Q>
-__device__ __forceinline__ void gather2(const uint32_t (&w)[BITS], uint32_t tab_s, uint32_t rep4,
+__device__ __forceinline__ void gather2(const uint32_t (&w)[BITS], uint32_t tab_s, uint32_t rep8,
                                         const __half2 (&sg)[16], float rn, float2 (&v)[32],
                                         std::integer_sequence<int, Q...>) {
-  constexpr int SH = rep_log2(BITS) + 2;
+  constexpr int SH = rep_log2(BITS) + 3;
   (
       [&] {
-        const uint32_t h = lds_u32(tab_s + (extract_off<BITS, Q, SH>(w) | rep4));
-        const float2 cw = __half22float2(*reinterpret_cast<const __half2*>(&h));
+        const float2 cw = lds_f2(tab_s + (extract_off<BITS, Q, SH>(w) | rep8));
         const float f = ((Q & 1) ? __high2float(sg[Q >> 1]) : __low2float(sg[Q >> 1])) * rn;
         v[Q] = mul2(cw, make_float2(f, f));
       }(),
@@ -117,11 +112,11 @@ __device__ __forceinline__ void gather2(const uint32_t (&w)[BITS], uint32_t tab_
 
 constexpr unsigned stage_bytes(int bits) { return 128u * (unsigned)bits; }
 
-// Shared memory (from a 1024-byte aligned base): table uint32 [K][replicas]
+// Shared memory (from a 1024-byte aligned base): table float2 [K][replicas]
 // (padded to 1 KB) | out tiles [12 warps][4 KB] | rings [12][2][128 bits] |
 // gtab float4 [16][32] | bars [12][2] (+ 1 KB of alignment slack).
 size_t decode_smem(int K, int bits) {
-  return 1024 + align1024((size_t)K << (rep_log2(bits) + 2)) + kDecWarps * kTileBytes +
+  return 1024 + align1024((size_t)K << (rep_log2(bits) + 3)) + kDecWarps * kTileBytes +
          (size_t)kDecWarps * kDecStages * stage_bytes(bits) + 16 * 32 * 16 +
          kDecWarps * kDecStages * 8;
 }
@@ -152,8 +147,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const __grid_constant
   // the 128-byte swizzle of the output tiles is a function of address bits
   // 4..9: tiles start on 1024-byte boundaries
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  const size_t tab_bytes = align1024((size_t)a.K << (RL + 2));
-  uint32_t* tab = reinterpret_cast<uint32_t*>(smem);
+  const size_t tab_bytes = align1024((size_t)a.K << (RL + 3));
+  float2* tab = reinterpret_cast<float2*>(smem);
   uint4* ostage = reinterpret_cast<uint4*>(smem + tab_bytes + warp * kTileBytes);
   unsigned char* rings = smem + tab_bytes + kDecWarps * kTileBytes;
   unsigned char* ring = rings + (size_t)warp * kDecStages * stage_bytes(BITS);
@@ -165,10 +160,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const __grid_constant
   // over the banks
   for (int j = tid; j < a.K; j += kDecThreads) {
     const float2 c = __ldg(a.codebook + j);
-    const __half2 h = a.fold ? __floats2half2_rn(c.x + c.y, c.x - c.y) : __floats2half2_rn(c.x, c.y);
-    const uint32_t u = *reinterpret_cast<const uint32_t*>(&h);
+    const float2 t = a.fold ? make_float2(c.x + c.y, c.x - c.y) : c;
 #pragma unroll
-    for (int r = 0; r < (1 << RL); ++r) tab[(j << RL) + ((r + lane) & ((1 << RL) - 1))] = u;
+    for (int r = 0; r < (1 << RL); ++r) tab[(j << RL) + ((r + lane) & ((1 << RL) - 1))] = t;
   }
   if (lane == 0) {
     for (int s = 0; s < kDecStages; ++s) mbar_init(&bars[s], 1);
@@ -180,7 +174,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const __grid_constant
   pdl_trigger();
 
   const uint32_t tab_s = smem_u32(tab);
-  const uint32_t rep4 = (uint32_t)(lane & ((1 << RL) - 1)) << 2;  // this lane's replica
+  const uint32_t rep8 = (uint32_t)(lane & ((1 << RL) - 1)) << 3;  // this lane's replica
   const uint32_t ostage_s = smem_u32(ostage);
   const int64_t lo = (int64_t)blockIdx.x * a.items / gridDim.x;
   const int64_t hi = ((int64_t)blockIdx.x + 1) * a.items / gridDim.x;
@@ -284,7 +278,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const __grid_constant
         if (lane == 0 && k + kDecStages < ntiles) issue(k + kDecStages);
         const float rn = __half2float(M.rnorm[row]);
         float2 v[32];
-        gather2<BITS>(w, tab_s, rep4, sg, rn, v, std::make_integer_sequence<int, 32>{});
+        gather2<BITS>(w, tab_s, rep8, sg, rn, v, std::make_integer_sequence<int, 32>{});
         // the span-1 stage is in the table
         if constexpr (FULL) {  // block >= 64: every in-register stage, straight-line
           fwht2_stage<1>(v);

@@ -1,11 +1,7 @@
 // encode.cu -- QAM-W encoder (paper section 3.1 steps 1-6, section 3.4, and the
 // activation-aware per-channel scaling).
 //
-// Kernels, in stream order:
-//   k_scales        s_j = binary16((a_j / mean a)^alpha)          (thread/channel)
-//   k_calib_rows    |z_k| sums of the first 1024 rows, per CTA       (128 CTAs)
-//   k_calib_ext     later rows when those held zero rows             (1 CTA)
-//   k_calib_finish  sigma_k = binary16(sum / (n sqrt(pi/2)))        (16 threads/pair)
+// The channel scales and eq. (1) come first (calibrate.cu); then
 //   k_encode        norm, rotate, normalise, nearest codeword, pack  (row groups)
 #include <algorithm>
 #include <cmath>
@@ -15,306 +11,6 @@
 
 namespace qamw {
 namespace {
-
-// ------------------------------------------------------------------ scales
-
-// One CTA of 1024 threads: thread t holds the statistic of channels t + 1024 i
-// (i < 32, d_in <= 32768) in registers, so the statistic is read once; the
-// fp64 sum is reduced in a fixed order (per-thread ascending i, a shuffle tree
-// per warp, then the 32 warp sums by the same tree), so the mean is bitwise
-// reproducible; each thread then rounds its own channels' scales.
-constexpr int kScaleThreads = 1024;
-__global__ void __launch_bounds__(kScaleThreads) k_scales(const float* __restrict__ a, int d_in,
-                                                          float alpha, __half* __restrict__ s,
-                                                          int32_t* status) {
-  __shared__ double red[32];
-  __shared__ double mean_s;
-  constexpr int kPer = kMaxDin / kScaleThreads;
-  float vals[kPer];
-  double sum = 0.0;
-  int bad = 0;
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int j = threadIdx.x + i * kScaleThreads;
-    vals[i] = j < d_in ? a[j] : 1.f;
-    if (j < d_in) {
-      if (vals[i] > 0.f && isfinite(vals[i]))
-        sum += (double)vals[i];
-      else
-        bad = 1;
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sum;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    double t = red[threadIdx.x];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-    if (threadIdx.x == 0) mean_s = t / (double)d_in;
-  }
-  bad = __syncthreads_or(bad);
-  const double mean = mean_s;
-  pdl_wait();  // s may still be read by the kernel ahead
-  pdl_trigger();
-  int range = 0;
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int j = threadIdx.x + i * kScaleThreads;
-    if (j >= d_in) break;
-    const float v = vals[i];
-    __half h;
-    if (v > 0.f && isfinite(v)) {
-      // binary16(pow(v / mean, alpha)) of the fp64 power: an fp32 evaluation
-      // decides unless it lies within its error bound (log2f 1 ulp, exp2f 2
-      // ulp, the ratio 2^-24: under (2 + |t| + |alpha|) 2^-23 relative for
-      // t = alpha log2 r; a 2x margin taken) of a binary16 rounding midpoint -- the
-      // midpoints between h and its neighbours are exact in fp32 -- or
-      // outside the normal/subnormal range; there the fp64 pow decides
-      const float t = alpha * log2f((float)((double)v / mean));
-      const float y = exp2f(t);
-      h = __float2half_rn(y);
-      const uint16_t hb = __half_as_ushort(h);
-      bool exact = y > 0.f && hb > 0u && hb < 0x7bffu;
-      if (exact) {
-        const float hf = __half2float(h);
-        const float up = __half2float(__ushort_as_half((uint16_t)(hb + 1)));
-        const float dn = __half2float(__ushort_as_half((uint16_t)(hb - 1)));
-        const float tol = y * (2.0f + fabsf(t) + fabsf(alpha)) * 2.4e-7f;
-        exact = fabsf(y - 0.5f * (hf + up)) > tol && fabsf(y - 0.5f * (hf + dn)) > tol;
-      }
-      if (!exact) h = __double2half(pow((double)v / mean, (double)alpha));
-      const float hf2 = __half2float(h);
-      if (isinf(hf2) || hf2 == 0.f) range = 1;
-    } else {
-      h = __float2half(1.0f);
-    }
-    s[j] = h;
-  }
-  raise_flag(status, ((threadIdx.x == 0 && bad) ? QAMW_STATUS_BAD_STAT : 0) |
-                         (range ? QAMW_STATUS_RANGE : 0));
-}
-
-__global__ void k_fill_half(__half* p, int n, float v) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) p[i] = __float2half(v);
-}
-
-// ------------------------------------------------------------- calibration
-
-// Eq. (1) over the first min(1024, #non-zero) non-zero rows, in three launches:
-//   k_calib_rows   CTA b takes rows [8b, 8b + 8) of the first 1024: row norm
-//                  (fixed-order reduction), rotation, |z_k| / r summed over
-//                  its non-zero rows into partial[b][k]; nonzero[b] = count.
-//   k_calib_ext    if the first 1024 rows held zero rows, one CTA walks on
-//                  from row 1024 in order, adding the next non-zero rows into
-//                  ext[k] until there are 1024 (a path only matrices with zero
-//                  rows take); else it only records the count.
-//   k_calib_finish sigma_k = binary16((sum_b partial[b][k] + ext[k]) /
-//                  (n sqrt(pi/2))), 1 when that rounds to 0.
-// Thread (g, c) holds chunk c of row group g; RPC row groups run at once.
-template <typename T, int MAXT>
-__global__ void __launch_bounds__(MAXT) k_calib_rows(const T* __restrict__ W,
-                                                     const __half* __restrict__ s, int d_out,
-                                                     int d_in, int block, uint64_t seed, int RPC,
-                                                     float* __restrict__ partial,
-                                                     int32_t* __restrict__ nonzero,
-                                                     int32_t* status) {
-  extern __shared__ __align__(16) float sm[];
-  pdl_wait();
-  pdl_trigger();
-  const int C = d_in / kE, P = d_in / 2;
-  float* fT = sm;                     // [j][c]: D * s of column 64c + j
-  float* red = sm + d_in;             // [g][q][c]
-  float* part = red + (size_t)RPC * P;  // [blockDim] partial sums of squares
-  float* rsum = part + blockDim.x;     // [RPC]
-  fill_interleaved<kE>(fT, s, d_in, C, [=](int j, float v) {
-    return mask_negative(seed, (uint32_t)j) ? -v : v;
-  });
-  __syncthreads();
-  const int g = threadIdx.x / C, c = threadIdx.x - g * C;
-  const bool lane_ok = g < RPC;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int nb = min(block, kE), lanes = max(block / kE, 1);
-  const float inv_sqrt_b = 1.0f / sqrtf((float)block);
-  const int rows = min(d_out, kCalRows);
-  const int per = kCalRows / gridDim.x;
-  const int t0 = blockIdx.x * per, t1 = min(t0 + per, rows);
-  float acc[kQ];
-#pragma unroll
-  for (int q = 0; q < kQ; ++q) acc[q] = 0.f;
-  int nz = 0, flags = 0;
-  for (int base = t0; base < t1; base += RPC) {
-    const int row = base + g;
-    const bool active = lane_ok && row < t1;
-    float x[kE];
-    float ss = 0.f;
-    if (active) {
-      load64(W + (int64_t)row * d_in + (int64_t)c * kE, x);
-#pragma unroll
-      for (int j = 0; j < kE; ++j) {
-        x[j] *= fT[j * C + c];
-        ss = fmaf(x[j], x[j], ss);
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < kE; ++j) x[j] = 0.f;
-    }
-    part[threadIdx.x] = ss;
-    fwht_reg<kE>(x, nb);
-    fwht_lanes<kE>(x, lanes);
-    __syncthreads();
-    for (int q = warp; q < RPC; q += nwarps) {
-      float t = 0.f;
-      for (int k = lane; k < C; k += 32) t += part[q * C + k];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-      if (lane == 0) rsum[q] = sqrtf(t);
-    }
-    __syncthreads();
-    if (active) {
-      const float r = rsum[g];
-      if (!isfinite(r)) flags = QAMW_STATUS_NONFINITE;
-      if (r > 0.f) {
-        if (c == 0) ++nz;
-        const float inv = inv_sqrt_b / r;
-#pragma unroll
-        for (int q = 0; q < kQ; ++q) {
-          const float zx = x[2 * q] * inv, zy = x[2 * q + 1] * inv;
-          acc[q] += sqrtf(fmaf(zx, zx, zy * zy));
-        }
-      }
-    }
-    __syncthreads();  // part / rsum are rewritten by the next batch
-  }
-  if (lane_ok) {
-#pragma unroll
-    for (int q = 0; q < kQ; ++q) red[(size_t)g * P + q * C + c] = acc[q];
-  }
-  // non-zero rows of this CTA: thread (g, 0) counted those of group g
-  __shared__ int cnt_sh;
-  if (threadIdx.x == 0) cnt_sh = 0;
-  __syncthreads();
-  if (nz) atomicAdd(&cnt_sh, nz);
-  for (int k = threadIdx.x; k < P; k += blockDim.x) {
-    float v = 0.f;
-    for (int gg = 0; gg < RPC; ++gg) v += red[(size_t)gg * P + (k % kQ) * C + k / kQ];
-    partial[(size_t)blockIdx.x * P + k] = v;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) nonzero[blockIdx.x] = cnt_sh;
-  raise_flag(status, flags);
-}
-
-// One CTA of at least C threads; thread c < C holds chunk c of the current row.
-template <typename T>
-__global__ void __launch_bounds__(512) k_calib_ext(const T* __restrict__ W,
-                                                   const __half* __restrict__ s, int d_out,
-                                                   int d_in, int block, uint64_t seed,
-                                                   const int32_t* __restrict__ nonzero, int nparts,
-                                                   float* __restrict__ ext,
-                                                   int32_t* __restrict__ n_cal) {
-  extern __shared__ __align__(16) float fT[];  // [j][c]
-  __shared__ float part[512];
-  __shared__ float rtot;
-  __shared__ int total;
-  pdl_wait();
-  pdl_trigger();
-  const int C = d_in / kE;
-  const int c = threadIdx.x;
-  const bool active_c = c < C;
-  if (threadIdx.x < 32) {  // the non-zero rows found among the first 1024 (integer sum)
-    int n = 0;
-    for (int b = threadIdx.x; b < nparts; b += 32) n += nonzero[b];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
-    if (threadIdx.x == 0) total = n;
-  }
-  float acc[kQ];
-#pragma unroll
-  for (int q = 0; q < kQ; ++q) acc[q] = 0.f;
-  __syncthreads();
-  if (total < kCalRows && d_out > kCalRows) {
-    fill_interleaved<kE>(fT, s, d_in, C, [=](int j, float v) {
-      return mask_negative(seed, (uint32_t)j) ? -v : v;
-    });
-    __syncthreads();
-    const int nb = min(block, kE), lanes = max(block / kE, 1);
-    const float inv_sqrt_b = 1.0f / sqrtf((float)block);
-    for (int row = kCalRows; row < d_out && total < kCalRows; ++row) {
-      float x[kE];
-      float ss = 0.f;
-      if (active_c) {
-        load64(W + (int64_t)row * d_in + (int64_t)c * kE, x);
-#pragma unroll
-        for (int j = 0; j < kE; ++j) {
-          x[j] *= fT[j * C + c];
-          ss = fmaf(x[j], x[j], ss);
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < kE; ++j) x[j] = 0.f;
-      }
-      part[threadIdx.x] = ss;
-      fwht_reg<kE>(x, nb);
-      fwht_lanes<kE>(x, lanes);
-      __syncthreads();
-      if (threadIdx.x < 32) {
-        float t = 0.f;
-        for (int k = threadIdx.x; k < C; k += 32) t += part[k];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-        if (threadIdx.x == 0) rtot = sqrtf(t);
-      }
-      __syncthreads();
-      const float r = rtot;
-      if (r > 0.f && active_c) {
-        const float inv = inv_sqrt_b / r;
-#pragma unroll
-        for (int q = 0; q < kQ; ++q) {
-          const float zx = x[2 * q] * inv, zy = x[2 * q + 1] * inv;
-          acc[q] += sqrtf(fmaf(zx, zx, zy * zy));
-        }
-      }
-      __syncthreads();
-      if (threadIdx.x == 0 && r > 0.f) ++total;
-      __syncthreads();
-    }
-  }
-  if (active_c) {
-#pragma unroll
-    for (int q = 0; q < kQ; ++q) ext[c * kQ + q] = acc[q];
-  }
-  if (threadIdx.x == 0) *n_cal = min(total, kCalRows);
-}
-
-// 16 threads per pair k: thread i sums partials i, i+16, ... in fp64, then the
-// 16 sums are combined by a fixed shuffle tree (deterministic).
-__global__ void __launch_bounds__(256) k_calib_finish(const float* __restrict__ partial,
-                                                      int nparts, const float* __restrict__ ext,
-                                                      const int32_t* __restrict__ n_cal_p, int P,
-                                                      __half* __restrict__ sigma,
-                                                      int32_t* status) {
-  pdl_wait();
-  pdl_trigger();
-  const int g = blockIdx.x * (blockDim.x / 16) + threadIdx.x / 16, i = threadIdx.x & 15;
-  const int k = min(g, P - 1);
-  double sum = 0.0;
-#pragma unroll 8
-  for (int p = i; p < nparts; p += 16) sum += (double)partial[(size_t)p * P + k];
-#pragma unroll
-  for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (i != 0 || g >= P) return;
-  sum += (double)ext[k];
-  const int n = *n_cal_p;
-  const double rayleigh = 1.2533141373155002512;  // sqrt(pi/2)
-  __half h = __double2half(n > 0 ? sum / (double)n / rayleigh : 0.0);
-  const float hf = __half2float(h);
-  if (hf == 0.f) h = __float2half(1.0f);
-  if (isinf(hf)) raise_flag(status, QAMW_STATUS_RANGE);
-  sigma[k] = h;
-}
 
 // ---------------------------------------------------------------- encoder
 
@@ -925,51 +621,6 @@ cudaError_t encode_rows_typed(const T* W, const qamw_matrix& m, int32_t* st,
   }
 }
 
-template <typename T>
-cudaError_t calibrate_typed(const T* W, const qamw_matrix& m, const EncodeWorkspace& ws,
-                            int32_t* st, cudaStream_t stream) {
-  const int d_out = m.d_out, d_in = m.d_in, P = d_in / 2;
-  const int C = d_in / kE;
-  const __half* s = reinterpret_cast<const __half*>(m.chan_scale);
-  cudaError_t err;
-  // rows per batch: at most the 8 rows a CTA owns; 256 threads (512 when one
-  // row has more than 256 chunks); ~200 KB of shared memory
-  const int maxt = C > 256 ? 512 : 256;
-  auto smem_for = [&](int rpc) {
-    const size_t threads = ((size_t)rpc * C + 31) / 32 * 32;
-    return (size_t)d_in * sizeof(float) + (size_t)rpc * P * sizeof(float) +
-           threads * sizeof(float) + (size_t)rpc * sizeof(float);
-  };
-  int RPC = kCalRows / kCalCtas;
-  if (RPC * C > maxt) RPC = maxt / C;
-  if (RPC < 1) RPC = 1;
-  while (RPC > 1 && smem_for(RPC) > 200 * 1024) --RPC;
-  const int threads = ((RPC * C + 31) / 32) * 32;
-  const size_t smem = smem_for(RPC);
-  const void* fn = maxt == 256 ? reinterpret_cast<const void*>(&k_calib_rows<T, 256>)
-                               : reinterpret_cast<const void*>(&k_calib_rows<T, 512>);
-  if ((err = allow_smem(fn, smem)) != cudaSuccess) return err;
-  if (maxt == 256)
-    err = launch_pdl(k_calib_rows<T, 256>, dim3(kCalCtas), dim3(threads), smem, stream, W, s,
-                     d_out, d_in, m.block, m.mask_seed, RPC, ws.cal_partial, ws.cal_nonzero, st);
-  else
-    err = launch_pdl(k_calib_rows<T, 512>, dim3(kCalCtas), dim3(threads), smem, stream, W, s,
-                     d_out, d_in, m.block, m.mask_seed, RPC, ws.cal_partial, ws.cal_nonzero, st);
-  if (err != cudaSuccess) return err;
-  {
-    const int et = ((C + 31) / 32) * 32;
-    const size_t esmem = (size_t)d_in * sizeof(float);
-    const void* efn = reinterpret_cast<const void*>(&k_calib_ext<T>);
-    if ((err = allow_smem(efn, esmem)) != cudaSuccess) return err;
-    err = launch_pdl(k_calib_ext<T>, dim3(1), dim3(et), esmem, stream, W, s, d_out, d_in, m.block,
-                     m.mask_seed, ws.cal_nonzero, kCalCtas, ws.cal_ext, ws.n_cal);
-    if (err != cudaSuccess) return err;
-  }
-  return launch_pdl(k_calib_finish, dim3((P + 15) / 16), dim3(256), 0, stream,
-                    (const float*)ws.cal_partial, kCalCtas, (const float*)ws.cal_ext,
-                    (const int32_t*)ws.n_cal, P, reinterpret_cast<__half*>(m.sigma), st);
-}
-
 // Section 3.5: Lloyd-Max levels of the unit Rayleigh density on one warp (lane
 // i owns level i, Na <= 32), fp64, from the equal-probability thresholds, then
 // the expanded table c[ia Np + ip] = a_ia (cos 2 pi ip / Np, sin 2 pi ip / Np).
@@ -1010,52 +661,10 @@ cudaError_t launch_polar_codebook(int bits, float* d_codebook, cudaStream_t stre
 
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-size_t calibrate_workspace_bytes(int d_out, int d_in, EncodeWorkspace* carve, void* base) {
-  (void)d_out;
-  const size_t P = (size_t)d_in / 2;
-  size_t off = 0;
-  const size_t o_nz = off;
-  off += align256(kCalCtas * sizeof(int32_t));
-  const size_t o_n = off;
-  off += align256(sizeof(int32_t));
-  const size_t o_ext = off;
-  off += align256(P * sizeof(float));
-  const size_t o_part = off;
-  off += align256((size_t)kCalCtas * P * sizeof(float));
-  if (carve) {
-    char* b = static_cast<char*>(base);
-    carve->cal_nonzero = reinterpret_cast<int32_t*>(b + o_nz);
-    carve->n_cal = reinterpret_cast<int32_t*>(b + o_n);
-    carve->cal_ext = reinterpret_cast<float*>(b + o_ext);
-    carve->cal_partial = reinterpret_cast<float*>(b + o_part);
-    carve->prefilter = nullptr;
-  }
-  return off;
-}
-
 size_t encode_workspace_bytes(int d_out, int d_in, int bits, EncodeWorkspace* carve, void* base) {
   const size_t off = calibrate_workspace_bytes(d_out, d_in, carve, base);
   if (carve) carve->prefilter = static_cast<char*>(base) + off;
   return off + align256(prefilter_bytes_for(prefilter_grid(bits)));
-}
-
-cudaError_t launch_channel_scales(const float* d_act_stat, int d_in, float alpha, uint16_t* d_scale,
-                                  int32_t* d_status, cudaStream_t stream) {
-  __half* s = reinterpret_cast<__half*>(d_scale);
-  if (d_act_stat != nullptr && alpha != 0.0f)
-    return launch_pdl(k_scales, dim3(1), dim3(kScaleThreads), 0, stream, d_act_stat, d_in, alpha, s,
-                      d_status);
-  else
-    k_fill_half<<<(d_in + 255) / 256, 256, 0, stream>>>(s, d_in, 1.0f);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_calibrate(const void* d_W, int dtype, const qamw_matrix& m,
-                             const EncodeWorkspace& ws, int32_t* d_status, cudaStream_t stream) {
-  if (dtype == QAMW_DTYPE_F32)
-    return calibrate_typed<float>(static_cast<const float*>(d_W), m, ws, d_status, stream);
-  return calibrate_typed<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(d_W), m, ws, d_status,
-                                        stream);
 }
 
 template <typename T>

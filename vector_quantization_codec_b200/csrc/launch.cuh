@@ -59,14 +59,16 @@ inline cudaError_t launch_pdl_ptr(const void* kernel, dim3 grid, dim3 block, siz
 // Workspace carve-up of qamw_encode.
 struct EncodeWorkspace {
   int32_t* cal_nonzero;  // [kCalCtas] non-zero rows each CTA found among rows 0..1023
+                         // (the first byte of the calibration workspace)
   int32_t* n_cal;        // [1] rows used by eq. (1)
   float* cal_ext;        // [P] |z_k| sums of rows past 1023 (zero rows present)
   float* cal_partial;    // [kCalCtas][P] partial sums of |z_k|
   void* prefilter;       // prefilter table (when the matrix carries none)
 };
 constexpr int kCalRows = 1024;
-constexpr int kCalCtas = 128;
+constexpr int kCalCtas = 32;  // CTAs per matrix of eq. (1): 32 rows each
 size_t calibrate_workspace_bytes(int d_out, int d_in, EncodeWorkspace* carve, void* base);
+size_t calibrate_many_workspace_bytes(const qamw_matrix* ms, int n);
 size_t encode_workspace_bytes(int d_out, int d_in, int bits, EncodeWorkspace* carve, void* base);
 
 size_t train_workspace_bytes(int bits);
@@ -80,6 +82,10 @@ cudaError_t launch_channel_scales(const float* d_act_stat, int d_in, float alpha
                                   int32_t* d_status, cudaStream_t stream);
 cudaError_t launch_calibrate(const void* d_W, int dtype, const qamw_matrix& m,
                              const EncodeWorkspace& ws, int32_t* d_status, cudaStream_t stream);
+// Channel scales and eq. (1) of n matrices (workspace: calibrate_many_workspace_bytes).
+cudaError_t launch_calibrate_many(const void* const* d_W, int dtype, const float* const* d_act,
+                                  float alpha, const qamw_matrix* ms, int n, void* d_ws,
+                                  int32_t* d_status, cudaStream_t stream);
 // Normalised points of rows [row0, row0 + nrows) as float2 [nrows][d_in / 2].
 cudaError_t launch_points(const void* d_W, int dtype, const qamw_matrix& m, int64_t row0,
                           int64_t nrows, float* d_points, int32_t* d_status, cudaStream_t stream);

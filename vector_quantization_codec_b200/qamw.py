@@ -44,7 +44,8 @@ QAMW_OP_CALIBRATE = 3
 EXPORTS = ("qamw_row_bytes", "qamw_default_block", "qamw_bits_per_weight",
            "qamw_workspace_bytes", "qamw_prefilter_bytes", "qamw_status_string",
            "qamw_train_codebook", "qamw_build_prefilter", "qamw_encode", "qamw_channel_scales",
-           "qamw_calibrate_sigma", "qamw_encode_rows", "qamw_decode", "qamw_decode_many",
+           "qamw_calibrate_sigma", "qamw_calibrate_many", "qamw_calibrate_many_workspace_bytes",
+           "qamw_encode_rows", "qamw_decode", "qamw_decode_many",
            "qamw_decode_gemv",
            "qamw_decode_gemv_noalloc", "qamw_polar_codebook", "qamw_encode_rows_polar",
            "qamw_normalised_pairs", "qamw_selftest_wait_timeout")
@@ -81,6 +82,9 @@ def _load() -> C.CDLL:
         "qamw_encode": (I, [V, I, V, C.c_float, I, C.POINTER(qamw_matrix), V, SZ, V, V]),
         "qamw_channel_scales": (I, [V, I, C.c_float, V, V, V]),
         "qamw_calibrate_sigma": (I, [V, I, C.POINTER(qamw_matrix), V, SZ, V, V]),
+        "qamw_calibrate_many": (I, [C.POINTER(C.c_void_p), I, C.POINTER(C.c_void_p), C.c_float,
+                                    C.POINTER(qamw_matrix), I, V, SZ, V, V]),
+        "qamw_calibrate_many_workspace_bytes": (SZ, [C.POINTER(qamw_matrix), I]),
         "qamw_encode_rows": (I, [V, I, C.POINTER(qamw_matrix), V, V, V]),
         "qamw_decode": (I, [C.POINTER(qamw_matrix), V, V, V]),
         "qamw_decode_many": (I, [C.POINTER(qamw_matrix), I, C.POINTER(C.c_void_p), V, V]),
@@ -261,6 +265,36 @@ def qamw_calibrate_sigma(W: torch.Tensor, m: EncodedMatrix, workspace: torch.Ten
     return m
 
 
+def _matrix_array(ms: list):
+    return (qamw_matrix * max(len(ms), 1))(*[m.struct() for m in ms])
+
+
+def qamw_calibrate_many_workspace_bytes(ms: list) -> int:
+    return int(_lib.qamw_calibrate_many_workspace_bytes(_matrix_array(ms), len(ms)))
+
+
+def qamw_calibrate_many(Ws: list, ms: list, act_stats: list | None = None, alpha: float = 0.0,
+                        workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                        stream=None) -> list:
+    """Channel scales and eq. (1) of every matrix of `ms` (weights `Ws`) in one call."""
+    n = len(ms)
+    if len(Ws) != n or (act_stats is not None and len(act_stats) != n):
+        raise ValueError("one weight tensor (and statistic) per matrix")
+    dtypes = {_dtype_code(W) for W in Ws}
+    if len(dtypes) != 1:
+        raise TypeError("all weights must have the same dtype")
+    arr = _matrix_array(ms)
+    if workspace is None:
+        workspace = _workspace(int(_lib.qamw_calibrate_many_workspace_bytes(arr, n)), Ws[0].device)
+    wp = (C.c_void_p * max(n, 1))(*[W.data_ptr() for W in Ws])
+    ap = None if act_stats is None else (C.c_void_p * max(n, 1))(
+        *[None if a is None else a.data_ptr() for a in act_stats])
+    rc = _lib.qamw_calibrate_many(wp, dtypes.pop(), ap, float(alpha), arr, n, _p(workspace),
+                                  workspace.numel(), _p(status), _s(stream))
+    _check("qamw_calibrate_many", rc)
+    return ms
+
+
 def qamw_encode_rows(W: torch.Tensor, m: EncodedMatrix, status: torch.Tensor | None = None,
                      stream=None, candidates: torch.Tensor | None = None) -> EncodedMatrix:
     """Steps 1-6 of section 3.1 with the side values already in m.  `candidates`
@@ -333,7 +367,7 @@ def qamw_decode_many(ms: list, outs: list | None = None, status: torch.Tensor | 
         outs = [torch.empty((m.d_out, m.d_in), dtype=torch.bfloat16, device=m.packed.device)
                 for m in ms]
     n = len(ms)
-    arr = (qamw_matrix * max(n, 1))(*[m.struct() for m in ms])
+    arr = _matrix_array(ms)
     ptrs = (C.c_void_p * max(n, 1))(*[o.data_ptr() for o in outs])
     rc = _lib.qamw_decode_many(arr, n, ptrs, _p(status), _s(stream))
     _check("qamw_decode_many", rc)
