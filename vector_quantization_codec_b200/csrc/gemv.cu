@@ -13,12 +13,11 @@
 //   come from an fp16x2 copy of the codebook replicated so that a warp's 32
 //   random lookups hit at most 2 lanes per bank.  Per-slice partial dot
 //   products are summed in a fixed order (bitwise reproducible).
-// batch 2..16 (k_rotate + k_gemv_s): xbar for all columns is written once to
-//   the workspace (chunk-interleaved so that lanes read consecutive words).
-//   Each CTA stages 4 or 8 of its columns in shared memory beside a replicated
-//   fp16x2 codebook, and a warp sums two rows at a time (batch 9..16: two
-//   column passes).  Where that does not fit (long rows), k_gemv reads xbar
-//   from the workspace with one warp per row.
+// batch 2..16 (k_rotate_mma + k_gemv_mma): x_bar for 8 or 16 columns is
+//   written once to the workspace in the operand order of the tensor cores;
+//   16-row tiles are products of gathered codewords with x_bar on m16n8k16
+//   MMAs (binary16 high/low parts, fp32 accumulation), the packed indices
+//   streaming into shared memory through per-warp bulk-copy rings.
 #include <utility>
 
 #include "common.cuh"
@@ -319,24 +318,68 @@ cudaError_t run_gemv1(const qamw_matrix& m, const uint16_t* d_x, uint16_t* d_y,
 
 // ------------------------------------------------------------- batch 2..16
 
-// xbarT[t][q][c] (float2) = pair 32c+q of xbar_t, for t < batch; zeros for
-// batch <= t < bpad.  A CTA takes 32 consecutive (t, chunk c) items: all its
-// threads form D x / s element by element into shared memory, then one warp
-// rotates the 32 chunks from there (lane = item), so that the per-element
-// divisions and sign hashes are spread over the whole CTA.
 constexpr int kRotItems = 32;
 constexpr int kRotThreads = 256;
 
-__global__ void __launch_bounds__(kRotThreads) k_rotate(const __nv_bfloat16* __restrict__ x,
-                                                        int batch, int bpad, int d_in, int block,
-                                                        uint64_t seed,
-                                                        const __half* __restrict__ s,
-                                                        const __half* __restrict__ sigma,
-                                                        float2* __restrict__ xbarT,
-                                                        int32_t* status) {
+// ------------------------------------------------------ tensor-core path
+//
+// y^T = C_hat x_bar^T on the tensor cores with m16n8k16 MMAs and fp32
+// accumulation: A = 16 rows x 16 k of gathered codewords (one k pair = one
+// codeword (x, y)), B = 16 k x 8 batch columns of x_bar, C = 16 rows x 8
+// columns.  Both operands are split into binary16 high and low parts (v = hi +
+// lo, lo = binary16(v - hi)) and C accumulates A_hi B_hi + A_lo B_hi + A_hi B_lo:
+// about 22 significant bits, where a single binary16 operand would spend most of
+// the 1e-2 tolerance on rows whose output is small.
+// The order of the k dimension makes each lane's A operands one whole
+// 64-column chunk of a row: in K-chunk j (128 pairs, 16 k-steps), k-step kk,
+// lane (g = lane / 4, t = lane % 4) holds pairs p0 = 128 j + 32 t + 2 kk (k
+// slots 2t, 2t+1) and p0 + 1 (slots 2t+8, 2t+9) of rows g and g + 8 -- its
+// indices are the `bits` words of chunk 4 j + t, extracted with fixed shifts.
+// B uses the same order: the rotation kernel writes x_bar in it.
+constexpr int kMmaWarps = 8;
+constexpr int kMmaThreads = 32 * kMmaWarps;
+constexpr int kMmaRows = 16;       // rows per CTA tile
+constexpr int kMmaPairs = 128;     // pairs per K-chunk
+constexpr int kMmaStages = 2;
+
+__host__ __device__ inline int mma_chunks(int P) { return (P + kMmaPairs - 1) / kMmaPairs; }
+
+// Bytes of x_bar in the tensor-core layout: [chunk][n-tile][kk][lane] uint4
+// {hi(x_bar_n[p]), hi(x_bar_n[p + 1]), lo(x_bar_n[p]), lo(x_bar_n[p + 1])}
+// (binary16 pairs), n = 8 nt + g, p = 128 j + 32 t + 2 kk; zero for n >= batch
+// and p >= P.
+__host__ __device__ inline size_t mma_xbar_bytes(int P, int NT) {
+  return (size_t)mma_chunks(P) * NT * 16 * 32 * sizeof(uint4);
+}
+
+// Codeword replicas (log2) of the hi/lo table (8 bytes an entry): 8 for K =
+// 2048, 16 below (at most 128 KB).
+constexpr int mma_rep_log2(int bits) { return bits >= 11 ? 3 : 4; }
+
+// binary16 high and low parts of a pair of floats, as two half2 words.
+__device__ __forceinline__ uint2 split_half2(float a, float b) {
+  const __half2 hi = __floats2half2_rn(a, b);
+  const float2 hf = __half22float2(hi);
+  const __half2 lo = __floats2half2_rn(a - hf.x, b - hf.y);
+  return make_uint2(*reinterpret_cast<const uint32_t*>(&hi), *reinterpret_cast<const uint32_t*>(&lo));
+}
+
+// x_bar = sigma (.) R_fwd(x / s) for n < 8 NT columns and every 64-column
+// chunk (padded to whole K-chunks), written in the tensor-core layout.  A CTA
+// takes 32 (column, chunk) items: all threads form D x / s element by element
+// into shared memory, then one warp rotates the 32 chunks (lane = item).
+__global__ void __launch_bounds__(kRotThreads) k_rotate_mma(const __nv_bfloat16* __restrict__ x,
+                                                            int batch, int NT, int d_in, int block,
+                                                            uint64_t seed,
+                                                            const __half* __restrict__ s,
+                                                            const __half* __restrict__ sigma,
+                                                            uint4* __restrict__ xb,
+                                                            int32_t* status) {
   __shared__ float buf[kRotItems][kE + 1];  // +1: conflict-free rows and columns
-  const int C = d_in / kE, P = d_in / 2;
-  const int64_t V = (int64_t)bpad * C;
+  const int C = d_in / kE;
+  const int Cpad = mma_chunks(d_in / 2) * 4;
+  const int ncol = 8 * NT;
+  const int64_t V = (int64_t)ncol * Cpad;
   const int nb = min(block, kE), lanes = max(block / kE, 1);
   const float inv_sqrt_b = 1.0f / sqrtf((float)block);
   int flags = 0;
@@ -345,17 +388,23 @@ __global__ void __launch_bounds__(kRotThreads) k_rotate(const __nv_bfloat16* __r
   pdl_trigger();
   for (int64_t base = (int64_t)blockIdx.x * kRotItems; base < V;
        base += (int64_t)gridDim.x * kRotItems) {
+    // item v = n Cpad + c: the b / 64 chunks of a Hadamard block are
+    // consecutive items, inside one CTA's 32 (Cpad and 32 are multiples of
+    // b / 64), and padding chunks c >= C form whole blocks of zeros
     for (int e = threadIdx.x; e < kRotItems * kE; e += kRotThreads) {
       const int i = e / kE, j = e - i * kE;
       const int64_t v = base + i;
-      const int64_t t = v < V ? v / C : bpad;
+      const int64_t n = v < V ? v / Cpad : ncol;
       float val = 0.f;
-      if (t < batch) {
-        const int col = (int)(v - t * C) * kE + j;
-        const float xv = __bfloat162float(x[t * d_in + col]);
-        if (!isfinite(xv)) flags = QAMW_STATUS_NONFINITE;
-        const float q = __fdiv_rn(xv, __half2float(s[col]));
-        val = mask_negative(seed, (uint32_t)col) ? -q : q;
+      if (n < batch) {
+        const int c = (int)(v - n * Cpad);
+        if (c < C) {
+          const int col = c * kE + j;
+          const float xv = __bfloat162float(x[n * d_in + col]);
+          if (!isfinite(xv)) flags |= QAMW_STATUS_NONFINITE;
+          const float q = __fdiv_rn(xv, __half2float(s[col]));
+          val = mask_negative(seed, (uint32_t)col) ? -q : q;
+        }
       }
       buf[i][j] = val;
     }
@@ -363,8 +412,8 @@ __global__ void __launch_bounds__(kRotThreads) k_rotate(const __nv_bfloat16* __r
     if (threadIdx.x < 32) {  // one whole warp: the lane shuffles need all 32
       const int64_t v = base + threadIdx.x;
       const bool active = v < V;
-      const int64_t t = active ? v / C : 0;
-      const int c = active ? (int)(v - t * C) : 0;
+      const int64_t n = active ? v / Cpad : 0;
+      const int c = active ? (int)(v - n * Cpad) : 0;
       float xv[kE];
 #pragma unroll
       for (int j = 0; j < kE; ++j) xv[j] = buf[threadIdx.x][j];
@@ -372,12 +421,23 @@ __global__ void __launch_bounds__(kRotThreads) k_rotate(const __nv_bfloat16* __r
       fwht_lanes<kE>(xv, lanes);
       if (active) {
         float sg[kQ];
-        load_halves<kQ>(sigma + (int64_t)c * kQ, sg);
-        float2* dst = xbarT + t * P + c;
+        if (c < C && n < batch) {
+          load_halves<kQ>(sigma + (int64_t)c * kQ, sg);
+        } else {
 #pragma unroll
-        for (int q = 0; q < kQ; ++q) {
-          const float f = sg[q] * inv_sqrt_b;
-          dst[(size_t)q * C] = make_float2(xv[2 * q] * f, xv[2 * q + 1] * f);
+          for (int q = 0; q < kQ; ++q) sg[q] = 0.f;
+        }
+        const int jc = c >> 2, tt = c & 3, nt = (int)(n >> 3), g = (int)(n & 7);
+        uint4* dst = xb + ((size_t)(jc * NT + nt) * 16) * 32 + 4 * g + tt;
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+          const float f0 = sg[2 * kk] * inv_sqrt_b, f1 = sg[2 * kk + 1] * inv_sqrt_b;
+          const float a = xv[4 * kk] * f0, b = xv[4 * kk + 1] * f0;
+          const float cc = xv[4 * kk + 2] * f1, d = xv[4 * kk + 3] * f1;
+          if (fmaxf(fmaxf(fabsf(a), fabsf(b)), fmaxf(fabsf(cc), fabsf(d))) > 65504.f)
+            flags |= QAMW_STATUS_RANGE;
+          const uint2 p0 = split_half2(a, b), p1 = split_half2(cc, d);
+          dst[kk * 32] = make_uint4(p0.x, p1.x, p0.y, p1.y);
         }
       }
     }
@@ -386,249 +446,239 @@ __global__ void __launch_bounds__(kRotThreads) k_rotate(const __nv_bfloat16* __r
   raise_flag(status, flags);
 }
 
-// One warp per output row; lanes take the row's 32-pair chunks round robin.
-template <int BITS, int B>
-__global__ void __launch_bounds__(256) k_gemv(const uint8_t* __restrict__ packed, int64_t row_bytes,
-                                              const __half* __restrict__ rnorm,
-                                              const float2* __restrict__ codebook, int K,
-                                              const float2* __restrict__ xbarT, int d_out, int d_in,
-                                              int batch, __nv_bfloat16* __restrict__ y) {
+__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint2 lds_u2(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
+struct GemvMmaArgs {
+  const uint8_t* packed;
+  const __half* rnorm;
+  const float2* codebook;
+  const uint4* xb;
+  __nv_bfloat16* y;
+  int32_t* status;
+  int64_t row_bytes;
+  int d_out, P, batch, K;
+};
+
+// Shared memory: table uint2 [K][replicas] | per warp ring [2][16 rows][16 bits
+// bytes] | red float [8 warps][16 rows][8 NT] | bars [8][2].
+size_t gemv_mma_smem(int K, int bits, int NT) {
+  return ((size_t)K << (mma_rep_log2(bits) + 3)) +
+         (size_t)kMmaWarps * kMmaStages * kMmaRows * 16 * bits +
+         (size_t)kMmaWarps * kMmaRows * 8 * NT * sizeof(float) + kMmaWarps * kMmaStages * 8;
+}
+
+// The CTA takes 16-row tiles tile = blockIdx.x, + gridDim.x, ...; warp w takes
+// K-chunks w, w + 8, ... of each.  The warp's (tile, chunk) items stream their
+// 16 row segments (16 bits bytes each) through the warp's own 2-stage ring of
+// bulk copies, one copy per lane, prefetching across tiles.  The 8 warps'
+// partial sums of a tile are added in a fixed order.
+template <int BITS, int NT>
+__global__ void __launch_bounds__(kMmaThreads, 1) k_gemv_mma(const GemvMmaArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  float2* cb = reinterpret_cast<float2*>(smem);
-  for (int i = threadIdx.x; i < K; i += blockDim.x) cb[i] = codebook[i];
+  constexpr int RL = mma_rep_log2(BITS);
+  constexpr unsigned kSeg = 16u * BITS;  // bytes of one row segment of a chunk
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  uint2* tab = reinterpret_cast<uint2*>(smem);
+  unsigned char* ring = smem + ((size_t)a.K << (RL + 3)) + (size_t)warp * kMmaStages * kMmaRows * kSeg;
+  float* red = reinterpret_cast<float*>(smem + ((size_t)a.K << (RL + 3)) +
+                                        (size_t)kMmaWarps * kMmaStages * kMmaRows * kSeg);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red + kMmaWarps * kMmaRows * 8 * NT) + warp * kMmaStages;
+  // the codeword table needs nothing from the kernels ahead
+  for (int j = tid; j < a.K; j += kMmaThreads) {
+    const float2 c = __ldg(a.codebook + j);
+    const uint2 u = split_half2(c.x, c.y);
+#pragma unroll
+    for (int r = 0; r < (1 << RL); ++r) tab[(j << RL) + ((r + lane) & ((1 << RL) - 1))] = u;
+  }
+  if (lane == 0) {
+    for (int s = 0; s < kMmaStages; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+  }
   __syncthreads();
-  const int lane = threadIdx.x & 31;
-  const int C = d_in / kE, P = d_in / 2;
-  const int warps = (gridDim.x * blockDim.x) >> 5;
-  for (int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < d_out; row += warps) {
-    float acc[B];
-#pragma unroll
-    for (int t = 0; t < B; ++t) acc[t] = 0.f;
-    const uint32_t* src = reinterpret_cast<const uint32_t*>(packed + (int64_t)row * row_bytes);
-    for (int c = lane; c < C; c += 32) {
-      uint32_t w[BITS];
-#pragma unroll
-      for (int t = 0; t < BITS; ++t) w[t] = __ldg(src + (size_t)c * BITS + t);
-      uint32_t idx[kQ];
-      unpack32<BITS>(w, idx);
-#pragma unroll
-      for (int q = 0; q < kQ; ++q) {
-        const float2 cw = cb[idx[q]];
-#pragma unroll
-        for (int t = 0; t < B; ++t) {
-          const float2 xb = __ldg(xbarT + (int64_t)t * P + (int64_t)q * C + c);
-          acc[t] = fmaf(xb.x, cw.x, fmaf(xb.y, cw.y, acc[t]));
-        }
-      }
-    }
-#pragma unroll
-    for (int t = 0; t < B; ++t) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
-    }
-    if (lane == 0) {
-      const float rn = __half2float(rnorm[row]);
-#pragma unroll
-      for (int t = 0; t < B; ++t)
-        if (t < batch) y[(int64_t)t * d_out + row] = __float2bfloat16_rn(acc[t] * rn);
-    }
-  }
-}
-
-template <int BITS, int B>
-cudaError_t run_gemv(const qamw_matrix& m, int batch, const float2* xbar, uint16_t* d_y,
-                     cudaStream_t stream) {
-  const int threads = 256, K = 1 << m.bits;
-  const size_t smem = (size_t)K * sizeof(float2);
-  const void* fn = reinterpret_cast<const void*>(&k_gemv<BITS, B>);
-  cudaError_t err = allow_smem(fn, smem);
-  if (err != cudaSuccess) return err;
-  const int grid = persistent_grid(fn, threads, smem, ((int64_t)m.d_out * 32 + threads - 1) / threads);
-  k_gemv<BITS, B><<<grid, threads, smem, stream>>>(
-      m.packed, m.row_bytes, reinterpret_cast<const __half*>(m.row_norm),
-      reinterpret_cast<const float2*>(m.codebook), K, xbar, m.d_out, m.d_in, batch,
-      reinterpret_cast<__nv_bfloat16*>(d_y));
-  return cudaGetLastError();
-}
-
-// The same product with B batch columns of xbar (columns t0 .. t0 + B - 1 of
-// the workspace) staged in shared memory once per CTA.  A warp sums R
-// consecutive rows at once, lanes over the rows' chunks, so that each xbar
-// value read from shared memory serves R rows.  Codewords come from an fp16x2
-// table with 2^cl replicas of each entry, lane l reading replica l mod 2^cl, as
-// in the batch-1 kernel.  Used when B columns of xbar and the table fit in
-// shared memory.
-template <int BITS, int B, int R>
-__global__ void __launch_bounds__(512, 1) k_gemv_s(const uint8_t* __restrict__ packed,
-                                                   int64_t row_bytes, const __half* __restrict__ rnorm,
-                                                   const float2* __restrict__ codebook, int K,
-                                                   int cl, const float2* __restrict__ xbarT,
-                                                   int t0, int d_out, int d_in, int batch,
-                                                   __nv_bfloat16* __restrict__ y) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  uint32_t* tab = reinterpret_cast<uint32_t*>(smem);
-  float2* xs = reinterpret_cast<float2*>(smem + gemv1_table_bytes(K, cl));  // [B][P]
-  const int C = d_in / kE, P = d_in / 2;
-  const int lane = threadIdx.x & 31;
-  const int copies = 1 << cl;
-#pragma unroll 4
-  for (int j = threadIdx.x; j < K; j += blockDim.x) {
-    const float2 cw = __ldg(codebook + j);
-    const __half2 h = __floats2half2_rn(cw.x, cw.y);
-    const uint32_t u = *reinterpret_cast<const uint32_t*>(&h);
-    for (int r = 0; r < copies; ++r) tab[(j << cl) + ((r + lane) & (copies - 1))] = u;
-  }
-  const uint32_t copy = (uint32_t)lane & (uint32_t)(copies - 1);
-  // xbar, the indices and r_hat come from the kernels ahead; the table build
-  // above overlaps their end
+  // x_bar, the indices and r_hat come from the kernels ahead
   pdl_wait();
   pdl_trigger();
-  {
-    const float4* src = reinterpret_cast<const float4*>(xbarT + (int64_t)t0 * P);
-    float4* dst = reinterpret_cast<float4*>(xs);
-    const int n4 = B * P / 2;
-#pragma unroll 4
-    for (int i = threadIdx.x; i < n4; i += blockDim.x) dst[i] = __ldg(src + i);
-  }
-  __syncthreads();
-  const int warps = (gridDim.x * blockDim.x) >> 5;
-  const int nt = min(B, batch - t0);
-  for (int row = ((blockIdx.x * blockDim.x + threadIdx.x) >> 5) * R; row < d_out;
-       row += warps * R) {
-    float acc[R][B];
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-      for (int t = 0; t < B; ++t) acc[r][t] = 0.f;
-    for (int c = lane; c < C; c += 32) {
-      uint32_t idx[R][kQ];
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        // rows past the end read index 0 and are not written
-        uint32_t w[BITS];
-        const bool ok = row + r < d_out;
-        const uint32_t* src =
-            reinterpret_cast<const uint32_t*>(packed + (int64_t)(ok ? row + r : row) * row_bytes);
-#pragma unroll
-        for (int t = 0; t < BITS; ++t) w[t] = ok ? __ldg(src + (size_t)c * BITS + t) : 0u;
-        unpack32<BITS>(w, idx[r]);
-      }
-#pragma unroll
-      for (int q = 0; q < kQ; ++q) {
-        float2 cw[R];
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const uint32_t h = tab[(idx[r][q] << cl) | copy];
-          cw[r] = __half22float2(*reinterpret_cast<const __half2*>(&h));
-        }
-#pragma unroll
-        for (int t = 0; t < B; ++t) {
-          const float2 xb = xs[t * P + q * C + c];
-#pragma unroll
-          for (int r = 0; r < R; ++r)
-            acc[r][t] = fmaf(xb.x, cw[r].x, fmaf(xb.y, cw[r].y, acc[r][t]));
-        }
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-      for (int t = 0; t < B; ++t) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc[r][t] += __shfl_xor_sync(0xffffffffu, acc[r][t], o);
-      }
+  const uint32_t tab_s = smem_u32(tab);
+  const uint32_t rep8 = (uint32_t)(lane & ((1 << RL) - 1)) << 3;
+  const int nchunks = mma_chunks(a.P);
+  const int ntiles = (a.d_out + kMmaRows - 1) / kMmaRows;
+  const int my_tiles = blockIdx.x < ntiles ? (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+  const int nmy = warp < nchunks ? (nchunks - warp + kMmaWarps - 1) / kMmaWarps : 0;
+  const int nitems = my_tiles * nmy;  // this warp's (tile, chunk) items
+  const unsigned used = (unsigned)a.row_bytes;
+  unsigned issued = 0;  // lane 0: bit s = stage s had a copy; bit 8 + s = its last phase
+  int flags = 0;
+  bool abort = false;
+  auto issue = [&](int i) {  // item i: one row segment per lane
+    const int tile = blockIdx.x + (i / nmy) * gridDim.x;
+    const int j = warp + (i % nmy) * kMmaWarps;
+    const int row0 = tile * kMmaRows, nrows = min(kMmaRows, a.d_out - row0);
+    const unsigned st = (unsigned)i % kMmaStages;
+    const unsigned bytes = min(kSeg, used - (unsigned)j * kSeg);
     if (lane == 0) {
+      mbar_expect_tx(&bars[st], bytes * (unsigned)nrows);
+      issued = (issued & (1u << st)) ? (issued ^ (1u << (8 + st))) : (issued | (1u << st));
+    }
+    __syncwarp();
+    if (lane < nrows)
+      bulk_g2s(ring + (st * kMmaRows + lane) * kSeg,
+               a.packed + (int64_t)(row0 + lane) * a.row_bytes + (int64_t)j * kSeg, bytes, &bars[st]);
+  };
+  for (int i = 0; i < min(kMmaStages, nitems); ++i) issue(i);
+  int item = 0;
+  for (int ti = 0; ti < my_tiles; ++ti) {
+    const int tile = blockIdx.x + ti * gridDim.x;
+    const int row0 = tile * kMmaRows, nrows = min(kMmaRows, a.d_out - row0);
+    float acc[NT][4];
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        if (row + r >= d_out) break;
-        const float rn = __half2float(rnorm[row + r]);
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int t = 0; t < B; ++t)
-          if (t < nt) y[(int64_t)(t0 + t) * d_out + row + r] = __float2bfloat16_rn(acc[r][t] * rn);
+      for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+    for (int ci = 0; ci < nmy && !abort; ++ci, ++item) {
+      const int j = warp + ci * kMmaWarps;
+      const unsigned st = (unsigned)item % kMmaStages;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars[st], ((unsigned)item / kMmaStages) & 1u))) {
+        flags |= QAMW_STATUS_TIMEOUT;
+        abort = true;
+        break;
+      }
+      uint32_t wa[BITS], wb[BITS];
+      {
+        const uint32_t* s0 = reinterpret_cast<const uint32_t*>(ring + (st * kMmaRows + g) * kSeg) + t * BITS;
+        const uint32_t* s1 = reinterpret_cast<const uint32_t*>(ring + (st * kMmaRows + g + 8) * kSeg) + t * BITS;
+#pragma unroll
+        for (int w = 0; w < BITS; ++w) {
+          wa[w] = s0[w];
+          wb[w] = s1[w];
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (item + kMmaStages < nitems) issue(item + kMmaStages);
+      const uint4* xbj = a.xb + ((size_t)j * NT * 16) * 32 + lane;
+      uint32_t ia[kQ], ib[kQ];
+      unpack32<BITS>(wa, ia);
+      unpack32<BITS>(wb, ib);
+#pragma unroll
+      for (int kk = 0; kk < 16; ++kk) {
+        const uint2 a0 = lds_u2(tab_s + ((ia[2 * kk] << (RL + 3)) | rep8));
+        const uint2 a1 = lds_u2(tab_s + ((ib[2 * kk] << (RL + 3)) | rep8));
+        const uint2 a2 = lds_u2(tab_s + ((ia[2 * kk + 1] << (RL + 3)) | rep8));
+        const uint2 a3 = lds_u2(tab_s + ((ib[2 * kk + 1] << (RL + 3)) | rep8));
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const uint4 b = __ldg(xbj + (nt * 16 + kk) * 32);
+          mma_16816(acc[nt], a0.x, a1.x, a2.x, a3.x, b.x, b.y);  // hi . hi
+          mma_16816(acc[nt], a0.y, a1.y, a2.y, a3.y, b.x, b.y);  // lo . hi
+          mma_16816(acc[nt], a0.x, a1.x, a2.x, a3.x, b.z, b.w);  // hi . lo
+        }
       }
     }
+    // partial sums of this warp: rows g, g + 8; columns 8 nt + 2 t, + 1
+    float* rw = red + (size_t)warp * kMmaRows * 8 * NT;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      rw[g * 8 * NT + 8 * nt + 2 * t] = acc[nt][0];
+      rw[g * 8 * NT + 8 * nt + 2 * t + 1] = acc[nt][1];
+      rw[(g + 8) * 8 * NT + 8 * nt + 2 * t] = acc[nt][2];
+      rw[(g + 8) * 8 * NT + 8 * nt + 2 * t + 1] = acc[nt][3];
+    }
+    if (__syncthreads_or(abort)) break;
+    for (int e = tid; e < kMmaRows * a.batch; e += kMmaThreads) {
+      const int r = e % kMmaRows, n = e / kMmaRows;
+      if (r >= nrows) continue;
+      float sum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kMmaWarps; ++w) sum += red[(size_t)w * kMmaRows * 8 * NT + r * 8 * NT + n];
+      a.y[(int64_t)n * a.d_out + row0 + r] = __float2bfloat16_rn(sum * __half2float(a.rnorm[row0 + r]));
+    }
+    __syncthreads();  // red is rewritten by the next tile
   }
+  // copies still in flight (after a timeout) land before shared memory goes away
+  if (lane == 0) {
+    for (int s = 0; s < kMmaStages; ++s)
+      if (issued & (1u << s)) mbar_wait_bounded(&bars[s], (issued >> (8 + s)) & 1u);
+  }
+  raise_flag(a.status, flags);
 }
 
-constexpr size_t kGemvSmemCap = 200 * 1024;
-constexpr int kGemvRows = 2;  // rows per warp in k_gemv_s
-
-size_t gemv_s_smem(int K, int cl, int B, int d_in) {
-  return gemv1_table_bytes(K, cl) + (size_t)B * (d_in / 2) * sizeof(float2);
-}
-
-// Most codebook replicas (up to 16, 32 for K <= 1024) with which the table and
-// B columns of xbar fit in shared memory; -1 if not even one copy does.
-int gemv_s_copies_log2(int K, int B, int d_in) {
-  for (int cl = K <= 1024 ? 5 : 4; cl >= 0; --cl)
-    if (gemv_s_smem(K, cl, B, d_in) <= kGemvSmemCap) return cl;
-  return -1;
-}
-
-template <int BITS, int B, int R>
-cudaError_t run_gemv_s(const qamw_matrix& m, int batch, int t0, int cl, const float2* xbar,
-                       uint16_t* d_y, cudaStream_t stream) {
-  const int threads = 512, K = 1 << m.bits;
-  const size_t smem = gemv_s_smem(K, cl, B, m.d_in);
-  const void* fn = reinterpret_cast<const void*>(&k_gemv_s<BITS, B, R>);
+template <int BITS, int NT>
+cudaError_t run_gemv_mma(const qamw_matrix& m, int batch, const uint4* xb, uint16_t* d_y,
+                         int32_t* d_status, cudaStream_t stream) {
+  GemvMmaArgs a;
+  a.packed = m.packed;
+  a.rnorm = reinterpret_cast<const __half*>(m.row_norm);
+  a.codebook = reinterpret_cast<const float2*>(m.codebook);
+  a.xb = xb;
+  a.y = reinterpret_cast<__nv_bfloat16*>(d_y);
+  a.status = d_status;
+  a.row_bytes = m.row_bytes;
+  a.d_out = m.d_out;
+  a.P = m.d_in / 2;
+  a.batch = batch;
+  a.K = 1 << m.bits;
+  const size_t smem = gemv_mma_smem(a.K, BITS, NT);
+  const void* fn = reinterpret_cast<const void*>(&k_gemv_mma<BITS, NT>);
   cudaError_t err = allow_smem(fn, smem);
   if (err != cudaSuccess) return err;
-  const int64_t warps = (m.d_out + R - 1) / R;
-  const int grid = persistent_grid(fn, threads, smem, (warps * 32 + threads - 1) / threads);
-  return launch_pdl(k_gemv_s<BITS, B, R>, dim3(grid), dim3(threads), smem, stream, m.packed,
-                    m.row_bytes, reinterpret_cast<const __half*>(m.row_norm),
-                    reinterpret_cast<const float2*>(m.codebook), K, cl,
-                    static_cast<const float2*>(xbar), t0, m.d_out, m.d_in, batch,
-                    reinterpret_cast<__nv_bfloat16*>(d_y));
+  const int ntiles = (m.d_out + kMmaRows - 1) / kMmaRows;
+  const int grid = ntiles < sm_count() ? ntiles : sm_count();
+  return launch_pdl(k_gemv_mma<BITS, NT>, dim3(grid), dim3(kMmaThreads), smem, stream, a);
+}
+
+cudaError_t rotate_mma(const qamw_matrix& m, const uint16_t* d_x, int batch, int NT, uint4* xb,
+                       int32_t* d_status, cudaStream_t stream) {
+  const int64_t V = (int64_t)8 * NT * mma_chunks(m.d_in / 2) * 4;
+  const void* fn = reinterpret_cast<const void*>(&k_rotate_mma);
+  const int grid = persistent_grid(fn, kRotThreads, 0, (V + kRotItems - 1) / kRotItems);
+  return launch_pdl(k_rotate_mma, dim3(grid), dim3(kRotThreads), 0, stream,
+                    reinterpret_cast<const __nv_bfloat16*>(d_x), batch, NT, m.d_in, m.block,
+                    m.mask_seed, reinterpret_cast<const __half*>(m.chan_scale),
+                    reinterpret_cast<const __half*>(m.sigma), xb, d_status);
 }
 
 template <int BITS>
 cudaError_t gemv_bits(const qamw_matrix& m, const uint16_t* d_x, int batch, const float2* xbar,
                       uint16_t* d_y, int32_t* d_status, cudaStream_t stream) {
   if (batch == 1) return run_gemv1<BITS>(m, d_x, d_y, d_status, stream);
-  const int K = 1 << m.bits;
-  const int cl4 = gemv_s_copies_log2(K, 4, m.d_in), cl8 = gemv_s_copies_log2(K, 8, m.d_in);
-  if (batch <= 4 && cl4 >= 0)
-    return run_gemv_s<BITS, 4, kGemvRows>(m, batch, 0, cl4, xbar, d_y, stream);
-  if (cl8 >= 0) {  // column passes of 8
-    for (int t0 = 0; t0 < batch; t0 += 8) {
-      const cudaError_t err =
-          run_gemv_s<BITS, 8, kGemvRows>(m, batch, t0, cl8, xbar, d_y, stream);
-      if (err != cudaSuccess) return err;
-    }
-    return cudaSuccess;
-  }
-  if (batch <= 4) return run_gemv<BITS, 4>(m, batch, xbar, d_y, stream);
-  if (batch <= 8) return run_gemv<BITS, 8>(m, batch, xbar, d_y, stream);
-  return run_gemv<BITS, 16>(m, batch, xbar, d_y, stream);
+  // batch 2..16: rotation into the tensor-core layout, then the MMA kernel
+  uint4* xb = reinterpret_cast<uint4*>(const_cast<float2*>(xbar));
+  const int NT = batch <= 8 ? 1 : 2;
+  cudaError_t err = rotate_mma(m, d_x, batch, NT, xb, d_status, stream);
+  if (err != cudaSuccess) return err;
+  return NT == 1 ? run_gemv_mma<BITS, 1>(m, batch, xb, d_y, d_status, stream)
+                 : run_gemv_mma<BITS, 2>(m, batch, xb, d_y, d_status, stream);
 }
 
 }  // namespace
 
 size_t gemv_workspace_bytes(int d_in, int batch) {
-  // xbar padded to 16 batch columns so that the widest kernel can read them
+  // x_bar of batch > 1 in the tensor-core layout (8 or 16 columns, whole
+  // K-chunks); never less than 16 columns of fp32 pairs
   (void)batch;
-  return (size_t)16 * (size_t)(d_in / 2) * sizeof(float2);
+  const size_t mma = mma_xbar_bytes(d_in / 2, 2);
+  const size_t f32 = (size_t)16 * (size_t)(d_in / 2) * sizeof(float2);
+  return mma > f32 ? mma : f32;
 }
 
 cudaError_t launch_decode_gemv(const qamw_matrix& m, const uint16_t* d_x, int batch,
                                uint16_t* d_y, void* d_ws, int32_t* d_status,
                                cudaStream_t stream) {
   float2* xbar = static_cast<float2*>(d_ws);
-  if (batch > 1) {
-    const int bpad = batch <= 4 ? 4 : (batch <= 8 ? 8 : 16);
-    const int64_t V = (int64_t)bpad * (m.d_in / kE);
-    const void* fn = reinterpret_cast<const void*>(&k_rotate);
-    const int grid = persistent_grid(fn, kRotThreads, 0, (V + kRotItems - 1) / kRotItems);
-    cudaError_t err = launch_pdl(k_rotate, dim3(grid), dim3(kRotThreads), 0, stream,
-                                 reinterpret_cast<const __nv_bfloat16*>(d_x), batch, bpad,
-                                 m.d_in, m.block, m.mask_seed,
-                                 reinterpret_cast<const __half*>(m.chan_scale),
-                                 reinterpret_cast<const __half*>(m.sigma), xbar, d_status);
-    if (err != cudaSuccess) return err;
-  }
-  // The batch 2..16 kernels run B = 4/8/16 columns; columns batch..B-1 read
-  // the zeroed xbar padding and are not written to y.
   switch (m.bits) {
     case 1: return gemv_bits<1>(m, d_x, batch, xbar, d_y, d_status, stream);
     case 2: return gemv_bits<2>(m, d_x, batch, xbar, d_y, d_status, stream);
