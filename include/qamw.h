@@ -328,8 +328,14 @@ QAMW_API int qamw_decode_gemv(const qamw_matrix *m, const uint16_t *d_x, int bat
  *   d_in the library accepts); larger problems return QAMW_ERR_SHAPE and
  *   enqueue nothing.
  *   The first call on each device looks up that array's device address (with
- *   the device current) and caches it; make that first call before any stream
- *   capture.  The call allocates nothing and calls no allocating routine.
+ *   the device current) and caches it with the device's CUDA context, looking
+ *   it up again if that context is ever recreated (e.g. after
+ *   cudaDeviceReset); make that first call before any stream capture.  With
+ *   lazy module loading (the CUDA default) the array is reserved on a device
+ *   only when the library's device code first loads there, so a caller that
+ *   reserves all free device memory for itself should make one library call
+ *   on each device before doing so.  The call allocates nothing and calls no
+ *   allocating routine.
  *   Every call on a device uses the same array, which keeps the previous
  *   call's contents (each call overwrites everything it reads): calls whose
  *   work overlaps on the GPU -- e.g. on two streams at once -- race on it, so

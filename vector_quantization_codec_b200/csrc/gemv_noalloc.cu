@@ -11,9 +11,15 @@
 // process exits.
 //
 // The array's name is only a host-side stand-in in host code, never a device
-// address: the host looks the real address up once per device with
-// cudaGetSymbolAddress (with that device current) and hands that pointer to
-// the unchanged qamw_decode_gemv kernels.
+// address: the host looks the real address up with cudaGetSymbolAddress (with
+// the device current) and hands that pointer to the unchanged
+// qamw_decode_gemv kernels.  The lookup is cached per device together with the
+// CUDA context it was made in; when the device's context has been recreated
+// (after cudaDeviceReset, for example) the address is looked up again, so a
+// stale address is never used.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -22,30 +28,50 @@
 namespace qamw {
 namespace {
 
-// Room for the rotated activation of up to kNoAllocPairs pairs summed over the
-// padded batch columns (batch is padded to 1, 4, 8 or 16): 1 MiB, e.g. batch 16
-// with d_in <= 16384, or batch 1 with d_in up to the library limit of 32768.
+// Room for the rotated activation: 1 MiB.  The call accepts padded batch x
+// d_in / 2 <= 131072 pairs, where the batch is padded to 1, 4, 8 or 16 (e.g.
+// batch 16 with d_in <= 16384, or any batch of 8 or fewer with d_in up to the
+// library limit of 32768); every accepted shape's activation fits.
 constexpr size_t kNoAllocPairs = 131072;
 static __device__ __align__(256) float2 g_xbar_scratch[kNoAllocPairs];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};
 
-// Address of g_xbar_scratch on the current device; looked up on the first call
-// per device and cached.
+// The current CUDA context (driver entry point looked up once), or null.
+CUcontext current_context() {
+  static PFN_cuCtxGetCurrent_v4000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  }();
+  CUcontext ctx = nullptr;
+  if (fn == nullptr || fn(&ctx) != CUDA_SUCCESS) return nullptr;
+  return ctx;
+}
+
+// Address of g_xbar_scratch on the current device, looked up on the first call
+// in each context of the device and cached.
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  const CUcontext ctx = current_context();
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
+  if (g_scratch_ptr[dev] == nullptr || ctx == nullptr || ctx != g_scratch_ctx[dev]) {
+    // the lookup makes the device's context current if no call has yet
     void* p = nullptr;
     err = cudaGetSymbolAddress(&p, g_xbar_scratch);
     if (err != cudaSuccess) return err;
     if (p == nullptr) return cudaErrorInvalidSymbol;
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = current_context();
   }
   *out = g_scratch_ptr[dev];
   return cudaSuccess;

@@ -400,8 +400,13 @@ def qamw_decode_gemv_noalloc(m: EncodedMatrix, x: torch.Tensor, y: torch.Tensor,
     (this wrapper allocates nothing either).  Calls that overlap on the GPU
     share that array and must be serialised."""
     x2 = x if x.dim() == 2 else x.view(1, -1)
+    batch = x2.shape[0]
+    if x2.dtype != torch.bfloat16 or not x2.is_contiguous() or x2.shape[1] != m.d_in:
+        raise ValueError("x must be a contiguous bf16 [batch, d_in] tensor")
+    if (y.dtype != torch.bfloat16 or not y.is_contiguous() or tuple(y.shape) != (batch, m.d_out)
+            or y.device != x2.device):
+        raise ValueError("y must be a contiguous bf16 [batch, d_out] tensor on x's device")
     st = m.struct()
-    rc = _lib.qamw_decode_gemv_noalloc(C.byref(st), _p(x2), x2.shape[0], _p(y), _p(status),
-                                       _s(stream))
+    rc = _lib.qamw_decode_gemv_noalloc(C.byref(st), _p(x2), batch, _p(y), _p(status), _s(stream))
     _check("qamw_decode_gemv_noalloc", rc)
     return y
