@@ -71,6 +71,11 @@ def _load():
         "ref_polar_codebook": (None, [I, P, P]),
         "ref_polar_index": (I, [D, D, P, I]),
         "ref_encode_rows_polar": (None, [P, I, I, I, U64, P, P, P, I, I, I, P, P, P]),
+        "ref_gauss_lloyd_max": (None, [I, I, P]),
+        "ref_gauss_mse": (D, [I, P]),
+        "ref_scalar_codebook": (None, [I, P, P]),
+        "ref_scalar_index": (I, [D, D, P, I]),
+        "ref_encode_rows_scalar": (None, [P, I, I, I, U64, P, P, P, I, I, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -362,6 +367,75 @@ def encode_polar(W: np.ndarray, bits: int, block: int, levels: np.ndarray, *, ma
     def run(a, b):
         lib.ref_encode_rows_polar(_p(W), d_out, d_in, block, mask_seed, _p(s_half),
                                   _p(sigma_half), _p(lv), bits, a, b, _p(rnorm), _p(idx), _p(pts))
+
+    _parallel_rows(d_out, run, threads)
+    rb = row_bytes(d_in, bits)
+    out = dict(s_half=s_half, sigma_half=sigma_half, rnorm_half=rnorm, idx=idx,
+               packed=pack(idx, bits, rb), row_bytes=rb, bits=bits, block=block,
+               mask_seed=mask_seed, d_in=d_in, d_out=d_out)
+    if want_points:
+        out["points"] = pts
+    return out
+
+
+# ------------------------------------------------------------- d = 1 ablation
+
+def gauss_lloyd_max(L: int, iters: int = 20000) -> np.ndarray:
+    """Section 2 (parallel work), the d = 1 ablation: L-level Lloyd-Max quantiser of N(0, 1)."""
+    lv = np.empty(L, dtype=np.float64)
+    _load().ref_gauss_lloyd_max(L, iters, _p(lv))
+    return lv
+
+
+def gauss_mse(levels: np.ndarray) -> float:
+    """Mean squared error of the midpoint quantiser with these levels on N(0, 1)."""
+    lv = np.ascontiguousarray(levels, dtype=np.float64)
+    return float(_load().ref_gauss_mse(len(lv), _p(lv)))
+
+
+def scalar_levels(bits: int, iters: int = 20000) -> np.ndarray:
+    """The 2^(bits/2) levels of the scalar code with `bits` (even) per pair."""
+    if bits % 2:
+        raise ValueError("the scalar code needs an even number of bits per pair")
+    return gauss_lloyd_max(1 << (bits // 2), iters)
+
+
+def scalar_codebook(bits: int, levels: np.ndarray | None = None) -> np.ndarray:
+    """Product table: entry ix * L + iy = (l_ix, l_iy)."""
+    if levels is None:
+        levels = scalar_levels(bits)
+    lv = np.ascontiguousarray(levels, dtype=np.float64)
+    cb = np.empty((1 << bits, 2), dtype=np.float64)
+    _load().ref_scalar_codebook(bits, _p(lv), _p(cb))
+    return cb
+
+
+def scalar_index(points: np.ndarray, levels: np.ndarray, bits: int) -> np.ndarray:
+    lib = _load()
+    lv = np.ascontiguousarray(levels, dtype=np.float64)
+    pts = np.asarray(points, dtype=np.float64).reshape(-1, 2)
+    return np.array([lib.ref_scalar_index(float(x), float(y), _p(lv), bits) for x, y in pts],
+                    dtype=np.int32)
+
+
+def encode_scalar(W: np.ndarray, bits: int, block: int, levels: np.ndarray, *, mask_seed: int = 0,
+                  s_half: np.ndarray, sigma_half: np.ndarray, want_points: bool = False,
+                  threads: int | None = None) -> dict:
+    """Encoder of section 3.1 with the d = 1 scalar quantiser (given s, sigma)."""
+    W = np.ascontiguousarray(W, dtype=np.float64)
+    d_out, d_in = W.shape
+    P = d_in // 2
+    lv = np.ascontiguousarray(levels, dtype=np.float64)
+    s_half = np.ascontiguousarray(s_half, dtype=np.uint16)
+    sigma_half = np.ascontiguousarray(sigma_half, dtype=np.uint16)
+    rnorm = np.zeros(d_out, dtype=np.uint16)
+    idx = np.zeros((d_out, P), dtype=np.int32)
+    pts = np.zeros((d_out, P, 2), dtype=np.float64) if want_points else None
+    lib = _load()
+
+    def run(a, b):
+        lib.ref_encode_rows_scalar(_p(W), d_out, d_in, block, mask_seed, _p(s_half),
+                                   _p(sigma_half), _p(lv), bits, a, b, _p(rnorm), _p(idx), _p(pts))
 
     _parallel_rows(d_out, run, threads)
     rb = row_bytes(d_in, bits)

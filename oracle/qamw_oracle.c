@@ -579,3 +579,129 @@ void ref_encode_rows_polar(const double *W, int d_out, int d_in, int b, uint64_t
     free(scratch);
     free(y);
 }
+
+/* ------------------------------------------------------------------------ */
+/* Section 2 ("parallel work"), the d = 1 ablation the paper names as its    */
+/* first follow-up: the same pipeline with a one-dimensional codebook.       */
+/* Readings: each normalised coordinate of pair k (p = z_k / sigma_k; under   */
+/* eq. (1)'s model each coordinate is ~ N(0, 1)) is quantised on its own to   */
+/* the nearest of L = 2^(B/2) levels (ascending, strict '<', lowest index on */
+/* ties); the levels are the L-level Lloyd-Max quantiser of N(0, 1); B is     */
+/* even, so the scalar code spends B/2 bits per weight like the joint code    */
+/* with K = 2^B; index = i_x * L + i_y, so that it is an ordinary K-entry     */
+/* product table (l_ix, l_iy) for the decoder.                                */
+/* ------------------------------------------------------------------------ */
+
+/* Probability mass and first moment of N(0, 1) on [t0, t1) (infinite ends
+ * allowed): mass = (erf(t1/sqrt2) - erf(t0/sqrt2)) / 2,
+ * int x phi(x) dx = phi(t0) - phi(t1). */
+static void gauss_cell(double t0, double t1, double *mass, double *moment)
+{
+    double e0 = isinf(t0) ? -1.0 : erf(t0 / sqrt(2.0));
+    double e1 = isinf(t1) ? 1.0 : erf(t1 / sqrt(2.0));
+    double p0 = isinf(t0) ? 0.0 : exp(-0.5 * t0 * t0) / sqrt(2.0 * M_PI);
+    double p1 = isinf(t1) ? 0.0 : exp(-0.5 * t1 * t1) / sqrt(2.0 * M_PI);
+    *mass = 0.5 * (e1 - e0);
+    *moment = p0 - p1;
+}
+
+/* Lloyd-Max on N(0, 1): thresholds start evenly spaced on [-3, 3] (the paper
+ * gives no start; N(0, 1) is log-concave, so the fixed point is unique);
+ * alternate conditional means and midpoint thresholds for `iters` iterations. */
+void ref_gauss_lloyd_max(int L, int iters, double *levels)
+{
+    double *t = malloc(sizeof(double) * (size_t)(L + 1));
+    t[0] = -INFINITY;
+    t[L] = INFINITY;
+    for (int i = 1; i < L; ++i)
+        t[i] = -3.0 + 6.0 * i / L;
+    for (int it = 0; it <= iters; ++it) {
+        for (int i = 0; i < L; ++i) {
+            double m, mom;
+            gauss_cell(t[i], t[i + 1], &m, &mom);
+            levels[i] = mom / m;
+        }
+        if (it == iters)
+            break;
+        for (int i = 1; i < L; ++i)
+            t[i] = 0.5 * (levels[i - 1] + levels[i]);
+    }
+    free(t);
+}
+
+/* Mean squared error of the quantiser with these levels (midpoint cells) on
+ * N(0, 1): sum over cells of int (x - l)^2 phi = second moment - 2 l m1 + l^2 m0,
+ * with int x^2 phi on [a, b) = m0 + a phi(a) - b phi(b). */
+double ref_gauss_mse(int L, const double *levels)
+{
+    double mse = 0.0;
+    for (int i = 0; i < L; ++i) {
+        double a = i == 0 ? -INFINITY : 0.5 * (levels[i - 1] + levels[i]);
+        double b = i == L - 1 ? INFINITY : 0.5 * (levels[i] + levels[i + 1]);
+        double m0, m1;
+        gauss_cell(a, b, &m0, &m1);
+        double pa = isinf(a) ? 0.0 : a * exp(-0.5 * a * a) / sqrt(2.0 * M_PI);
+        double pb = isinf(b) ? 0.0 : b * exp(-0.5 * b * b) / sqrt(2.0 * M_PI);
+        double m2 = m0 + pa - pb;
+        mse += m2 - 2.0 * levels[i] * m1 + levels[i] * levels[i] * m0;
+    }
+    return mse;
+}
+
+void ref_scalar_codebook(int bits, const double *levels, double *codebook)
+{
+    int L = 1 << (bits / 2);
+    for (int ix = 0; ix < L; ++ix)
+        for (int iy = 0; iy < L; ++iy) {
+            codebook[2 * (ix * L + iy)] = levels[ix];
+            codebook[2 * (ix * L + iy) + 1] = levels[iy];
+        }
+}
+
+static int nearest_level(double v, const double *levels, int L)
+{
+    int best = 0;
+    double bd = INFINITY;
+    for (int i = 0; i < L; ++i) {
+        double d = fabs(v - levels[i]);
+        if (d < bd) {
+            bd = d;
+            best = i;
+        }
+    }
+    return best;
+}
+
+int ref_scalar_index(double px, double py, const double *levels, int bits)
+{
+    int L = 1 << (bits / 2);
+    return nearest_level(px, levels, L) * L + nearest_level(py, levels, L);
+}
+
+/* Encoder rows with the scalar quantiser in place of the joint 2D one. */
+void ref_encode_rows_scalar(const double *W, int d_out, int d_in, int b, uint64_t mask_seed,
+                            const uint16_t *s_half, const uint16_t *sigma_half,
+                            const double *levels, int bits, int row_begin, int row_end,
+                            uint16_t *rnorm_half, int32_t *idx, double *points_out)
+{
+    (void)d_out;
+    int P = d_in / 2;
+    double *scratch = malloc(sizeof(double) * (size_t)d_in);
+    double *y = malloc(sizeof(double) * (size_t)d_in);
+    for (int i = row_begin; i < row_end; ++i) {
+        double r = row_to_rotated(W + (int64_t)i * d_in, d_in, b, mask_seed, s_half, scratch, y);
+        rnorm_half[i] = ref_double_to_half(r);
+        for (int k = 0; k < P; ++k) {
+            double sg = ref_half_to_double(sigma_half[k]);
+            double px = y[2 * k] / sg, py = y[2 * k + 1] / sg;
+            int64_t o = (int64_t)i * P + k;
+            idx[o] = (r == 0.0) ? 0 : ref_scalar_index(px, py, levels, bits);
+            if (points_out) {
+                points_out[2 * o] = px;
+                points_out[2 * o + 1] = py;
+            }
+        }
+    }
+    free(scratch);
+    free(y);
+}
