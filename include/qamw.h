@@ -80,6 +80,9 @@ extern "C" {
 #define QAMW_SCALES_GIVEN 0x2 /* encode: use m->chan_scale as given           */
 #define QAMW_POLAR 0x4        /* encode: polar baseline quantiser (section    */
                               /* 3.5) against a qamw_polar_codebook table     */
+#define QAMW_SCALAR 0x8       /* encode: d = 1 scalar quantiser (section 2)   */
+                              /* against a qamw_scalar_codebook table; even   */
+                              /* bits only                                    */
 
 #define QAMW_OP_TRAIN 0
 #define QAMW_OP_ENCODE 1
@@ -184,7 +187,7 @@ QAMW_API int qamw_build_prefilter(const float *d_codebook, int bits, void *d_tab
  *              activation RMS), nullable.  s_j = binary16((a_j/mean a)^alpha);
  *              NULL or alpha == 0 gives s_j = 1.  Ignored with
  *              QAMW_SCALES_GIVEN (then m->chan_scale is read).
- *   flags      QAMW_SIGMA_GIVEN | QAMW_SCALES_GIVEN | QAMW_POLAR.
+ *   flags      QAMW_SIGMA_GIVEN | QAMW_SCALES_GIVEN | QAMW_POLAR or QAMW_SCALAR.
  *   m          shape, block, bits, mask_seed, row_bytes and buffers (in);
  *              packed, row_norm, sigma (unless given), chan_scale (unless
  *              given) (out).
@@ -283,6 +286,25 @@ QAMW_API int qamw_polar_codebook(int bits, float *d_codebook, void *stream);
  * is ignored.  Same as qamw_encode with QAMW_POLAR. */
 QAMW_API int qamw_encode_rows_polar(const void *d_W, int dtype, const qamw_matrix *m,
                                     int32_t *d_status, void *stream);
+
+/* The d = 1 ablation that section 2 ("parallel work") names as the first
+ * follow-up: the same pipeline with a one-dimensional codebook.  Each
+ * normalised coordinate of pair k (p = z_k / sigma_k, ~ N(0, 1) under eq. 1's
+ * model) is quantised on its own to the nearest of L = 2^(bits/2) levels (lowest
+ * index on ties); the levels are the L-level Lloyd-Max quantiser of N(0, 1);
+ * index = i_x * L + i_y, so the scalar code spends bits/2 bits per weight like
+ * the joint code with K = 2^bits.  bits must be even (2..10).
+ * qamw_scalar_codebook computes the levels (fp64 Lloyd-Max iteration, 20000
+ * steps from thresholds evenly spaced on [-3, 3]) and writes the product table
+ * d_codebook[ix * L + iy] = (l_ix, l_iy), [2^bits][2] fp32, 16-byte aligned: an
+ * ordinary codebook for qamw_decode and qamw_decode_gemv. */
+QAMW_API int qamw_scalar_codebook(int bits, float *d_codebook, void *stream);
+
+/* qamw_encode_rows with the d = 1 scalar quantiser; the levels are read from
+ * m->codebook (a qamw_scalar_codebook table); m->prefilter is ignored.  Same as
+ * qamw_encode with QAMW_SCALAR.  Errors: QAMW_ERR_INVALID for odd bits. */
+QAMW_API int qamw_encode_rows_scalar(const void *d_W, int dtype, const qamw_matrix *m,
+                                     int32_t *d_status, void *stream);
 
 /* Section 3.2 decoder: unpack, look up the codeword, rescale pair k by
  * sigma_k, reassemble, apply R_inv = diag(D) blockdiag(H_b) / sqrt(b),

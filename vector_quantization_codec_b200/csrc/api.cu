@@ -234,7 +234,10 @@ int qamw_encode(const void* d_W, int dtype, const float* d_act_stat, float alpha
   int rc = check_matrix(m, true);
   if (rc != QAMW_OK) return rc;
   if (dtype != QAMW_DTYPE_F32 && dtype != QAMW_DTYPE_BF16) return QAMW_ERR_INVALID;
-  if (flags & ~(QAMW_SIGMA_GIVEN | QAMW_SCALES_GIVEN | QAMW_POLAR)) return QAMW_ERR_INVALID;
+  if (flags & ~(QAMW_SIGMA_GIVEN | QAMW_SCALES_GIVEN | QAMW_POLAR | QAMW_SCALAR))
+    return QAMW_ERR_INVALID;
+  if ((flags & QAMW_POLAR) && (flags & QAMW_SCALAR)) return QAMW_ERR_INVALID;
+  if ((flags & QAMW_SCALAR) && m->bits % 2 != 0) return QAMW_ERR_INVALID;
   if (!std::isfinite(alpha)) return QAMW_ERR_INVALID;
   if (m->d_out == 0) return QAMW_OK;
   if (!d_W) return QAMW_ERR_INVALID;
@@ -310,7 +313,7 @@ int qamw_encode_rows(const void* d_W, int dtype, const qamw_matrix* m, uint64_t*
   if (!aligned16(d_W)) return QAMW_ERR_ALIGN;
   if (d_candidates && (reinterpret_cast<uintptr_t>(d_candidates) & 7u)) return QAMW_ERR_ALIGN;
   return cuda_rc(launch_encode_rows(d_W, dtype, *m, d_status,
-                                    reinterpret_cast<unsigned long long*>(d_candidates), false,
+                                    reinterpret_cast<unsigned long long*>(d_candidates), kJointMode,
                                     static_cast<cudaStream_t>(stream)));
 }
 
@@ -335,8 +338,27 @@ int qamw_encode_rows_polar(const void* d_W, int dtype, const qamw_matrix* m, int
   if (m->d_out == 0) return QAMW_OK;
   if (!d_W) return QAMW_ERR_INVALID;
   if (!aligned16(d_W)) return QAMW_ERR_ALIGN;
-  return cuda_rc(launch_encode_rows(d_W, dtype, *m, d_status, nullptr, true,
+  return cuda_rc(launch_encode_rows(d_W, dtype, *m, d_status, nullptr, kPolarMode,
                                     static_cast<cudaStream_t>(stream)));
+}
+
+int qamw_encode_rows_scalar(const void* d_W, int dtype, const qamw_matrix* m, int32_t* d_status,
+                            void* stream) {
+  int rc = check_matrix(m, true);
+  if (rc != QAMW_OK) return rc;
+  if (m->bits % 2 != 0) return QAMW_ERR_INVALID;
+  if (dtype != QAMW_DTYPE_F32 && dtype != QAMW_DTYPE_BF16) return QAMW_ERR_INVALID;
+  if (m->d_out == 0) return QAMW_OK;
+  if (!d_W) return QAMW_ERR_INVALID;
+  if (!aligned16(d_W)) return QAMW_ERR_ALIGN;
+  return cuda_rc(launch_encode_rows(d_W, dtype, *m, d_status, nullptr, kScalarMode,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+int qamw_scalar_codebook(int bits, float* d_codebook, void* stream) {
+  if (bits < 2 || bits > 10 || bits % 2 != 0 || !d_codebook) return QAMW_ERR_INVALID;
+  if (!aligned16(d_codebook)) return QAMW_ERR_ALIGN;
+  return cuda_rc(launch_scalar_codebook(bits, d_codebook, static_cast<cudaStream_t>(stream)));
 }
 
 int qamw_polar_codebook(int bits, float* d_codebook, void* stream) {

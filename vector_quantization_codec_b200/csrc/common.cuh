@@ -19,6 +19,9 @@
 namespace qamw {
 
 constexpr int kE = 64;  // columns per thread chunk
+// Quantiser of the row encoder: the joint 2D codebook, the polar baseline
+// (section 3.5) or the d = 1 scalar ablation (section 2).
+constexpr int kJointMode = 0, kPolarMode = 1, kScalarMode = 2;
 constexpr int kQ = 32;  // pairs per thread chunk
 // Largest d_in: the encoder keeps 6 bytes per column (D_j s_j and 1/sigma) plus
 // a 32 KB codebook in shared memory, within the 227 KB a CTA may use.
@@ -662,6 +665,25 @@ __device__ __forceinline__ uint2 pf_head_shared(float px, float py, const Prefil
 __device__ __forceinline__ int nearest_pf2(float px, float py, const float2* cb, int K,
                                            const PrefilterView& pf, unsigned& scored, bool count) {
   return pf_finish2(pf_head(px, py, pf), px, py, cb, K, pf, scored, count);
+}
+
+// d = 1 ablation: each coordinate to the nearest of the L levels (ascending,
+// strict '<', lowest index on ties); index = ix * L + iy.
+__device__ __forceinline__ int scalar_index(float px, float py, const float* lev, int L) {
+  int ix = 0, iy = 0;
+  float bx = INFINITY, by = INFINITY;
+  for (int i = 0; i < L; ++i) {
+    const float dx = fabsf(px - lev[i]), dy = fabsf(py - lev[i]);
+    if (dx < bx) {
+      bx = dx;
+      ix = i;
+    }
+    if (dy < by) {
+      by = dy;
+      iy = i;
+    }
+  }
+  return ix * L + iy;
 }
 
 // Polar baseline (paper section 3.5): amplitude |p| to the nearest of the Na

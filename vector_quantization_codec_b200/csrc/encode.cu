@@ -39,7 +39,7 @@ struct EncodeArgs {
 // butterflies, division by r sqrt(b) and sigma_k, nearest codeword, packing.
 // This form searches straight from the 64 rotated values in registers; it
 // serves rows too wide for k_encode's shared-memory point buffer.
-template <int BITS, typename T, bool POLAR>
+template <int BITS, typename T, int MODE>
 __global__ void __launch_bounds__(512, 1) k_encode_wide(const EncodeArgs<T> a) {
   extern __shared__ __align__(16) unsigned char smem[];
   pdl_wait();
@@ -52,10 +52,11 @@ __global__ void __launch_bounds__(512, 1) k_encode_wide(const EncodeArgs<T> a) {
   float* isgT = fT + a.d_in;                        // [q][c]: 1 / sigma of pair 32c + q
   float* part = isgT + P;                           // [blockDim] partial sums of squares
   float* rsum = part + blockDim.x;                  // [R] row norms
-  // polar: amplitude levels a_i = codeword (i Np).x of the expanded table
+  // polar: amplitude levels a_i = codeword (i Np).x of the expanded table;
+  // scalar: levels l_i = codeword (i L).x of the product table
   constexpr int kBa = BITS / 2, kNa = 1 << kBa, kNp = 1 << (BITS - kBa);
   float* lev = reinterpret_cast<float*>(cb2);
-  if constexpr (POLAR) {
+  if constexpr (MODE != kJointMode) {
     for (int i = threadIdx.x; i < kNa; i += blockDim.x) lev[i] = a.codebook[i * kNp].x;
   } else {
     // table fills: unrolled so that each thread's loads are in flight together
@@ -130,13 +131,16 @@ __global__ void __launch_bounds__(512, 1) k_encode_wide(const EncodeArgs<T> a) {
     uint32_t w[BITS];
 #pragma unroll
     for (int t = 0; t < BITS; ++t) w[t] = 0u;
-    if constexpr (POLAR) {
+    if constexpr (MODE != kJointMode) {
       const float np_over_2pi = (float)kNp * 0.159154943f;
 #pragma unroll
       for (int q = 0; q < kQ; ++q) {
         const float f = inv * isgT[q * C + c];
         const float px = x[2 * q] * f, py = x[2 * q + 1] * f;
-        const uint32_t id = zero ? 0u : (uint32_t)polar_index(px, py, lev, kNa, kNp, np_over_2pi);
+        const uint32_t id =
+            zero ? 0u
+                 : (uint32_t)(MODE == kPolarMode ? polar_index(px, py, lev, kNa, kNp, np_over_2pi)
+                                                 : scalar_index(px, py, lev, kNa));
         scored += kNa;
         const int bit = q * BITS, wi = bit >> 5, sh = bit & 31;
         w[wi] |= id << sh;
@@ -201,7 +205,7 @@ __global__ void __launch_bounds__(512, 1) k_encode_wide(const EncodeArgs<T> a) {
 // Shared memory: cb2 float2[K] | fT4 float4[16][C] | isg4 float4[8][C] |
 // part float[2][T] | rsum float[R] (padded) | pts float2[16][T] | hs uint2[S][S]
 // | bar uint64.
-template <int BITS, typename T, bool POLAR>
+template <int BITS, typename T, int MODE>
 __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int C = a.d_in / kE, NT = blockDim.x, R = a.rows_per_cta;
@@ -226,7 +230,7 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
   }
   // the shared copy of the inner grid: its table must be the one the launch
   // was sized for (a table for another codebook size reads as none)
-  const int S = (!POLAR && pf.G > 0 && pf.Gi == a.hs_gi) ? a.hs_side : 0;
+  const int S = (MODE == kJointMode && pf.G > 0 && pf.Gi == a.hs_gi) ? a.hs_side : 0;
   const int c0 = (pf.Gi - S) / 2;
   if (threadIdx.x == 0) {
     mbar_init(bar, 1);
@@ -238,9 +242,11 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
     for (int r = threadIdx.x; r < S; r += NT)
       bulk_g2s(hs + (size_t)r * S, pf.inner + (size_t)(c0 + r) * pf.Gi + c0, (unsigned)(S * 8), bar);
   }
+  // polar: amplitude levels a_i = codeword (i Np).x of the expanded table;
+  // scalar: levels l_i = codeword (i L).x of the product table
   constexpr int kBa = BITS / 2, kNa = 1 << kBa, kNp = 1 << (BITS - kBa);
   float* lev = reinterpret_cast<float*>(cb2);
-  if constexpr (POLAR) {
+  if constexpr (MODE != kJointMode) {
     for (int i = threadIdx.x; i < kNa; i += NT) lev[i] = a.codebook[i * kNp].x;
   } else {
 #pragma unroll 4
@@ -369,12 +375,14 @@ __global__ void __launch_bounds__(512, 1) k_encode(const EncodeArgs<T> a) {
           mypts[(4 * i + 2) * NT] = make_float2(x[2 * q0 + 4] * f2, x[2 * q0 + 5] * f2);
           mypts[(4 * i + 3) * NT] = make_float2(x[2 * q0 + 6] * f3, x[2 * q0 + 7] * f3);
         }
-        if constexpr (POLAR) {
+        if constexpr (MODE != kJointMode) {
           const float np_over_2pi = (float)kNp * 0.159154943f;
 #pragma unroll 4
           for (int q = 0; q < kQ / 2; ++q) {
             const float2 p = mypts[q * NT];
-            myid[q * 2 * NT] = (uint32_t)polar_index(p.x, p.y, lev, kNa, kNp, np_over_2pi);
+            myid[q * 2 * NT] =
+                (uint32_t)(MODE == kPolarMode ? polar_index(p.x, p.y, lev, kNa, kNp, np_over_2pi)
+                                              : scalar_index(p.x, p.y, lev, kNa));
             scored += kNa;
           }
         } else {
@@ -557,21 +565,21 @@ bool encode_shared_shape(int C, int K, int d_in, int gi, int* R_out, int* thread
   return true;
 }
 
-template <int BITS, typename T, bool POLAR>
+template <int BITS, typename T, int MODE>
 cudaError_t run_encode(EncodeArgs<T> a, cudaStream_t stream) {
   const int C = a.d_in / kE;
-  const int gi = (a.prefilter != nullptr && !POLAR) ? prefilter_inner(prefilter_grid(BITS)) : 0;
+  const int gi = (a.prefilter != nullptr && MODE == kJointMode) ? prefilter_inner(prefilter_grid(BITS)) : 0;
   int R, threads, side = 0;
   size_t smem;
   const void* fn;
   if (encode_shared_shape(C, a.K, a.d_in, gi, &R, &threads, &side, &smem)) {
-    fn = reinterpret_cast<const void*>(&k_encode<BITS, T, POLAR>);
+    fn = reinterpret_cast<const void*>(&k_encode<BITS, T, MODE>);
   } else {
     encode_shape(C, &R, &threads);
     smem = (size_t)((a.K + 1) & ~1) * sizeof(float2) + (size_t)a.d_in * sizeof(float) +
            (size_t)(a.d_in / 2) * sizeof(float) + (size_t)threads * sizeof(float) +
            (size_t)R * sizeof(float);
-    fn = reinterpret_cast<const void*>(&k_encode_wide<BITS, T, POLAR>);
+    fn = reinterpret_cast<const void*>(&k_encode_wide<BITS, T, MODE>);
   }
   a.rows_per_cta = R;
   a.hs_side = side;
@@ -583,7 +591,7 @@ cudaError_t run_encode(EncodeArgs<T> a, cudaStream_t stream) {
   return launch_pdl_ptr(fn, dim3(grid), dim3(threads), smem, stream, args);
 }
 
-template <typename T, bool POLAR>
+template <typename T, int MODE>
 cudaError_t encode_rows_typed(const T* W, const qamw_matrix& m, int32_t* st,
                               unsigned long long* cand, cudaStream_t stream) {
   EncodeArgs<T> a;
@@ -606,17 +614,17 @@ cudaError_t encode_rows_typed(const T* W, const qamw_matrix& m, int32_t* st,
   a.hs_gi = 0;
   a.seed = m.mask_seed;
   switch (m.bits) {
-    case 1: return run_encode<1, T, POLAR>(a, stream);
-    case 2: return run_encode<2, T, POLAR>(a, stream);
-    case 3: return run_encode<3, T, POLAR>(a, stream);
-    case 4: return run_encode<4, T, POLAR>(a, stream);
-    case 5: return run_encode<5, T, POLAR>(a, stream);
-    case 6: return run_encode<6, T, POLAR>(a, stream);
-    case 7: return run_encode<7, T, POLAR>(a, stream);
-    case 8: return run_encode<8, T, POLAR>(a, stream);
-    case 9: return run_encode<9, T, POLAR>(a, stream);
-    case 10: return run_encode<10, T, POLAR>(a, stream);
-    case 11: return run_encode<11, T, POLAR>(a, stream);
+    case 1: return run_encode<1, T, MODE>(a, stream);
+    case 2: return run_encode<2, T, MODE>(a, stream);
+    case 3: return run_encode<3, T, MODE>(a, stream);
+    case 4: return run_encode<4, T, MODE>(a, stream);
+    case 5: return run_encode<5, T, MODE>(a, stream);
+    case 6: return run_encode<6, T, MODE>(a, stream);
+    case 7: return run_encode<7, T, MODE>(a, stream);
+    case 8: return run_encode<8, T, MODE>(a, stream);
+    case 9: return run_encode<9, T, MODE>(a, stream);
+    case 10: return run_encode<10, T, MODE>(a, stream);
+    case 11: return run_encode<11, T, MODE>(a, stream);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -652,10 +660,45 @@ __global__ void __launch_bounds__(32) k_polar_codebook(int bits, int iters, floa
   }
 }
 
+// The d = 1 ablation (paper section 2, parallel work): Lloyd-Max levels of
+// N(0, 1) on one warp (lane i owns level i, L = 2^(bits/2) <= 32), fp64, from
+// thresholds evenly spaced on [-3, 3]; then the product table
+// c[ix L + iy] = (l_ix, l_iy).
+__global__ void __launch_bounds__(32) k_scalar_codebook(int bits, int iters, float2* __restrict__ cb) {
+  const int L = 1 << (bits / 2);
+  const int i = threadIdx.x;
+  const double rt2 = 1.4142135623730950488, inv_sqrt2pi = 0.39894228040143267794;
+  double t0 = i == 0 ? -INFINITY : -3.0 + 6.0 * i / L;
+  double t1 = i + 1 < L ? -3.0 + 6.0 * (i + 1) / L : INFINITY;
+  double lv = 0.0;
+  for (int it = 0; it <= iters; ++it) {
+    // centroid of [t0, t1): (phi(t0) - phi(t1)) / (Phi(t1) - Phi(t0))
+    const double p0 = isinf(t0) ? 0.0 : inv_sqrt2pi * exp(-0.5 * t0 * t0);
+    const double p1 = isinf(t1) ? 0.0 : inv_sqrt2pi * exp(-0.5 * t1 * t1);
+    const double e0 = isinf(t0) ? -1.0 : erf(t0 / rt2);
+    const double e1 = isinf(t1) ? 1.0 : erf(t1 / rt2);
+    lv = (p0 - p1) / (0.5 * (e1 - e0));
+    if (it == iters) break;
+    const double below = __shfl_up_sync(0xffffffffu, lv, 1);
+    const double above = __shfl_down_sync(0xffffffffu, lv, 1);
+    if (i > 0 && i < L) t0 = 0.5 * (below + lv);
+    if (i + 1 < L) t1 = 0.5 * (lv + above);
+  }
+  for (int j = 0; j < L; ++j) {
+    const double lj = __shfl_sync(0xffffffffu, lv, j);
+    if (i < L) cb[j * L + i] = make_float2((float)lj, (float)lv);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_polar_codebook(int bits, float* d_codebook, cudaStream_t stream) {
   k_polar_codebook<<<1, 32, 0, stream>>>(bits, 20000, reinterpret_cast<float2*>(d_codebook));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scalar_codebook(int bits, float* d_codebook, cudaStream_t stream) {
+  k_scalar_codebook<<<1, 32, 0, stream>>>(bits, 20000, reinterpret_cast<float2*>(d_codebook));
   return cudaGetLastError();
 }
 
@@ -703,19 +746,21 @@ cudaError_t launch_points(const void* d_W, int dtype, const qamw_matrix& m, int6
 }
 
 cudaError_t launch_encode_rows(const void* d_W, int dtype, const qamw_matrix& m, int32_t* d_status,
-                               unsigned long long* d_candidates, bool polar, cudaStream_t stream) {
-  if (polar) {
-    if (dtype == QAMW_DTYPE_F32)
-      return encode_rows_typed<float, true>(static_cast<const float*>(d_W), m, d_status,
-                                            d_candidates, stream);
-    return encode_rows_typed<__nv_bfloat16, true>(static_cast<const __nv_bfloat16*>(d_W), m,
-                                                  d_status, d_candidates, stream);
+                               unsigned long long* d_candidates, int mode, cudaStream_t stream) {
+  const bool f32 = dtype == QAMW_DTYPE_F32;
+  const float* Wf = static_cast<const float*>(d_W);
+  const __nv_bfloat16* Wb = static_cast<const __nv_bfloat16*>(d_W);
+  switch (mode) {
+    case kPolarMode:
+      return f32 ? encode_rows_typed<float, kPolarMode>(Wf, m, d_status, d_candidates, stream)
+                 : encode_rows_typed<__nv_bfloat16, kPolarMode>(Wb, m, d_status, d_candidates, stream);
+    case kScalarMode:
+      return f32 ? encode_rows_typed<float, kScalarMode>(Wf, m, d_status, d_candidates, stream)
+                 : encode_rows_typed<__nv_bfloat16, kScalarMode>(Wb, m, d_status, d_candidates, stream);
+    default:
+      return f32 ? encode_rows_typed<float, kJointMode>(Wf, m, d_status, d_candidates, stream)
+                 : encode_rows_typed<__nv_bfloat16, kJointMode>(Wb, m, d_status, d_candidates, stream);
   }
-  if (dtype == QAMW_DTYPE_F32)
-    return encode_rows_typed<float, false>(static_cast<const float*>(d_W), m, d_status,
-                                           d_candidates, stream);
-  return encode_rows_typed<__nv_bfloat16, false>(static_cast<const __nv_bfloat16*>(d_W), m,
-                                                 d_status, d_candidates, stream);
 }
 
 cudaError_t launch_encode(const void* d_W, int dtype, const float* d_act_stat, float alpha,
@@ -730,14 +775,17 @@ cudaError_t launch_encode(const void* d_W, int dtype, const float* d_act_stat, f
     err = launch_calibrate(d_W, dtype, m, ws, d_status, stream);
     if (err != cudaSuccess) return err;
   }
-  if (flags & QAMW_POLAR) return launch_encode_rows(d_W, dtype, m, d_status, nullptr, true, stream);
+  if (flags & QAMW_POLAR)
+    return launch_encode_rows(d_W, dtype, m, d_status, nullptr, kPolarMode, stream);
+  if (flags & QAMW_SCALAR)
+    return launch_encode_rows(d_W, dtype, m, d_status, nullptr, kScalarMode, stream);
   qamw_matrix mm = m;
   if (mm.prefilter == nullptr) {
     err = launch_build_prefilter(m.codebook, m.bits, prefilter_grid(m.bits), ws.prefilter, stream);
     if (err != cudaSuccess) return err;
     mm.prefilter = ws.prefilter;
   }
-  return launch_encode_rows(d_W, dtype, mm, d_status, nullptr, false, stream);
+  return launch_encode_rows(d_W, dtype, mm, d_status, nullptr, kJointMode, stream);
 }
 
 }  // namespace qamw

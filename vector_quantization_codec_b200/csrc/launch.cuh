@@ -90,8 +90,9 @@ cudaError_t launch_calibrate_many(const void* const* d_W, int dtype, const float
 cudaError_t launch_points(const void* d_W, int dtype, const qamw_matrix& m, int64_t row0,
                           int64_t nrows, float* d_points, int32_t* d_status, cudaStream_t stream);
 cudaError_t launch_encode_rows(const void* d_W, int dtype, const qamw_matrix& m, int32_t* d_status,
-                               unsigned long long* d_candidates, bool polar, cudaStream_t stream);
+                               unsigned long long* d_candidates, int mode, cudaStream_t stream);
 cudaError_t launch_polar_codebook(int bits, float* d_codebook, cudaStream_t stream);
+cudaError_t launch_scalar_codebook(int bits, float* d_codebook, cudaStream_t stream);
 cudaError_t launch_encode(const void* d_W, int dtype, const float* d_act_stat, float alpha,
                           int flags, const qamw_matrix& m, const EncodeWorkspace& ws,
                           int32_t* d_status, cudaStream_t stream);

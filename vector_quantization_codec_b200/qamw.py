@@ -35,6 +35,7 @@ QAMW_DTYPE_BF16 = 1
 QAMW_SIGMA_GIVEN = 0x1
 QAMW_SCALES_GIVEN = 0x2
 QAMW_POLAR = 0x4
+QAMW_SCALAR = 0x8
 QAMW_OP_TRAIN = 0
 QAMW_OP_ENCODE = 1
 QAMW_OP_GEMV = 2
@@ -48,6 +49,7 @@ EXPORTS = ("qamw_row_bytes", "qamw_default_block", "qamw_bits_per_weight",
            "qamw_encode_rows", "qamw_decode", "qamw_decode_many",
            "qamw_decode_gemv",
            "qamw_decode_gemv_noalloc", "qamw_polar_codebook", "qamw_encode_rows_polar",
+           "qamw_scalar_codebook", "qamw_encode_rows_scalar",
            "qamw_normalised_pairs", "qamw_selftest_wait_timeout")
 
 
@@ -92,6 +94,8 @@ def _load() -> C.CDLL:
         "qamw_decode_gemv_noalloc": (I, [C.POINTER(qamw_matrix), V, I, V, V, V]),
         "qamw_polar_codebook": (I, [I, V, V]),
         "qamw_encode_rows_polar": (I, [V, I, C.POINTER(qamw_matrix), V, V]),
+        "qamw_scalar_codebook": (I, [I, V, V]),
+        "qamw_encode_rows_scalar": (I, [V, I, C.POINTER(qamw_matrix), V, V]),
         "qamw_normalised_pairs": (I, [V, I, C.POINTER(qamw_matrix), I64, I64, V, V, V]),
         "qamw_selftest_wait_timeout": (I, [C.c_uint, V, V, V]),
     }
@@ -321,6 +325,24 @@ def qamw_encode_rows_polar(W: torch.Tensor, m: EncodedMatrix, status: torch.Tens
     st = m.struct()
     rc = _lib.qamw_encode_rows_polar(_p(W), _dtype_code(W), C.byref(st), _p(status), _s(stream))
     _check("qamw_encode_rows_polar", rc)
+    return m
+
+
+def qamw_scalar_codebook(bits: int, codebook: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """Product table [2^bits, 2] of the d = 1 scalar ablation (section 2)."""
+    if codebook is None:
+        codebook = torch.empty((1 << bits, 2), dtype=torch.float32, device="cuda")
+    _check("qamw_scalar_codebook", _lib.qamw_scalar_codebook(bits, _p(codebook), _s(stream)))
+    return codebook
+
+
+def qamw_encode_rows_scalar(W: torch.Tensor, m: EncodedMatrix, status: torch.Tensor | None = None,
+                            stream=None) -> EncodedMatrix:
+    """Steps 1-6 of section 3.1 with the d = 1 scalar quantiser."""
+    st = m.struct()
+    rc = _lib.qamw_encode_rows_scalar(_p(W), _dtype_code(W), C.byref(st), _p(status), _s(stream))
+    _check("qamw_encode_rows_scalar", rc)
     return m
 
 
