@@ -64,8 +64,8 @@ SMS = 148
 # the recorded sha256 (otherwise the roofline reports traffic null).  The
 # traffic of an average launch of the workload is this figure scaled by the
 # weights the launch encodes (encode traffic grows in proportion to the rows).
-ENCODE_TRAFFIC = {"bytes": 35311616 + 4608, "weights": 4096 * 4096,
-                  "sha256": "1f7e056fda94e64066c0105216993430be7fcc058e375719dcb48c9b4913154f"}
+ENCODE_TRAFFIC = {"bytes": 35319808 + 768, "weights": 4096 * 4096,
+                  "sha256": "02fd78878e92d576411fba459fdd97a0f5f389ccaa35710f8f911b3e9005098a"}
 ENCODE_SOURCES = ("vector_quantization_codec_b200/csrc/encode.cu",
                   "vector_quantization_codec_b200/csrc/common.cuh",
                   "vector_quantization_codec_b200/csrc/launch.cuh")
