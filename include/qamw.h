@@ -88,6 +88,7 @@ extern "C" {
 #define QAMW_OP_ENCODE 1
 #define QAMW_OP_GEMV 2
 #define QAMW_OP_CALIBRATE 3
+#define QAMW_OP_GEMM 4
 
 /* --------------------------------------------------------- encoded matrix */
 /* All pointers are device pointers owned by the caller.  The caller fills
@@ -124,7 +125,9 @@ QAMW_API double qamw_bits_per_weight(int d_in, int bits);
 /* Bytes of d_workspace needed by op (QAMW_OP_*).  TRAIN: d_out is ignored,
  * d_in is ignored, `bits` fixes K; ENCODE: includes room for a prefilter table
  * (needed when m->prefilter is NULL); CALIBRATE: row norms and partial sums of
- * qamw_calibrate_sigma; GEMV: batch columns of the rotated activation.
+ * qamw_calibrate_sigma; GEMV: batch columns of the rotated activation; GEMM:
+ * the rotated activation of `batch` tokens and the fp32 partial sums of
+ * qamw_decode_gemm (batch = tokens).
  * Returns 0 on invalid arguments. */
 QAMW_API size_t qamw_workspace_bytes(int op, int d_out, int d_in, int bits, int batch);
 
@@ -335,6 +338,19 @@ QAMW_API int qamw_decode_many(const qamw_matrix *ms, int n, uint16_t *const *d_W
  * Flags: NONFINITE (non-finite x). */
 QAMW_API int qamw_decode_gemv(const qamw_matrix *m, const uint16_t *d_x, int batch, uint16_t *d_y,
                      void *d_workspace, size_t ws_bytes, int32_t *d_status, void *stream);
+
+/* Prefill-size product Y = X * W_hat^T for many tokens, on the tensor cores,
+ * without forming W_hat (the form the paper's section 1 leaves to future work:
+ * fused kernels for latency).  The same identity as qamw_decode_gemv:
+ * Y[t][i] = r_i * sum_k < xbar_t[k], c[index_ik] >, xbar_t = sigma (.)
+ * R_fwd(x_t / s), as a dense contraction of gathered codewords with xbar
+ * (binary16 high and low parts of both, fp32 accumulation).
+ *   d_x [ntok][d_in] bf16, 16B-aligned; 1 <= ntok <= 65536.
+ *   d_y [ntok][d_out] bf16 output.
+ *   d_workspace qamw_workspace_bytes(QAMW_OP_GEMM, d_out, d_in, bits, ntok).
+ * Flags: NONFINITE (non-finite x), RANGE (|xbar| beyond binary16). */
+QAMW_API int qamw_decode_gemm(const qamw_matrix *m, const uint16_t *d_x, int ntok, uint16_t *d_y,
+                              void *d_workspace, size_t ws_bytes, int32_t *d_status, void *stream);
 
 /* Allocation-free variant of qamw_decode_gemv.  The paper has no counterpart:
  * this entry point exists for callers that cannot allocate device memory,

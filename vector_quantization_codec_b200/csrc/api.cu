@@ -185,6 +185,10 @@ size_t qamw_workspace_bytes(int op, int d_out, int d_in, int bits, int batch) {
     case QAMW_OP_GEMV:
       if (d_in <= 0 || d_in % kE || d_in > kMaxDin || batch < 1 || batch > 16) return 0;
       return gemv_workspace_bytes(d_in, batch);
+    case QAMW_OP_GEMM:
+      if (d_out < 0 || d_in <= 0 || d_in % kE || d_in > kMaxDin || batch < 1 || batch > kMaxTokens)
+        return 0;
+      return gemm_workspace_bytes(d_out, d_in, batch);
     default:
       return 0;
   }
@@ -401,6 +405,21 @@ int qamw_decode_gemv(const qamw_matrix* m, const uint16_t* d_x, int batch, uint1
   if (!d_workspace || ws_bytes < gemv_workspace_bytes(m->d_in, batch)) return QAMW_ERR_WORKSPACE;
   if (!aligned16(d_workspace)) return QAMW_ERR_ALIGN;
   return cuda_rc(launch_decode_gemv(*m, d_x, batch, d_y, d_workspace, d_status,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+int qamw_decode_gemm(const qamw_matrix* m, const uint16_t* d_x, int ntok, uint16_t* d_y,
+                     void* d_workspace, size_t ws_bytes, int32_t* d_status, void* stream) {
+  int rc = check_matrix(m, false);
+  if (rc != QAMW_OK) return rc;
+  if (ntok < 1 || ntok > kMaxTokens) return QAMW_ERR_INVALID;
+  if (m->d_out == 0) return QAMW_OK;
+  if (!d_x || !d_y) return QAMW_ERR_INVALID;
+  if (!aligned16(d_x)) return QAMW_ERR_ALIGN;
+  if (!d_workspace || ws_bytes < gemm_workspace_bytes(m->d_out, m->d_in, ntok))
+    return QAMW_ERR_WORKSPACE;
+  if (!aligned16(d_workspace)) return QAMW_ERR_ALIGN;
+  return cuda_rc(launch_decode_gemm(*m, d_x, ntok, d_y, d_workspace, d_status,
                                     static_cast<cudaStream_t>(stream)));
 }
 

@@ -26,6 +26,8 @@ constexpr int kQ = 32;  // pairs per thread chunk
 // Largest d_in: the encoder keeps 6 bytes per column (D_j s_j and 1/sigma) plus
 // a 32 KB codebook in shared memory, within the 227 KB a CTA may use.
 constexpr int kMaxDin = 32768;
+// Largest token count of the prefill decode-GEMM (qamw_decode_gemm).
+constexpr int kMaxTokens = 65536;
 
 // splitmix64 (Steele, Lea & Flood; Vigna's formulation) evaluated at a counter.
 __device__ __forceinline__ uint64_t mix64(uint64_t counter) {

@@ -103,6 +103,9 @@ cudaError_t launch_build_prefilter(const float* d_codebook, int bits, int G, voi
 cudaError_t launch_train(const float* d_samples, int64_t n, int bits, int iters,
                          float* d_codebook, double* d_distortion, void* d_ws,
                          int32_t* d_status, cudaStream_t stream);
+size_t gemm_workspace_bytes(int d_out, int d_in, int ntok);
+cudaError_t launch_decode_gemm(const qamw_matrix& m, const uint16_t* d_x, int ntok, uint16_t* d_y,
+                               void* d_ws, int32_t* d_status, cudaStream_t stream);
 cudaError_t launch_decode_gemv(const qamw_matrix& m, const uint16_t* d_x, int batch,
                                uint16_t* d_y, void* d_ws, int32_t* d_status,
                                cudaStream_t stream);

@@ -40,6 +40,7 @@ QAMW_OP_TRAIN = 0
 QAMW_OP_ENCODE = 1
 QAMW_OP_GEMV = 2
 QAMW_OP_CALIBRATE = 3
+QAMW_OP_GEMM = 4
 
 # Every symbol include/qamw.h declares (checked by the test suite).
 EXPORTS = ("qamw_row_bytes", "qamw_default_block", "qamw_bits_per_weight",
@@ -47,7 +48,7 @@ EXPORTS = ("qamw_row_bytes", "qamw_default_block", "qamw_bits_per_weight",
            "qamw_train_codebook", "qamw_build_prefilter", "qamw_encode", "qamw_channel_scales",
            "qamw_calibrate_sigma", "qamw_calibrate_many", "qamw_calibrate_many_workspace_bytes",
            "qamw_encode_rows", "qamw_decode", "qamw_decode_many",
-           "qamw_decode_gemv",
+           "qamw_decode_gemv", "qamw_decode_gemm",
            "qamw_decode_gemv_noalloc", "qamw_polar_codebook", "qamw_encode_rows_polar",
            "qamw_scalar_codebook", "qamw_encode_rows_scalar",
            "qamw_normalised_pairs", "qamw_selftest_wait_timeout")
@@ -91,6 +92,7 @@ def _load() -> C.CDLL:
         "qamw_decode": (I, [C.POINTER(qamw_matrix), V, V, V]),
         "qamw_decode_many": (I, [C.POINTER(qamw_matrix), I, C.POINTER(C.c_void_p), V, V]),
         "qamw_decode_gemv": (I, [C.POINTER(qamw_matrix), V, I, V, V, SZ, V, V]),
+        "qamw_decode_gemm": (I, [C.POINTER(qamw_matrix), V, I, V, V, SZ, V, V]),
         "qamw_decode_gemv_noalloc": (I, [C.POINTER(qamw_matrix), V, I, V, V, V]),
         "qamw_polar_codebook": (I, [I, V, V]),
         "qamw_encode_rows_polar": (I, [V, I, C.POINTER(qamw_matrix), V, V]),
@@ -411,6 +413,23 @@ def qamw_decode_gemv(m: EncodedMatrix, x: torch.Tensor, y: torch.Tensor | None =
     rc = _lib.qamw_decode_gemv(C.byref(st), _p(x2), batch, _p(y), _p(workspace), workspace.numel(),
                                _p(status), _s(stream))
     _check("qamw_decode_gemv", rc)
+    return y
+
+
+def qamw_decode_gemm(m: EncodedMatrix, x: torch.Tensor, y: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """Y = X W_hat^T (bf16 [ntok, d_out]) for many tokens on the tensor cores."""
+    ntok = x.shape[0]
+    if y is None:
+        y = torch.empty((ntok, m.d_out), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = _workspace(qamw_workspace_bytes(QAMW_OP_GEMM, m.d_out, m.d_in, m.bits, ntok),
+                               x.device)
+    st = m.struct()
+    rc = _lib.qamw_decode_gemm(C.byref(st), _p(x), ntok, _p(y), _p(workspace), workspace.numel(),
+                               _p(status), _s(stream))
+    _check("qamw_decode_gemm", rc)
     return y
 
 
