@@ -29,6 +29,8 @@ with its own seeds: weak scaling, no data-path collective).
 Also measured, outside the step and reported under `components`:
   * decode-GEMV on the 11008x4096 and 4096x11008 matrices at batch 1, 4 and 16,
     cycling through the 32 layers' gate (resp. down) matrices;
+  * the prefill-size decode-GEMM (tensor cores) on the same matrices at 64 and
+    128 tokens;
   * the 3.5 bpw variant: every linear weight of 40 13B-shaped layers with a
     K = 128 codebook, encode and decode, and the polar amplitude x phase
     quantiser of the same K as the comparison path.
@@ -56,6 +58,7 @@ LAYERS, LAYERS_13B = 32, 40
 WL_7B, WL_13B = 3, 4  # workload ids in the input seeds
 TRAIN_N, TRAIN_ITERS = 1 << 20, 50
 GEMV_BATCHES = (1, 4, 16)
+GEMM_TOKENS = (64, 128)
 FP32_LANES_PER_SM = 128
 SMS = 148
 
@@ -259,9 +262,10 @@ def measured_peaks() -> dict:
     try:
         with open(path) as f:
             p = json.load(f)
-        return dict(hbm_gbs=float(p["hbm_gbs"]), source="measured")
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16_tflops=float(p.get("bf16_tflops", 1590.0)),
+                    source="measured")
     except (OSError, KeyError, ValueError):
-        return dict(hbm_gbs=6650.0, source="fallback")
+        return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, source="fallback")
 
 
 def workload_config(layers: int, world: int) -> dict:
@@ -465,6 +469,7 @@ def run_gpu(args) -> dict | None:
 
     # ---- decode-GEMV on the MLP shapes at batch 1 / 4 / 16 (cycling 32 layers)
     gemv_lines = run_gemv_lines(args, wl, dev, stream, hbm)
+    gemm_lines = run_gemm_lines(args, wl, dev, stream, hbm, peaks["bf16_tflops"])
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(args, wl, stream, world, dev)
     del wl
@@ -500,6 +505,7 @@ def run_gpu(args) -> dict | None:
         "decode_gemv_b1_all": dict(ms=gemv_ms, GB_per_s=ab["gemv"] / (gemv_ms * 1e-3) / 1e9,
                                    frac_hbm=ab["gemv"] / (gemv_ms * 1e-3) / 1e9 / hbm),
         "decode_gemv_mlp": gemv_lines,
+        "decode_gemm_prefill": gemm_lines,
         "train": dict(ms=train_ms, samples=TRAIN_N, iters=TRAIN_ITERS, K=1 << BITS,
                       note="per-codec constant, outside the step"),
     }
@@ -593,6 +599,46 @@ def run_gemv_lines(args, wl, dev, stream, hbm) -> dict:
                 gflops=2.0 * b * d0["d_out"] * d0["d_in"] / (ms * 1e-3) / 1e9,
                 matrices_cycled=len(sel))
     wl.check_status("decode-GEMV lines")
+    return lines
+
+
+def run_gemm_lines(args, wl, dev, stream, hbm, bf16_tflops) -> dict:
+    """Prefill-size decode-GEMM (qamw_decode_gemm, tensor cores) on the 11008x4096
+    and 4096x11008 matrices at 64 and 128 tokens, each line one CUDA graph of
+    the calls on all layers' matrices of that shape."""
+    import torch
+
+    from vector_quantization_codec_b200 import qamw, synth
+    lines = {}
+    for name in ("gate", "down"):
+        sel = [i for i, d in enumerate(wl.mats) if d["name"] == name]
+        d0 = wl.mats[sel[0]]
+        for M in GEMM_TOKENS:
+            ws = torch.empty(qamw.qamw_workspace_bytes(qamw.QAMW_OP_GEMM, d0["d_out"], d0["d_in"], BITS, M),
+                             dtype=torch.uint8, device=dev)
+            xs = [torch.from_numpy(synth.gemv_x(M, d0["d_in"], seed=9000 + i)).to(torch.bfloat16).to(dev)
+                  for i in sel]
+            ys = [torch.empty((M, d0["d_out"]), dtype=torch.bfloat16, device=dev) for _ in sel]
+
+            def calls():
+                for i, x, y in zip(sel, xs, ys):
+                    qamw.qamw_decode_gemm(wl.m[i], x, y, workspace=ws, status=wl.status)
+
+            calls()
+            torch.cuda.synchronize()
+            g = capture(calls)
+            g.replay()
+            ms = time_graph(g, max(3, args.steps // 2), stream) / len(sel)
+            del g
+            flops = 2.0 * M * d0["d_out"] * d0["d_in"]
+            lines[f"{d0['d_out']}x{d0['d_in']}_m{M}"] = dict(
+                us_per_call=ms * 1e3, useful_tflops=flops / (ms * 1e-3) / 1e12,
+                executed_tflops=3 * flops / (ms * 1e-3) / 1e12,
+                frac_bf16_peak_executed=3 * flops / (ms * 1e-3) / 1e12 / bf16_tflops,
+                index_GB_per_s=d0["d_out"] * row_bytes(d0["d_in"], BITS) / (ms * 1e-3) / 1e9,
+                matrices_cycled=len(sel),
+                note="three binary16 MMAs per product (hi.hi, lo.hi, hi.lo)")
+    wl.check_status("decode-GEMM lines")
     return lines
 
 
@@ -853,8 +899,10 @@ def run_single_stage(args) -> dict:
         qamw.qamw_encode(W, m, act, ALPHA)
     ws_cal = torch.empty(qamw.qamw_workspace_bytes(qamw.QAMW_OP_CALIBRATE, rows, d_in, bits),
                          dtype=torch.uint8, device=dev)
-    ws_g = torch.empty(qamw.qamw_workspace_bytes(qamw.QAMW_OP_GEMV, rows, d_in, bits, args.batch),
+    ws_g = torch.empty(qamw.qamw_workspace_bytes(qamw.QAMW_OP_GEMV, rows, d_in, bits, min(args.batch, 16)),
                        dtype=torch.uint8, device=dev)
+    ws_gm = torch.empty(qamw.qamw_workspace_bytes(qamw.QAMW_OP_GEMM, rows, d_in, bits, args.batch),
+                        dtype=torch.uint8, device=dev)
     W_hat = torch.empty((rows, d_in), dtype=torch.bfloat16, device=dev)
     y = torch.empty((args.batch, rows), dtype=torch.bfloat16, device=dev)
     fns = {
@@ -862,6 +910,7 @@ def run_single_stage(args) -> dict:
         "calibrate": lambda: qamw.qamw_calibrate_sigma(W, m, workspace=ws_cal),
         "decode": lambda: qamw.qamw_decode(m, W_hat),
         "gemv": lambda: qamw.qamw_decode_gemv(m, x, y, workspace=ws_g),
+        "gemm": lambda: qamw.qamw_decode_gemm(m, x, y, workspace=ws_gm),
         "train": lambda: qamw.qamw_train_codebook(samples, bits, 1, codebook),
     }
     fn = fns[args.only]
@@ -889,7 +938,8 @@ def run_single_stage(args) -> dict:
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
     ab = algorithmic_bytes(rows, d_in, bits, args.batch)
-    key = {"encode": "encode", "calibrate": "encode", "decode": "decode", "gemv": "gemv"}.get(args.only)
+    key = {"encode": "encode", "calibrate": "encode", "decode": "decode", "gemv": "gemv",
+           "gemm": "gemv"}.get(args.only)
     out = dict(stage=args.only, rows=rows, d_in=d_in, bits=bits, batch=args.batch, ms=ms,
                timing="eager" if args.eager else "cuda graph of back-to-back calls",
                Mweights_per_s=rows * d_in / (ms * 1e-3) / 1e6)
@@ -913,12 +963,12 @@ def main(argv=None) -> int:
     ap.add_argument("--ref-rows", type=int, default=ORACLE_SAMPLE_ROWS,
                     help="--impl reference: rows of each sample step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["encode", "calibrate", "decode", "gemv", "train"],
+    ap.add_argument("--only", choices=["encode", "calibrate", "decode", "gemv", "gemm", "train"],
                     help="profiling mode: time one stage alone (no step, no JSON contract)")
     ap.add_argument("--rows", type=int, default=16384, help="--only: rows of the matrix")
     ap.add_argument("--din", type=int, default=4096, help="--only: columns of the matrix")
     ap.add_argument("--bits", type=int, default=BITS, help="--only: bits per pair")
-    ap.add_argument("--batch", type=int, default=1, help="--only gemv: batch columns")
+    ap.add_argument("--batch", type=int, default=1, help="--only gemv / gemm: batch columns / tokens")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--eager", action="store_true", help="--only: time eager calls, not a graph")
     args = ap.parse_args(argv)

@@ -15,13 +15,19 @@
 //                   and tile of 64 tokens, as the exact shared-memory image of a
 //                   K-major operand tile with the 128-byte swizzle (hi and lo),
 //                   so one bulk copy brings a B tile in;
-//   k_gemm_tc       a CTA owns 128 weight rows x 64 tokens x a range of K-chunks:
-//                   its threads decode the chunk's packed indices into swizzled
-//                   A tiles (hi, lo) in shared memory while one thread issues
-//                   the MMAs of the chunk before (2-stage ring; completion by
-//                   tcgen05.commit on an mbarrier); the fp32 accumulator lives in
-//                   64 columns of tensor memory and is written as a partial sum;
-//   k_gemm_reduce   Y = bf16(r_i * sum of the K-range partial sums, fixed order).
+//   k_gemm_tc       persistent and warp-specialised.  The work is the sequence
+//                   of units (tile of 128 weight rows, group of NT tokens,
+//                   K-chunk), chunks fastest; each CTA takes an equal share of
+//                   consecutive units.  Eight decode warps gather the codewords
+//                   of a chunk into swizzled A tiles (hi, lo) in shared memory,
+//                   a copy warp brings the chunk's B tiles in, one thread
+//                   issues the MMAs into an fp32 accumulator in tensor memory,
+//                   and four epilogue warps write the accumulator out as the
+//                   partial sum of the CTA's part of the (row tile, token group)
+//                   while the next one accumulates in the other buffer.  The
+//                   roles meet only at mbarriers (stage ring of A and B tiles,
+//                   two accumulator buffers);
+//   k_gemm_reduce   Y = bf16(r_i * sum of the partial sums, in CTA order).
 #include <algorithm>
 
 #include "common.cuh"
@@ -30,17 +36,22 @@
 namespace qamw {
 namespace {
 
-constexpr int kTcRows = 128;     // M of the MMA: weight rows per CTA tile
-constexpr int kTcTok = 64;       // N of the MMA: tokens per CTA tile
-constexpr int kTcK = 64;         // K-chunk: 64 columns = 32 pairs = one 128-byte row
-constexpr int kTcThreads = 256;  // two threads per weight row decode a chunk
-constexpr int kTcStages = 2;
-constexpr int kTcRepLog2 = 2;    // codeword replicas in the hi/lo table
+constexpr int kTcRows = 128;  // M of the MMA: weight rows per tile
+constexpr int kTcK = 64;      // K-chunk: 64 columns = 32 pairs = one 128-byte row
+constexpr int kImgTok = 64;   // tokens per x_bar image
+constexpr int kTcDecWarps = 8;          // warps 0-7: decode (two per 32 rows)
+constexpr int kTcEpiWarp = 8;           // warps 8-11: epilogue (tensor-memory lane quarters)
+constexpr int kTcMmaWarp = 12;          // warp 12: tensor-memory owner, lane 0 issues the MMAs
+constexpr int kTcCopyWarp = 13;         // warp 13: lane 0 copies the B tiles
+constexpr int kTcThreads = 14 * 32;
+constexpr int kTcRepLog2 = 2;           // codeword replicas in the hi/lo table
+constexpr int kMinUnits = 4;            // chunks per CTA at least
+constexpr int kMaxStages = 4;
 constexpr uint32_t kTileA = kTcRows * kTcK * 2;  // 16 KB: one binary16 A tile
-constexpr uint32_t kTileB = kTcTok * kTcK * 2;   // 8 KB: one binary16 B tile
-constexpr uint32_t kStage = 2 * kTileA + 2 * kTileB;  // A hi, A lo, B hi, B lo
+constexpr uint32_t kImg = kImgTok * kTcK * 2;    // 8 KB: one binary16 image of 64 tokens
+constexpr int kWordStride = 7;  // words per row in a decode warp's word buffer (odd)
 
-__host__ __device__ inline int tok_tiles(int ntok) { return (ntok + kTcTok - 1) / kTcTok; }
+__host__ __device__ inline int tok_tiles(int ntok) { return (ntok + kImgTok - 1) / kImgTok; }
 
 // binary16 high and low parts of a pair of floats.
 __device__ __forceinline__ uint2 split_h2(float a, float b) {
@@ -64,16 +75,19 @@ __host__ __device__ inline uint32_t swz(int r, int u) {
 
 // ------------------------------------------------------------ x_bar images
 
-// Image (c, tt, part) = 8 KB at ((c * ntt + tt) * 2 + part) * 8 KB: row = token
-// within the tile, 64 binary16 values of x_bar at columns 64c .. 64c + 63.
-// A CTA takes 32 (token, chunk) items: all threads form D x / s into shared
-// memory, then one warp rotates the 32 chunks (lane = item, consecutive chunks
-// of one token in consecutive lanes, so the shuffles of a block > 64 work).
+// Image (c, part, tt) = 8 KB at ((c * 2 + part) * ntt + tt) * 8 KB: row = token
+// within the tile of 64, 64 binary16 values of x_bar at columns 64c .. 64c + 63
+// (part 0: high, 1: low parts); the images of consecutive token tiles are
+// adjacent, so a group of 128 tokens is one 16 KB operand tile.  Tokens from
+// ntok to ntt * 64 are zero.  A CTA takes 32 (token, chunk) items: all threads
+// form D x / s into shared memory, then one warp rotates the 32 chunks (lane =
+// item, consecutive chunks of one token in consecutive lanes, so the shuffles
+// of a block > 64 work).
 constexpr int kImgItems = 32;
 constexpr int kImgThreads = 256;
 
 __global__ void __launch_bounds__(kImgThreads) k_xbar_images(const __nv_bfloat16* __restrict__ x,
-                                                             int ntok, int d_in, int block,
+                                                             int ntok, int ntt, int d_in, int block,
                                                              uint64_t seed,
                                                              const __half* __restrict__ s,
                                                              const __half* __restrict__ sigma,
@@ -81,8 +95,7 @@ __global__ void __launch_bounds__(kImgThreads) k_xbar_images(const __nv_bfloat16
                                                              int32_t* status) {
   __shared__ float buf[kImgItems][kE + 1];
   const int C = d_in / kE;
-  const int ntt = tok_tiles(ntok);
-  const int npad = ntt * kTcTok;
+  const int npad = ntt * kImgTok;
   const int64_t V = (int64_t)npad * C;
   const int nb = min(block, kE), lanes = max(block / kE, 1);
   const float inv_sqrt_b = 1.0f / sqrtf((float)block);
@@ -122,9 +135,9 @@ __global__ void __launch_bounds__(kImgThreads) k_xbar_images(const __nv_bfloat16
       if (active) {
         float sg[kQ];
         load_halves<kQ>(sigma + (int64_t)c * kQ, sg);
-        const int tt = (int)(t / kTcTok), row = (int)(t % kTcTok);
-        uint8_t* hi = img + ((size_t)(c * ntt + tt) * 2) * kTileB;
-        uint8_t* lo = hi + kTileB;
+        const int tt = (int)(t / kImgTok), row = (int)(t % kImgTok);
+        uint8_t* hi = img + ((size_t)(c * 2) * ntt + tt) * kImg;
+        uint8_t* lo = hi + (size_t)ntt * kImg;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {  // unit u: columns 8u .. 8u + 7 = pairs 4u .. 4u + 3
           uint32_t h[4], l[4];
@@ -159,16 +172,20 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-// Instruction descriptor of kind::f16: binary16 A and B (formats 0), fp32
-// accumulator (bits 4-5 = 1), both K-major, N >> 3 at bits 17-22, M >> 4 at
-// bits 24-28.
-constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kTcTok >> 3) << 17) | ((uint32_t)(kTcRows >> 4) << 24);
+// Instruction descriptor of kind::f16 for N tokens: binary16 A and B (formats
+// 0), fp32 accumulator (bits 4-5 = 1), both K-major, N >> 3 at bits 17-22,
+// M >> 4 at bits 24-28.
+template <int NT>
+constexpr uint32_t idesc_f16() {
+  return (1u << 4) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(kTcRows >> 4) << 24);
+}
 
+template <int NT>
 __device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t accumulate) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
-      "l"(da), "l"(db), "r"(kIdesc), "r"(accumulate)
+      "l"(da), "l"(db), "r"(idesc_f16<NT>()), "r"(accumulate)
       : "memory");
 }
 
@@ -187,6 +204,10 @@ __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // 16 consecutive fp32 columns of this warp's 32 tensor-memory lanes.
 __device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
@@ -202,38 +223,170 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// ------------------------------------------------------------ the GEMM
+
 struct GemmTcArgs {
   const uint8_t* packed;
   const float2* codebook;
   const uint8_t* img;  // x_bar images
-  float* partial;      // [splits][ntok pad][d_out] fp32
+  float* partial;      // [slot][ntt * 64][d_out] fp32
   int32_t* status;
   int64_t row_bytes;
-  int d_out, C, ntok, K, splits, ntt;
+  int64_t U;  // units: row tiles x token groups x chunks
+  int d_out, C, K, ntt, TG, stages;
 };
 
-// Shared memory: stages [2][A hi | A lo | B hi | B lo] (1024-byte aligned) |
-// table uint2 [K][4] | bars: B full [2], MMA done [2] | tensor-memory address.
-size_t gemm_tc_smem(int K) {
-  return 1024 + (size_t)kTcStages * kStage + ((size_t)K << (kTcRepLog2 + 3)) + 4 * 8 + 16;
+// The CTA (of G) whose share of the U units holds unit v: CTA b holds
+// [floor(b U / G), floor((b + 1) U / G)).
+__host__ __device__ inline int cta_of(int64_t v, int64_t U, int G) {
+  return (int)(((v + 1) * G - 1) / U);
 }
 
-template <int BITS>
+template <int NT>
+constexpr uint32_t stage_bytes() {
+  return 2 * kTileA + 2 * (uint32_t)NT * 128u;  // A hi, A lo, B hi, B lo
+}
+
+// Shared memory: stages [S][A hi | A lo | B hi | B lo] (1024-byte aligned) |
+// table uint2 [K][4] | decode warps' word buffers | bars: A full [S], B full
+// [S], MMA done [S], accumulator full [2], accumulator empty [2], final |
+// tensor-memory address.
+size_t gemm_tc_smem(uint32_t stage, int S, int K) {
+  return 1024 + (size_t)S * stage + ((size_t)K << (kTcRepLog2 + 3)) +
+         (size_t)kTcDecWarps * 32 * kWordStride * 4 + (size_t)(3 * S + 5) * 8 + 16;
+}
+
+int gemm_tc_stages(uint32_t stage, int K) {
+  const size_t limit = 227 * 1024;
+  int S = kMaxStages;
+  while (S > 2 && gemm_tc_smem(stage, S, K) > limit) --S;
+  return S;
+}
+
+// Words [F, F + NW) of a row's chunk hold the indices of half H (pairs 16 H ..
+// 16 H + 15).
+template <int BITS, int H>
+struct HalfWords {
+  static constexpr int F = (16 * H * BITS) >> 5;
+  static constexpr int L = (16 * (H + 1) * BITS - 1) >> 5;
+  static constexpr int NW = L - F + 1;
+};
+
+// Decode warps: warp w decodes half H = w / 4 (pairs 16 H .. 16 H + 15) of the
+// 32 rows 32 (w % 4) .. + 31 of every unit into the A tiles of the unit's stage.
+// The packed words are loaded coalesced (lane i of load j takes word j * 32 + i
+// of the 32 rows' half-chunks), two units ahead, and pass through the warp's
+// word buffer to the lane of their row.
+template <int BITS, int NT, int H>
+__device__ __forceinline__ void decode_role(const GemmTcArgs& a, unsigned char* smem, uint32_t stage,
+                                            uint32_t tab_s, uint32_t* wbuf, uint64_t* afull,
+                                            uint64_t* mdone, int64_t v_lo, int64_t v_hi,
+                                            int& flags) {
+  using HW = HalfWords<BITS, H>;
+  constexpr int NW = HW::NW;
+  const int lane = threadIdx.x & 31, q4 = (threadIdx.x >> 5) & 3;
+  const int r = 32 * q4 + lane;  // row within the tile
+  const uint32_t rep8 = (uint32_t)(lane & ((1 << kTcRepLog2) - 1)) << 3;
+  // load j of this lane: row rr[j] of the 32, word HW::F + wj[j] of its half
+  uint32_t goff[NW], soff[NW];
+  int rr[NW];
+#pragma unroll
+  for (int j = 0; j < NW; ++j) {
+    const int f = 32 * j + lane, row = f / NW, wj = f - row * NW;
+    rr[j] = row;
+    goff[j] = (uint32_t)(row * a.row_bytes) + 4u * (uint32_t)(HW::F + wj);
+    soff[j] = (uint32_t)(row * kWordStride + wj);
+  }
+  auto gload = [&](int64_t v, uint32_t (&g)[NW]) {
+    const int64_t item = v / a.C;
+    const int c = (int)(v - item * a.C);
+    const int rt = (int)(item / a.TG);
+    const int64_t row0 = (int64_t)rt * kTcRows + 32 * q4;
+    const uint8_t* base = a.packed + row0 * a.row_bytes + (size_t)c * BITS * 4;
+#pragma unroll
+    for (int j = 0; j < NW; ++j)
+      g[j] = (row0 + rr[j] < a.d_out)
+                 ? __ldg(reinterpret_cast<const uint32_t*>(base + goff[j]))
+                 : 0u;
+  };
+  int s = 0;
+  uint32_t u = 0;
+  bool ok = true;
+  auto step = [&](int64_t v, uint32_t (&g)[NW]) {
+    // this unit's words to the lanes of their rows; unit v + 2's words into g
+#pragma unroll
+    for (int j = 0; j < NW; ++j) wbuf[soff[j]] = g[j];
+    __syncwarp();
+    uint32_t w[NW];
+#pragma unroll
+    for (int j = 0; j < NW; ++j) w[j] = wbuf[lane * kWordStride + j];
+    __syncwarp();
+    if (v + 2 < v_hi) gload(v + 2, g);
+    const int64_t item = v / a.C;
+    const bool row_ok = (int64_t)(item / a.TG) * kTcRows + r < a.d_out;
+    uint2 cw[kQ / 2];
+#pragma unroll
+    for (int q = 0; q < kQ / 2; ++q) {
+      const int bit = (16 * H + q) * BITS - 32 * HW::F, wi = bit >> 5, sh = bit & 31;
+      uint32_t id;
+      if (sh + BITS <= 32)
+        id = w[wi] >> sh;
+      else
+        id = __funnelshift_r(w[wi], w[wi + 1], sh);
+      id &= (1u << BITS) - 1u;
+      cw[q] = lds_u2_tc(tab_s + ((id << (kTcRepLog2 + 3)) | rep8));
+      if (!row_ok) cw[q] = make_uint2(0u, 0u);
+    }
+    // the stage is free once the MMAs of its previous unit are done
+    if (u > 0 && !mbar_wait_bounded(&mdone[s], (u - 1) & 1u)) {
+      flags |= QAMW_STATUS_TIMEOUT;
+      ok = false;
+      return;
+    }
+    unsigned char* st = smem + (size_t)s * stage;
+#pragma unroll
+    for (int uu = 0; uu < 4; ++uu) {
+      const uint32_t o = swz(r, 4 * H + uu);
+      *reinterpret_cast<uint4*>(st + o) =
+          make_uint4(cw[4 * uu].x, cw[4 * uu + 1].x, cw[4 * uu + 2].x, cw[4 * uu + 3].x);
+      *reinterpret_cast<uint4*>(st + kTileA + o) =
+          make_uint4(cw[4 * uu].y, cw[4 * uu + 1].y, cw[4 * uu + 2].y, cw[4 * uu + 3].y);
+    }
+    fence_proxy_async_smem();  // the A tiles, written by the threads, to the tensor cores
+    mbar_arrive(&afull[s]);
+    if (++s == a.stages) {
+      s = 0;
+      ++u;
+    }
+  };
+  uint32_t gA[NW], gB[NW];
+  if (v_lo < v_hi) gload(v_lo, gA);
+  if (v_lo + 1 < v_hi) gload(v_lo + 1, gB);
+  for (int64_t v = v_lo; v < v_hi && ok; v += 2) {
+    step(v, gA);
+    if (ok && v + 1 < v_hi) step(v + 1, gB);
+  }
+}
+
+template <int BITS, int NT>
 __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const GemmTcArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint2* tab = reinterpret_cast<uint2*>(smem + (size_t)kTcStages * kStage);
-  uint64_t* bfull = reinterpret_cast<uint64_t*>(tab + ((size_t)a.K << kTcRepLog2));
-  uint64_t* mdone = bfull + kTcStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + kTcStages);
+  constexpr uint32_t stage = stage_bytes<NT>();
+  const int S = a.stages;
+  uint2* tab = reinterpret_cast<uint2*>(smem + (size_t)S * stage);
+  uint32_t* words = reinterpret_cast<uint32_t*>(tab + ((size_t)a.K << kTcRepLog2));
+  uint64_t* afull = reinterpret_cast<uint64_t*>(words + kTcDecWarps * 32 * kWordStride);
+  uint64_t* bfull = afull + S;
+  uint64_t* mdone = bfull + S;
+  uint64_t* accfull = mdone + S;
+  uint64_t* accempty = accfull + 2;
+  uint64_t* fin = accempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // tile: (row tile, token tile, K split), the split fastest
-  const int split = blockIdx.x % a.splits;
-  const int tt = (blockIdx.x / a.splits) % a.ntt;
-  const int rt = blockIdx.x / (a.splits * a.ntt);
-  const int c_lo = (int)((int64_t)split * a.C / a.splits);
-  const int c_hi = (int)((int64_t)(split + 1) * a.C / a.splits);
-  const int nc = c_hi - c_lo;
+  const int G = gridDim.x;
+  const int64_t v_lo = (int64_t)blockIdx.x * a.U / G;
+  const int64_t v_hi = ((int64_t)blockIdx.x + 1) * a.U / G;
 
   // the hi/lo codeword table needs nothing from the kernels ahead
   for (int j = tid; j < a.K; j += kTcThreads) {
@@ -244,16 +397,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const GemmTcArgs a) {
       tab[(j << kTcRepLog2) + ((r + lane) & ((1 << kTcRepLog2) - 1))] = u;
   }
   if (tid == 0) {
-    for (int s = 0; s < kTcStages; ++s) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&afull[s], kTcDecWarps * 32);
       mbar_init(&bfull[s], 1);
       mbar_init(&mdone[s], 1);
     }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], 128);
+    }
+    mbar_init(fin, 1);
     fence_mbar_init();
   }
-  if (warp == 0) {  // 64 columns of tensor memory for the 128 x 64 fp32 accumulator
+  if (warp == kTcMmaWarp) {  // two accumulators of NT fp32 columns each
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
-                 "r"(kTcTok)
+                 "r"(2 * NT)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -264,121 +423,135 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const GemmTcArgs a) {
   // the indices and x_bar come from the kernels ahead
   pdl_wait();
   pdl_trigger();
-
-  const int r = tid >> 1, h = tid & 1;  // weight row of the tile, half of the chunk
-  const int64_t row = (int64_t)rt * kTcRows + r;
-  const bool row_ok = row < a.d_out;
-  const uint32_t rep8 = (uint32_t)(lane & ((1 << kTcRepLog2) - 1)) << 3;
-  const uint32_t tab_s = smem_u32(tab);
   int flags = 0;
-  int issued = 0;  // chunks whose MMAs were committed (to mdone[chunk % 2])
-  int done = 0;    // chunks whose commit was waited for
-  for (int i = 0; i < nc; ++i) {
-    const int c = c_lo + i;
-    const int st = i % kTcStages;
-    unsigned char* stage = smem + (size_t)st * kStage;
-    // the stage is free once the MMAs of chunk i - 2 are done
-    if (i >= kTcStages) {
-      const int j = i - kTcStages;
-      const bool ok = mbar_wait_bounded(&mdone[st], (unsigned)(j / kTcStages) & 1u);
-      if (__syncthreads_or(!ok)) {
+
+  if (warp < kTcDecWarps) {
+    uint32_t* wbuf = words + warp * 32 * kWordStride;
+    if (warp < 4)
+      decode_role<BITS, NT, 0>(a, smem, stage, smem_u32(tab), wbuf, afull, mdone, v_lo, v_hi, flags);
+    else
+      decode_role<BITS, NT, 1>(a, smem, stage, smem_u32(tab), wbuf, afull, mdone, v_lo, v_hi, flags);
+  } else if (warp < kTcEpiWarp + 4) {
+    // epilogue: warp q4 reads lanes (rows) 32 q4 .. + 31 of the accumulator
+    const int q4 = warp & 3;
+    int n = 0;
+    for (int64_t v = v_lo; v < v_hi; ++n) {
+      const int64_t item = v / a.C;
+      const int64_t v_end = min(v_hi, (item + 1) * a.C);
+      const int b = n & 1;
+      const bool ok = mbar_wait_bounded(&accfull[b], (uint32_t)(n >> 1) & 1u);
+      if (__any_sync(0xffffffffu, !ok)) {
         flags |= QAMW_STATUS_TIMEOUT;
         break;
       }
-      done = j + 1;
-    }
-    if (tid == 0) {  // B tiles of this chunk and token tile: two 8 KB images
-      mbar_expect_tx(&bfull[st], 2 * kTileB);
-      bulk_g2s(stage + 2 * kTileA, a.img + ((size_t)(c * a.ntt + tt) * 2) * kTileB, 2 * kTileB,
-               &bfull[st]);
-    }
-    // A tiles: thread (r, h) decodes pairs 16h .. 16h + 15 of the chunk of row r
-    // into units 4h .. 4h + 3 of row r (hi and lo)
-    {
-      uint32_t w[BITS];
-      if (row_ok) {
-        const uint32_t* src =
-            reinterpret_cast<const uint32_t*>(a.packed + row * a.row_bytes) + (size_t)c * BITS;
+      tc_fence_after();
+      const int rt = (int)(item / a.TG), tg = (int)(item - (int64_t)rt * a.TG);
+      const int slot = (int)blockIdx.x - cta_of(item * a.C, a.U, G);
+      const int64_t orow = (int64_t)rt * kTcRows + 32 * q4 + lane;
+      float* dst = a.partial + ((size_t)slot * a.ntt * kImgTok + (size_t)tg * NT) * a.d_out;
 #pragma unroll
-        for (int t = 0; t < BITS; ++t) w[t] = __ldg(src + t);
-      } else {
+      for (int q = 0; q < NT / 16; ++q) {
+        float val[16];
+        tc_ld16(tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(b * NT + 16 * q), val);
+        if (orow < a.d_out) {
 #pragma unroll
-        for (int t = 0; t < BITS; ++t) w[t] = 0u;
-      }
-      uint32_t idx[kQ];
-      unpack32<BITS>(w, idx);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t q = h ? idx[16 + 4 * u + e] : idx[4 * u + e];
-          uint2 v = lds_u2_tc(tab_s + ((q << (kTcRepLog2 + 3)) | rep8));
-          if (!row_ok) v = make_uint2(0u, 0u);
-          hi[e] = v.x;
-          lo[e] = v.y;
+          for (int e = 0; e < 16; ++e) dst[(size_t)(16 * q + e) * a.d_out + orow] = val[e];
         }
-        *reinterpret_cast<uint4*>(stage + swz(r, 4 * h + u)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(stage + kTileA + swz(r, 4 * h + u)) =
-            make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
+      tc_fence_before();
+      mbar_arrive(&accempty[b]);
+      v = v_end;
     }
-    fence_proxy_async_smem();  // the A tiles, written by the threads, to the tensor cores
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      if (!mbar_wait_bounded(&bfull[st], (unsigned)(i / kTcStages) & 1u)) {
-        flags |= QAMW_STATUS_TIMEOUT;  // the MMAs of this chunk are skipped
-      } else {
+  } else if (warp == kTcMmaWarp) {
+    if (lane == 0) {
+      int s = 0;
+      uint32_t u = 0;
+      int n = 0;
+      bool ok = true;
+      for (int64_t v = v_lo; v < v_hi && ok; ++n) {
+        const int64_t v_end = min(v_hi, (v / a.C + 1) * a.C);
+        const int b = n & 1;
+        // the buffer's previous accumulation has been read out
+        if (n >= 2 && !mbar_wait_bounded(&accempty[b], (uint32_t)((n >> 1) - 1) & 1u)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t sa = smem_u32(stage);
-        const uint32_t ahi = sa, alo = sa + kTileA, bhi = sa + 2 * kTileA, blo = bhi + kTileB;
+        const uint32_t d = tmem + (uint32_t)(b * NT);
+        for (bool first = true; v < v_end; ++v, first = false) {
+          if (!mbar_wait_bounded(&afull[s], u & 1u) || !mbar_wait_bounded(&bfull[s], u & 1u)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + (size_t)s * stage);
+          const uint32_t ahi = sa, alo = sa + kTileA, bhi = sa + 2 * kTileA, blo = bhi + NT * 128;
 #pragma unroll
-        for (int k = 0; k < kTcK / 16; ++k) {  // 16 columns (32 bytes) per MMA
-          const uint32_t off = 32u * k;
-          tc_mma(tmem, smem_desc_sw128(ahi + off), smem_desc_sw128(bhi + off),
-                 (i > 0 || k > 0) ? 1u : 0u);
-          tc_mma(tmem, smem_desc_sw128(alo + off), smem_desc_sw128(bhi + off), 1u);
-          tc_mma(tmem, smem_desc_sw128(ahi + off), smem_desc_sw128(blo + off), 1u);
+          for (int k = 0; k < kTcK / 16; ++k) {  // 16 columns (32 bytes) per MMA
+            const uint32_t off = 32u * k;
+            tc_mma<NT>(d, smem_desc_sw128(ahi + off), smem_desc_sw128(bhi + off),
+                       (first && k == 0) ? 0u : 1u);
+            tc_mma<NT>(d, smem_desc_sw128(alo + off), smem_desc_sw128(bhi + off), 1u);
+            tc_mma<NT>(d, smem_desc_sw128(ahi + off), smem_desc_sw128(blo + off), 1u);
+          }
+          tc_commit(&mdone[s]);  // the stage is free once these MMAs are done
+          if (++s == S) {
+            s = 0;
+            ++u;
+          }
+        }
+        if (ok) tc_commit(&accfull[b]);
+      }
+      if (!ok) flags |= QAMW_STATUS_TIMEOUT;
+      // every MMA is done before the tensor memory is released
+      tc_commit(fin);
+      if (!mbar_wait_bounded(fin, 0)) flags |= QAMW_STATUS_TIMEOUT;
+    }
+  } else if (warp == kTcCopyWarp) {
+    if (lane == 0) {
+      int s = 0;
+      uint32_t u = 0;
+      int64_t issued = 0;
+      for (int64_t v = v_lo; v < v_hi; ++v) {
+        if (u > 0 && !mbar_wait_bounded(&mdone[s], (u - 1) & 1u)) {
+          flags |= QAMW_STATUS_TIMEOUT;
+          break;
+        }
+        const int64_t item = v / a.C;
+        const int c = (int)(v - item * a.C);
+        const int tg = (int)(item % a.TG);
+        unsigned char* st = smem + (size_t)s * stage + 2 * kTileA;
+        const uint8_t* src = a.img + ((size_t)(c * 2) * a.ntt + (size_t)tg * (NT / kImgTok)) * kImg;
+        mbar_expect_tx(&bfull[s], 2u * NT * 128u);
+        bulk_g2s(st, src, NT * 128u, &bfull[s]);
+        bulk_g2s(st + NT * 128, src + (size_t)a.ntt * kImg, NT * 128u, &bfull[s]);
+        ++issued;
+        if (++s == S) {
+          s = 0;
+          ++u;
         }
       }
-      tc_commit(&mdone[st]);  // arrives when the MMAs issued so far are done
-    }
-    issued = i + 1;
-  }
-  // every committed chunk's MMAs are done before the accumulator is read or the
-  // tensor memory released (also after a timeout)
-  for (int j = done; j < issued; ++j)
-    if (!mbar_wait_bounded(&mdone[j % kTcStages], (unsigned)(j / kTcStages) & 1u))
-      flags |= QAMW_STATUS_TIMEOUT;
-  tc_fence_after();
-  const bool failed = __syncthreads_or(flags & QAMW_STATUS_TIMEOUT);
-  // epilogue: warps 0-3 read their 32 lanes (rows) of the accumulator
-  if (warp < 4 && nc > 0 && !failed) {
-    const int64_t orow = (int64_t)rt * kTcRows + warp * 32 + lane;
-    float* dst = a.partial + ((size_t)split * a.ntt * kTcTok + (size_t)tt * kTcTok) * a.d_out;
-#pragma unroll
-    for (int q = 0; q < kTcTok / 16; ++q) {
-      float v[16];
-      tc_ld16(tmem + ((uint32_t)(warp * 32) << 16) + 16u * q, v);
-      if (orow < a.d_out) {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) dst[(size_t)(16 * q + e) * a.d_out + orow] = v[e];
-      }
+      // no copy in flight at exit: the last use of each stage has landed
+      for (int64_t j = max((int64_t)0, issued - S); j < issued; ++j)
+        if (!mbar_wait_bounded(&bfull[j % S], (uint32_t)(j / S) & 1u)) flags |= QAMW_STATUS_TIMEOUT;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcTok)
+  if (warp == kTcMmaWarp) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * NT)
                  : "memory");
   }
   raise_flag(a.status, flags);
 }
 
-// Y[t][i] = bf16(r_i * sum over splits of partial[split][t][i]), in split order.
-__global__ void __launch_bounds__(256) k_gemm_reduce(const float* __restrict__ partial, int splits,
-                                                     int ntok_pad, int ntok, int d_out,
+// Y[t][i] = bf16(r_i * sum of the partial sums of (row tile, token group) in
+// CTA order).
+__global__ void __launch_bounds__(256) k_gemm_reduce(const float* __restrict__ partial, int64_t U,
+                                                     int G, int C, int TG, int NT, int ntok_pad,
+                                                     int ntok, int d_out,
                                                      const __half* __restrict__ rnorm,
                                                      __nv_bfloat16* __restrict__ y) {
   pdl_wait();
@@ -387,24 +560,41 @@ __global__ void __launch_bounds__(256) k_gemm_reduce(const float* __restrict__ p
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
        e += (int64_t)gridDim.x * blockDim.x) {
     const int64_t t = e / d_out, i = e - t * d_out;
+    const int64_t item = (i / kTcRows) * TG + t / NT;
+    const int nseg = cta_of(item * C + C - 1, U, G) - cta_of(item * C, U, G) + 1;
     float sum = 0.f;
-    for (int s = 0; s < splits; ++s) sum += partial[((size_t)s * ntok_pad + t) * d_out + i];
+    for (int s = 0; s < nseg; ++s) sum += partial[((size_t)s * ntok_pad + t) * d_out + i];
     y[e] = __float2bfloat16_rn(sum * __half2float(rnorm[i]));
   }
 }
 
-// Splits of the K range: enough CTAs to cover the SMs about twice, at least
-// four chunks each.
-int gemm_splits(int d_out, int ntok, int C) {
-  const int tiles = ((d_out + kTcRows - 1) / kTcRows) * tok_tiles(ntok);
-  int s = (2 * sm_count() + tiles - 1) / tiles;
-  s = std::min(s, std::max(1, C / 4));
-  return std::max(s, 1);
+// The launch plan of a (d_out, d_in, ntok) product on the current device.
+struct GemmPlan {
+  int NT;      // tokens per tile: 64 or 128
+  int TG;      // token groups
+  int ntt;     // 64-token images (TG * NT / 64)
+  int G;       // CTAs
+  int segmax;  // partial sums per (row tile, token group) at most
+  int64_t U;   // units
+};
+
+GemmPlan plan_gemm(int d_out, int d_in, int ntok) {
+  GemmPlan p;
+  const int C = d_in / kE;
+  p.NT = ntok > kImgTok ? 128 : 64;
+  p.TG = (ntok + p.NT - 1) / p.NT;
+  p.ntt = p.TG * (p.NT / kImgTok);
+  p.U = (int64_t)((d_out + kTcRows - 1) / kTcRows) * p.TG * C;
+  p.G = (int)std::min<int64_t>(sm_count(), std::max<int64_t>(1, p.U / kMinUnits));
+  // an item of C units meets at most ceil((C - 1) / per) + 1 CTA shares
+  const int64_t per = std::max<int64_t>(1, p.U / p.G);
+  p.segmax = (int)std::min<int64_t>(p.G, (C - 1 + per - 1) / per + 1);
+  return p;
 }
 
-template <int BITS>
-cudaError_t run_gemm_tc(const qamw_matrix& m, const uint8_t* img, int ntok, float* partial,
-                        int splits, int32_t* d_status, cudaStream_t stream) {
+template <int BITS, int NT>
+cudaError_t run_gemm_tc(const qamw_matrix& m, const uint8_t* img, const GemmPlan& p, float* partial,
+                        int32_t* d_status, cudaStream_t stream) {
   GemmTcArgs a;
   a.packed = m.packed;
   a.codebook = reinterpret_cast<const float2*>(m.codebook);
@@ -412,67 +602,77 @@ cudaError_t run_gemm_tc(const qamw_matrix& m, const uint8_t* img, int ntok, floa
   a.partial = partial;
   a.status = d_status;
   a.row_bytes = m.row_bytes;
+  a.U = p.U;
   a.d_out = m.d_out;
   a.C = m.d_in / kE;
-  a.ntok = ntok;
   a.K = 1 << m.bits;
-  a.splits = splits;
-  a.ntt = tok_tiles(ntok);
-  const size_t smem = gemm_tc_smem(a.K);
-  const void* fn = reinterpret_cast<const void*>(&k_gemm_tc<BITS>);
+  a.ntt = p.ntt;
+  a.TG = p.TG;
+  a.stages = gemm_tc_stages(stage_bytes<NT>(), a.K);
+  const size_t smem = gemm_tc_smem(stage_bytes<NT>(), a.stages, a.K);
+  const void* fn = reinterpret_cast<const void*>(&k_gemm_tc<BITS, NT>);
   cudaError_t err = allow_smem(fn, smem);
   if (err != cudaSuccess) return err;
-  const int grid = ((m.d_out + kTcRows - 1) / kTcRows) * a.ntt * splits;
-  return launch_pdl(k_gemm_tc<BITS>, dim3(grid), dim3(kTcThreads), smem, stream, a);
+  return launch_pdl(k_gemm_tc<BITS, NT>, dim3(p.G), dim3(kTcThreads), smem, stream, a);
 }
+
+template <int BITS>
+cudaError_t run_gemm_bits(const qamw_matrix& m, const uint8_t* img, const GemmPlan& p,
+                          float* partial, int32_t* d_status, cudaStream_t stream) {
+  return p.NT == 128 ? run_gemm_tc<BITS, 128>(m, img, p, partial, d_status, stream)
+                     : run_gemm_tc<BITS, 64>(m, img, p, partial, d_status, stream);
+}
+
+size_t images_bytes(int C, int ntt) { return (size_t)C * 2 * ntt * kImg; }
 
 }  // namespace
 
 size_t gemm_workspace_bytes(int d_out, int d_in, int ntok) {
-  const int C = d_in / kE;
-  const size_t img = (size_t)C * tok_tiles(ntok) * 2 * kTileB;
-  const int splits_max = std::max(1, C / 4);
-  return img + (size_t)splits_max * tok_tiles(ntok) * kTcTok * (size_t)d_out * sizeof(float);
+  const GemmPlan p = plan_gemm(d_out, d_in, ntok);
+  return images_bytes(d_in / kE, p.ntt) +
+         (size_t)p.segmax * p.ntt * kImgTok * (size_t)d_out * sizeof(float);
 }
 
 cudaError_t launch_decode_gemm(const qamw_matrix& m, const uint16_t* d_x, int ntok, uint16_t* d_y,
                                void* d_ws, int32_t* d_status, cudaStream_t stream) {
   const int C = m.d_in / kE;
+  const GemmPlan p = plan_gemm(m.d_out, m.d_in, ntok);
+  if (p.U == 0) return cudaSuccess;
   uint8_t* img = static_cast<uint8_t*>(d_ws);
-  float* partial = reinterpret_cast<float*>(img + (size_t)C * tok_tiles(ntok) * 2 * kTileB);
-  const int splits = gemm_splits(m.d_out, ntok, C);
+  float* partial = reinterpret_cast<float*>(img + images_bytes(C, p.ntt));
   {
-    const int64_t V = (int64_t)tok_tiles(ntok) * kTcTok * C;
+    const int64_t V = (int64_t)p.ntt * kImgTok * C;
     const void* fn = reinterpret_cast<const void*>(&k_xbar_images);
     const int grid = persistent_grid(fn, kImgThreads, 0, (V + kImgItems - 1) / kImgItems);
     cudaError_t err = launch_pdl(k_xbar_images, dim3(grid), dim3(kImgThreads), 0, stream,
-                                 reinterpret_cast<const __nv_bfloat16*>(d_x), ntok, m.d_in,
+                                 reinterpret_cast<const __nv_bfloat16*>(d_x), ntok, p.ntt, m.d_in,
                                  m.block, m.mask_seed, reinterpret_cast<const __half*>(m.chan_scale),
                                  reinterpret_cast<const __half*>(m.sigma), img, d_status);
     if (err != cudaSuccess) return err;
   }
   cudaError_t err;
   switch (m.bits) {
-    case 1: err = run_gemm_tc<1>(m, img, ntok, partial, splits, d_status, stream); break;
-    case 2: err = run_gemm_tc<2>(m, img, ntok, partial, splits, d_status, stream); break;
-    case 3: err = run_gemm_tc<3>(m, img, ntok, partial, splits, d_status, stream); break;
-    case 4: err = run_gemm_tc<4>(m, img, ntok, partial, splits, d_status, stream); break;
-    case 5: err = run_gemm_tc<5>(m, img, ntok, partial, splits, d_status, stream); break;
-    case 6: err = run_gemm_tc<6>(m, img, ntok, partial, splits, d_status, stream); break;
-    case 7: err = run_gemm_tc<7>(m, img, ntok, partial, splits, d_status, stream); break;
-    case 8: err = run_gemm_tc<8>(m, img, ntok, partial, splits, d_status, stream); break;
-    case 9: err = run_gemm_tc<9>(m, img, ntok, partial, splits, d_status, stream); break;
-    case 10: err = run_gemm_tc<10>(m, img, ntok, partial, splits, d_status, stream); break;
-    case 11: err = run_gemm_tc<11>(m, img, ntok, partial, splits, d_status, stream); break;
+    case 1: err = run_gemm_bits<1>(m, img, p, partial, d_status, stream); break;
+    case 2: err = run_gemm_bits<2>(m, img, p, partial, d_status, stream); break;
+    case 3: err = run_gemm_bits<3>(m, img, p, partial, d_status, stream); break;
+    case 4: err = run_gemm_bits<4>(m, img, p, partial, d_status, stream); break;
+    case 5: err = run_gemm_bits<5>(m, img, p, partial, d_status, stream); break;
+    case 6: err = run_gemm_bits<6>(m, img, p, partial, d_status, stream); break;
+    case 7: err = run_gemm_bits<7>(m, img, p, partial, d_status, stream); break;
+    case 8: err = run_gemm_bits<8>(m, img, p, partial, d_status, stream); break;
+    case 9: err = run_gemm_bits<9>(m, img, p, partial, d_status, stream); break;
+    case 10: err = run_gemm_bits<10>(m, img, p, partial, d_status, stream); break;
+    case 11: err = run_gemm_bits<11>(m, img, p, partial, d_status, stream); break;
     default: return cudaErrorInvalidValue;
   }
   if (err != cudaSuccess) return err;
   const int64_t n = (int64_t)ntok * m.d_out;
   const void* rfn = reinterpret_cast<const void*>(&k_gemm_reduce);
   const int rgrid = persistent_grid(rfn, 256, 0, (n + 255) / 256);
-  return launch_pdl(k_gemm_reduce, dim3(rgrid), dim3(256), 0, stream, (const float*)partial, splits,
-                    tok_tiles(ntok) * kTcTok, ntok, m.d_out,
-                    reinterpret_cast<const __half*>(m.row_norm), reinterpret_cast<__nv_bfloat16*>(d_y));
+  return launch_pdl(k_gemm_reduce, dim3(rgrid), dim3(256), 0, stream, (const float*)partial, p.U,
+                    p.G, C, p.TG, p.NT, p.ntt * kImgTok, ntok, m.d_out,
+                    reinterpret_cast<const __half*>(m.row_norm),
+                    reinterpret_cast<__nv_bfloat16*>(d_y));
 }
 
 }  // namespace qamw
