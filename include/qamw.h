@@ -347,8 +347,13 @@ QAMW_API int qamw_decode_gemv(const qamw_matrix *m, const uint16_t *d_x, int bat
  * (binary16 high and low parts of both, fp32 accumulation).
  *   d_x [ntok][d_in] bf16, 16B-aligned; 1 <= ntok <= 65536.
  *   d_y [ntok][d_out] bf16 output.
- *   d_workspace qamw_workspace_bytes(QAMW_OP_GEMM, d_out, d_in, bits, ntok).
- * Flags: NONFINITE (non-finite x), RANGE (|xbar| beyond binary16). */
+ *   d_workspace qamw_workspace_bytes(QAMW_OP_GEMM, d_out, d_in, bits, ntok),
+ *     queried with the same device current (the work is shared out over its
+ *     SMs, and the partial sums of that split live in the workspace).
+ * The result is deterministic for a given device (fixed split, fixed order of
+ * the partial sums).
+ * Flags: NONFINITE (non-finite x), RANGE (|xbar| beyond binary16), TIMEOUT (a
+ * bounded wait inside the kernel ran out; the output is then not valid). */
 QAMW_API int qamw_decode_gemm(const qamw_matrix *m, const uint16_t *d_x, int ntok, uint16_t *d_y,
                               void *d_workspace, size_t ws_bytes, int32_t *d_status, void *stream);
 

@@ -60,8 +60,14 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
     os.makedirs(LIB_DIR, exist_ok=True)
     extra = list(extra or [])
 
+    # an object is rebuilt when its source, a header or this script is newer
+    deps = max(os.path.getmtime(p) for p in _inputs() if not p.endswith(".cu"))
+
     def compile_one(src: str) -> str:
         obj = os.path.join(OBJ_DIR, os.path.basename(src) + ".o")
+        if (not force and not extra and os.path.exists(obj)
+                and os.path.getmtime(obj) >= max(deps, os.path.getmtime(src))):
+            return obj
         cmd = [nvcc, *ARCH, *FLAGS, *extra, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)

@@ -47,7 +47,6 @@ constexpr int kTcThreads = 14 * 32;
 constexpr int kTcRepLog2 = 2;           // codeword replicas in the hi/lo table
 constexpr int kMinUnits = 4;            // chunks per CTA at least
 constexpr int kMaxStages = 4;
-constexpr uint32_t kTileA = kTcRows * kTcK * 2;  // 16 KB: one binary16 A tile
 constexpr uint32_t kImg = kImgTok * kTcK * 2;    // 8 KB: one binary16 image of 64 tokens
 constexpr int kWordStride = 7;  // words per row in a decode warp's word buffer (odd)
 
@@ -180,12 +179,25 @@ constexpr uint32_t idesc_f16() {
   return (1u << 4) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(kTcRows >> 4) << 24);
 }
 
+// One MMA, D (+)= A B^T, with A in tensor memory (lane = row of A, column =
+// two binary16 values along K) and B a K-major shared-memory tile.
 template <int NT>
-__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t accumulate) {
+__device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db,
+                                          uint32_t accumulate) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
-      "l"(da), "l"(db), "r"(idesc_f16<NT>()), "r"(accumulate)
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(db), "r"(idesc_f16<NT>()), "r"(accumulate)
+      : "memory");
+}
+
+// 16 consecutive 32-bit columns of this warp's 32 tensor-memory lanes.
+__device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
 }
 
@@ -242,24 +254,54 @@ __host__ __device__ inline int cta_of(int64_t v, int64_t U, int G) {
   return (int)(((v + 1) * G - 1) / U);
 }
 
+// Position in the unit sequence (chunk c of token group tg of row tile rt),
+// advanced without divisions.
+struct UnitCursor {
+  int c, tg, rt;
+  __device__ __forceinline__ void start(int64_t v, int C, int TG) {
+    const int64_t item = v / C;
+    c = (int)(v - item * C);
+    rt = (int)(item / TG);
+    tg = (int)(item - (int64_t)rt * TG);
+  }
+  __device__ __forceinline__ void next(int C, int TG) {
+    if (++c == C) {
+      c = 0;
+      if (++tg == TG) {
+        tg = 0;
+        ++rt;
+      }
+    }
+  }
+};
+
 template <int NT>
 constexpr uint32_t stage_bytes() {
-  return 2 * kTileA + 2 * (uint32_t)NT * 128u;  // A hi, A lo, B hi, B lo
+  return 2 * (uint32_t)NT * 128u;  // B hi, B lo
 }
 
-// Shared memory: stages [S][A hi | A lo | B hi | B lo] (1024-byte aligned) |
-// table uint2 [K][4] | decode warps' word buffers | bars: A full [S], B full
-// [S], MMA done [S], accumulator full [2], accumulator empty [2], final |
-// tensor-memory address.
+// Tensor memory (all 512 columns): accumulators [2][NT] from column 0, then
+// the A tiles of stage s at column 2 NT + 64 s (32 columns of binary16 pairs
+// for the high parts, 32 for the low parts; lane = weight row).
+constexpr uint32_t kTmemCols = 512;
+constexpr int kAStageCols = 64;
+
+// Shared memory: B stages [S][B hi | B lo] (1024-byte aligned) | table uint2
+// [K][4] | decode warps' word buffers | bars: A full [S], B full [S], MMA
+// done [S], accumulator full [2], accumulator empty [2], final |
+// tensor-memory address.  At least 116 KB, so that one CTA (the owner of the
+// whole tensor memory) runs per SM.
 size_t gemm_tc_smem(uint32_t stage, int S, int K) {
-  return 1024 + (size_t)S * stage + ((size_t)K << (kTcRepLog2 + 3)) +
-         (size_t)kTcDecWarps * 32 * kWordStride * 4 + (size_t)(3 * S + 5) * 8 + 16;
+  const size_t need = 1024 + (size_t)S * stage + ((size_t)K << (kTcRepLog2 + 3)) +
+                      (size_t)kTcDecWarps * 32 * kWordStride * 4 + (size_t)(3 * S + 5) * 8 + 16;
+  return std::max(need, (size_t)116 * 1024);
 }
 
-int gemm_tc_stages(uint32_t stage, int K) {
+template <int NT>
+int gemm_tc_stages(int K) {
   const size_t limit = 227 * 1024;
-  int S = kMaxStages;
-  while (S > 2 && gemm_tc_smem(stage, S, K) > limit) --S;
+  int S = std::min(kMaxStages, (int)(kTmemCols - 2 * NT) / kAStageCols);
+  while (S > 2 && gemm_tc_smem(stage_bytes<NT>(), S, K) > limit) --S;
   return S;
 }
 
@@ -278,8 +320,8 @@ struct HalfWords {
 // of the 32 rows' half-chunks), two units ahead, and pass through the warp's
 // word buffer to the lane of their row.
 template <int BITS, int NT, int H>
-__device__ __forceinline__ void decode_role(const GemmTcArgs& a, unsigned char* smem, uint32_t stage,
-                                            uint32_t tab_s, uint32_t* wbuf, uint64_t* afull,
+__device__ __forceinline__ void decode_role(const GemmTcArgs& a, uint32_t tmem, uint32_t tab_s,
+                                            uint32_t* wbuf, uint64_t* afull,
                                             uint64_t* mdone, int64_t v_lo, int64_t v_hi,
                                             int& flags) {
   using HW = HalfWords<BITS, H>;
@@ -297,21 +339,20 @@ __device__ __forceinline__ void decode_role(const GemmTcArgs& a, unsigned char* 
     goff[j] = (uint32_t)(row * a.row_bytes) + 4u * (uint32_t)(HW::F + wj);
     soff[j] = (uint32_t)(row * kWordStride + wj);
   }
-  auto gload = [&](int64_t v, uint32_t (&g)[NW]) {
-    const int64_t item = v / a.C;
-    const int c = (int)(v - item * a.C);
-    const int rt = (int)(item / a.TG);
-    const int64_t row0 = (int64_t)rt * kTcRows + 32 * q4;
-    const uint8_t* base = a.packed + row0 * a.row_bytes + (size_t)c * BITS * 4;
+  auto gload = [&](const UnitCursor& cu, uint32_t (&g)[NW]) {
+    const int64_t row0 = (int64_t)cu.rt * kTcRows + 32 * q4;
+    const uint8_t* base = a.packed + row0 * a.row_bytes + (size_t)cu.c * BITS * 4;
 #pragma unroll
     for (int j = 0; j < NW; ++j)
-      g[j] = (row0 + rr[j] < a.d_out)
-                 ? __ldg(reinterpret_cast<const uint32_t*>(base + goff[j]))
-                 : 0u;
+      g[j] = (row0 + rr[j] < a.d_out) ? __ldg(reinterpret_cast<const uint32_t*>(base + goff[j])) : 0u;
   };
   int s = 0;
   uint32_t u = 0;
   bool ok = true;
+  // cu: the unit decoded; pf: the unit two ahead, whose words are loaded
+  UnitCursor cu, pf;
+  cu.start(v_lo, a.C, a.TG);
+  pf = cu;
   auto step = [&](int64_t v, uint32_t (&g)[NW]) {
     // this unit's words to the lanes of their rows; unit v + 2's words into g
 #pragma unroll
@@ -321,9 +362,10 @@ __device__ __forceinline__ void decode_role(const GemmTcArgs& a, unsigned char* 
 #pragma unroll
     for (int j = 0; j < NW; ++j) w[j] = wbuf[lane * kWordStride + j];
     __syncwarp();
-    if (v + 2 < v_hi) gload(v + 2, g);
-    const int64_t item = v / a.C;
-    const bool row_ok = (int64_t)(item / a.TG) * kTcRows + r < a.d_out;
+    if (v + 2 < v_hi) gload(pf, g);
+    pf.next(a.C, a.TG);
+    const bool row_ok = (int64_t)cu.rt * kTcRows + r < a.d_out;
+    cu.next(a.C, a.TG);
     uint2 cw[kQ / 2];
 #pragma unroll
     for (int q = 0; q < kQ / 2; ++q) {
@@ -337,22 +379,28 @@ __device__ __forceinline__ void decode_role(const GemmTcArgs& a, unsigned char* 
       cw[q] = lds_u2_tc(tab_s + ((id << (kTcRepLog2 + 3)) | rep8));
       if (!row_ok) cw[q] = make_uint2(0u, 0u);
     }
-    // the stage is free once the MMAs of its previous unit are done
-    if (u > 0 && !mbar_wait_bounded(&mdone[s], (u - 1) & 1u)) {
+    // the stage is free once the MMAs of its previous unit are done (a
+    // warp-uniform decision: the tensor-memory stores below are warp-wide)
+    const bool free_ok = u == 0 || mbar_wait_bounded(&mdone[s], (u - 1) & 1u);
+    if (__any_sync(0xffffffffu, !free_ok)) {
       flags |= QAMW_STATUS_TIMEOUT;
       ok = false;
       return;
     }
-    unsigned char* st = smem + (size_t)s * stage;
+    // row r = lane 32 q4 + lane of tensor memory; pair 16 H + q -> column
+    // 16 H + q of the stage's high (then low) block
+    const uint32_t ta = tmem + ((uint32_t)(32 * q4) << 16) +
+                        (uint32_t)(2 * NT + kAStageCols * s + 16 * H);
+    uint32_t hv[16], lv[16];
 #pragma unroll
-    for (int uu = 0; uu < 4; ++uu) {
-      const uint32_t o = swz(r, 4 * H + uu);
-      *reinterpret_cast<uint4*>(st + o) =
-          make_uint4(cw[4 * uu].x, cw[4 * uu + 1].x, cw[4 * uu + 2].x, cw[4 * uu + 3].x);
-      *reinterpret_cast<uint4*>(st + kTileA + o) =
-          make_uint4(cw[4 * uu].y, cw[4 * uu + 1].y, cw[4 * uu + 2].y, cw[4 * uu + 3].y);
+    for (int q = 0; q < 16; ++q) {
+      hv[q] = cw[q].x;
+      lv[q] = cw[q].y;
     }
-    fence_proxy_async_smem();  // the A tiles, written by the threads, to the tensor cores
+    tc_st16(ta, hv);
+    tc_st16(ta + kAStageCols / 2, lv);
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    tc_fence_before();
     mbar_arrive(&afull[s]);
     if (++s == a.stages) {
       s = 0;
@@ -360,8 +408,10 @@ __device__ __forceinline__ void decode_role(const GemmTcArgs& a, unsigned char* 
     }
   };
   uint32_t gA[NW], gB[NW];
-  if (v_lo < v_hi) gload(v_lo, gA);
-  if (v_lo + 1 < v_hi) gload(v_lo + 1, gB);
+  if (v_lo < v_hi) gload(pf, gA);
+  pf.next(a.C, a.TG);
+  if (v_lo + 1 < v_hi) gload(pf, gB);
+  pf.next(a.C, a.TG);
   for (int64_t v = v_lo; v < v_hi && ok; v += 2) {
     step(v, gA);
     if (ok && v + 1 < v_hi) step(v + 1, gB);
@@ -409,10 +459,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const GemmTcArgs a) {
     mbar_init(fin, 1);
     fence_mbar_init();
   }
-  if (warp == kTcMmaWarp) {  // two accumulators of NT fp32 columns each
+  if (warp == kTcMmaWarp) {  // the accumulators and the A stages
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
-                 "r"(2 * NT)
+                 "r"(kTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -428,9 +478,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const GemmTcArgs a) {
   if (warp < kTcDecWarps) {
     uint32_t* wbuf = words + warp * 32 * kWordStride;
     if (warp < 4)
-      decode_role<BITS, NT, 0>(a, smem, stage, smem_u32(tab), wbuf, afull, mdone, v_lo, v_hi, flags);
+      decode_role<BITS, NT, 0>(a, tmem, smem_u32(tab), wbuf, afull, mdone, v_lo, v_hi, flags);
     else
-      decode_role<BITS, NT, 1>(a, smem, stage, smem_u32(tab), wbuf, afull, mdone, v_lo, v_hi, flags);
+      decode_role<BITS, NT, 1>(a, tmem, smem_u32(tab), wbuf, afull, mdone, v_lo, v_hi, flags);
   } else if (warp < kTcEpiWarp + 4) {
     // epilogue: warp q4 reads lanes (rows) 32 q4 .. + 31 of the accumulator
     const int q4 = warp & 3;
@@ -484,15 +534,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const GemmTcArgs a) {
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + (size_t)s * stage);
-          const uint32_t ahi = sa, alo = sa + kTileA, bhi = sa + 2 * kTileA, blo = bhi + NT * 128;
+          const uint32_t bhi = smem_u32(smem + (size_t)s * stage), blo = bhi + NT * 128;
+          const uint32_t ahi = tmem + (uint32_t)(2 * NT + kAStageCols * s), alo = ahi + kAStageCols / 2;
 #pragma unroll
-          for (int k = 0; k < kTcK / 16; ++k) {  // 16 columns (32 bytes) per MMA
-            const uint32_t off = 32u * k;
-            tc_mma<NT>(d, smem_desc_sw128(ahi + off), smem_desc_sw128(bhi + off),
-                       (first && k == 0) ? 0u : 1u);
-            tc_mma<NT>(d, smem_desc_sw128(alo + off), smem_desc_sw128(bhi + off), 1u);
-            tc_mma<NT>(d, smem_desc_sw128(ahi + off), smem_desc_sw128(blo + off), 1u);
+          for (int k = 0; k < kTcK / 16; ++k) {  // 16 K-columns per MMA: 8 tensor-memory
+                                                 // columns of A, 32 bytes of a B row
+            const uint64_t dbh = smem_desc_sw128(bhi + 32u * k), dbl = smem_desc_sw128(blo + 32u * k);
+            tc_mma_ts<NT>(d, ahi + 8u * k, dbh, (first && k == 0) ? 0u : 1u);
+            tc_mma_ts<NT>(d, alo + 8u * k, dbh, 1u);
+            tc_mma_ts<NT>(d, ahi + 8u * k, dbl, 1u);
           }
           tc_commit(&mdone[s]);  // the stage is free once these MMAs are done
           if (++s == S) {
@@ -512,16 +562,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const GemmTcArgs a) {
       int s = 0;
       uint32_t u = 0;
       int64_t issued = 0;
-      for (int64_t v = v_lo; v < v_hi; ++v) {
+      UnitCursor cu;
+      cu.start(v_lo, a.C, a.TG);
+      for (int64_t v = v_lo; v < v_hi; ++v, cu.next(a.C, a.TG)) {
         if (u > 0 && !mbar_wait_bounded(&mdone[s], (u - 1) & 1u)) {
           flags |= QAMW_STATUS_TIMEOUT;
           break;
         }
-        const int64_t item = v / a.C;
-        const int c = (int)(v - item * a.C);
-        const int tg = (int)(item % a.TG);
-        unsigned char* st = smem + (size_t)s * stage + 2 * kTileA;
-        const uint8_t* src = a.img + ((size_t)(c * 2) * a.ntt + (size_t)tg * (NT / kImgTok)) * kImg;
+        unsigned char* st = smem + (size_t)s * stage;
+        const uint8_t* src =
+            a.img + ((size_t)(cu.c * 2) * a.ntt + (size_t)cu.tg * (NT / kImgTok)) * kImg;
         mbar_expect_tx(&bfull[s], 2u * NT * 128u);
         bulk_g2s(st, src, NT * 128u, &bfull[s]);
         bulk_g2s(st + NT * 128, src + (size_t)a.ntt * kImg, NT * 128u, &bfull[s]);
@@ -541,31 +591,41 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const GemmTcArgs a) {
   if (warp == kTcMmaWarp) {
     __syncwarp();
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * NT)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                  : "memory");
   }
   raise_flag(a.status, flags);
 }
 
 // Y[t][i] = bf16(r_i * sum of the partial sums of (row tile, token group) in
-// CTA order).
-__global__ void __launch_bounds__(256) k_gemm_reduce(const float* __restrict__ partial, int64_t U,
-                                                     int G, int C, int TG, int NT, int ntok_pad,
-                                                     int ntok, int d_out,
-                                                     const __half* __restrict__ rnorm,
-                                                     __nv_bfloat16* __restrict__ y) {
+// CTA order).  Block (rt, j): rows 128 rt .. + 127 (one per thread) and tokens
+// 8 j .. 8 j + 7, all in one token group (whose partial sums exist for all its
+// tokens, padding included).
+constexpr int kRedTok = 8;
+__global__ void __launch_bounds__(kTcRows) k_gemm_reduce(const float* __restrict__ partial,
+                                                         int64_t U, int G, int C, int TG, int NT,
+                                                         int ntok_pad, int ntok, int d_out,
+                                                         const __half* __restrict__ rnorm,
+                                                         __nv_bfloat16* __restrict__ y) {
+  const int rt = blockIdx.x, t0 = blockIdx.y * kRedTok;
+  const int64_t i = (int64_t)rt * kTcRows + threadIdx.x;
+  const int64_t item = (int64_t)rt * TG + t0 / NT;
+  const int nseg = cta_of(item * C + C - 1, U, G) - cta_of(item * C, U, G) + 1;
   pdl_wait();
   pdl_trigger();
-  const int64_t n = (int64_t)ntok * d_out;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t t = e / d_out, i = e - t * d_out;
-    const int64_t item = (i / kTcRows) * TG + t / NT;
-    const int nseg = cta_of(item * C + C - 1, U, G) - cta_of(item * C, U, G) + 1;
-    float sum = 0.f;
-    for (int s = 0; s < nseg; ++s) sum += partial[((size_t)s * ntok_pad + t) * d_out + i];
-    y[e] = __float2bfloat16_rn(sum * __half2float(rnorm[i]));
+  if (i >= d_out) return;
+  float acc[kRedTok];
+#pragma unroll
+  for (int j = 0; j < kRedTok; ++j) acc[j] = 0.f;
+  for (int s = 0; s < nseg; ++s) {
+    const float* src = partial + ((size_t)s * ntok_pad + t0) * d_out + i;
+#pragma unroll
+    for (int j = 0; j < kRedTok; ++j) acc[j] += __ldg(src + (size_t)j * d_out);
   }
+  const float rn = __half2float(rnorm[i]);
+#pragma unroll
+  for (int j = 0; j < kRedTok; ++j)
+    if (t0 + j < ntok) y[(size_t)(t0 + j) * d_out + i] = __float2bfloat16_rn(acc[j] * rn);
 }
 
 // The launch plan of a (d_out, d_in, ntok) product on the current device.
@@ -608,7 +668,7 @@ cudaError_t run_gemm_tc(const qamw_matrix& m, const uint8_t* img, const GemmPlan
   a.K = 1 << m.bits;
   a.ntt = p.ntt;
   a.TG = p.TG;
-  a.stages = gemm_tc_stages(stage_bytes<NT>(), a.K);
+  a.stages = gemm_tc_stages<NT>(a.K);
   const size_t smem = gemm_tc_smem(stage_bytes<NT>(), a.stages, a.K);
   const void* fn = reinterpret_cast<const void*>(&k_gemm_tc<BITS, NT>);
   cudaError_t err = allow_smem(fn, smem);
@@ -666,10 +726,8 @@ cudaError_t launch_decode_gemm(const qamw_matrix& m, const uint16_t* d_x, int nt
     default: return cudaErrorInvalidValue;
   }
   if (err != cudaSuccess) return err;
-  const int64_t n = (int64_t)ntok * m.d_out;
-  const void* rfn = reinterpret_cast<const void*>(&k_gemm_reduce);
-  const int rgrid = persistent_grid(rfn, 256, 0, (n + 255) / 256);
-  return launch_pdl(k_gemm_reduce, dim3(rgrid), dim3(256), 0, stream, (const float*)partial, p.U,
+  const dim3 rgrid((m.d_out + kTcRows - 1) / kTcRows, (ntok + kRedTok - 1) / kRedTok);
+  return launch_pdl(k_gemm_reduce, rgrid, dim3(kTcRows), 0, stream, (const float*)partial, p.U,
                     p.G, C, p.TG, p.NT, p.ntt * kImgTok, ntok, m.d_out,
                     reinterpret_cast<const __half*>(m.row_norm),
                     reinterpret_cast<__nv_bfloat16*>(d_y));
