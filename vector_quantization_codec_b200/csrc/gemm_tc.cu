@@ -44,7 +44,7 @@ constexpr int kTcEpiWarp = 8;           // warps 8-11: epilogue (tensor-memory l
 constexpr int kTcMmaWarp = 12;          // warp 12: tensor-memory owner, lane 0 issues the MMAs
 constexpr int kTcCopyWarp = 13;         // warp 13: lane 0 copies the B tiles
 constexpr int kTcThreads = 14 * 32;
-constexpr int kTcRepLog2 = 2;           // codeword replicas in the hi/lo table
+constexpr int kTcRepLog2 = 3;           // codeword replicas in the hi/lo table
 constexpr int kMinUnits = 4;            // chunks per CTA at least
 constexpr int kMaxStages = 4;
 constexpr uint32_t kImg = kImgTok * kTcK * 2;    // 8 KB: one binary16 image of 64 tokens
@@ -327,7 +327,6 @@ __device__ __forceinline__ void decode_role(const GemmTcArgs& a, uint32_t tmem, 
   using HW = HalfWords<BITS, H>;
   constexpr int NW = HW::NW;
   const int lane = threadIdx.x & 31, q4 = (threadIdx.x >> 5) & 3;
-  const int r = 32 * q4 + lane;  // row within the tile
   const uint32_t rep8 = (uint32_t)(lane & ((1 << kTcRepLog2) - 1)) << 3;
   // load j of this lane: row rr[j] of the 32, word HW::F + wj[j] of its half
   uint32_t goff[NW], soff[NW];
@@ -349,10 +348,9 @@ __device__ __forceinline__ void decode_role(const GemmTcArgs& a, uint32_t tmem, 
   int s = 0;
   uint32_t u = 0;
   bool ok = true;
-  // cu: the unit decoded; pf: the unit two ahead, whose words are loaded
-  UnitCursor cu, pf;
-  cu.start(v_lo, a.C, a.TG);
-  pf = cu;
+  // pf: the unit whose words are loaded next (two ahead of the one decoded)
+  UnitCursor pf;
+  pf.start(v_lo, a.C, a.TG);
   auto step = [&](int64_t v, uint32_t (&g)[NW]) {
     // this unit's words to the lanes of their rows; unit v + 2's words into g
 #pragma unroll
@@ -364,8 +362,7 @@ __device__ __forceinline__ void decode_role(const GemmTcArgs& a, uint32_t tmem, 
     __syncwarp();
     if (v + 2 < v_hi) gload(pf, g);
     pf.next(a.C, a.TG);
-    const bool row_ok = (int64_t)cu.rt * kTcRows + r < a.d_out;
-    cu.next(a.C, a.TG);
+    // rows past d_out decode index 0: their accumulator rows are never read
     uint2 cw[kQ / 2];
 #pragma unroll
     for (int q = 0; q < kQ / 2; ++q) {
@@ -377,7 +374,6 @@ __device__ __forceinline__ void decode_role(const GemmTcArgs& a, uint32_t tmem, 
         id = __funnelshift_r(w[wi], w[wi + 1], sh);
       id &= (1u << BITS) - 1u;
       cw[q] = lds_u2_tc(tab_s + ((id << (kTcRepLog2 + 3)) | rep8));
-      if (!row_ok) cw[q] = make_uint2(0u, 0u);
     }
     // the stage is free once the MMAs of its previous unit are done (a
     // warp-uniform decision: the tensor-memory stores below are warp-wide)
