@@ -316,6 +316,12 @@ class Workload:
         gw = max(qamw.qamw_workspace_bytes(qamw.QAMW_OP_GEMV, d["d_out"], d["d_in"], bits, 16)
                  for d in mats)
         self.ws_gemv = torch.empty(gw, dtype=torch.uint8, device=dev)
+        # the batch-1 products of all matrices in one list call, in d_in order
+        # (matrices of one d_in share launches)
+        self.gemv_order = sorted(range(len(mats)), key=lambda i: mats[i]["d_in"])
+        self.ws_gemv_many = torch.empty(
+            max(16, qamw.qamw_decode_gemv_many_workspace_bytes([self.m[i] for i in self.gemv_order])),
+            dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
 
     @property
@@ -347,6 +353,12 @@ class Workload:
 
     def gemv(self, stream=None):
         from vector_quantization_codec_b200 import qamw
+        if self.x[0].shape[0] == 1:
+            o = self.gemv_order
+            qamw.qamw_decode_gemv_many([self.m[i] for i in o], [self.x[i] for i in o],
+                                       [self.y[i] for i in o], workspace=self.ws_gemv_many,
+                                       status=self.status, stream=stream)
+            return
         for m, x, y in zip(self.m, self.x, self.y):
             qamw.qamw_decode_gemv(m, x, y, workspace=self.ws_gemv, status=self.status, stream=stream)
 
@@ -547,7 +559,7 @@ def run_gpu(args) -> dict | None:
         "roofline": roofline,
         "clocks": clocks,
         "e2e": e2e,
-        "gpu_launches": args.steps * launches_per_step(nm),
+        "gpu_launches": args.steps * launches_per_step(mats),
         "wall_s_timed": wall1 - wall0,
     }
     if world == 1 and not args.no_cpu_baseline:
@@ -558,11 +570,17 @@ def run_gpu(args) -> dict | None:
 # kernels of one step: per matrix, encode 1 and decode-GEMV 1 (batch 1); per
 # group of 64 matrices, calibration 4 (scales, rows, extension, finish) and
 # decode 1
-LAUNCHES_PER_MATRIX = 2
-
-
-def launches_per_step(n_matrices: int) -> int:
-    return n_matrices * LAUNCHES_PER_MATRIX + 5 * ((n_matrices + 63) // 64)
+def launches_per_step(mats) -> int:
+    """Kernel launches of one step: an encoder launch per matrix; per run of up
+    to 64 matrices, four of calibration and one of decoding; per run of up to 64
+    matrices of one d_in, two of the batch-1 products (x_bar, then the GEMV)."""
+    n = len(mats)
+    runs = (n + 63) // 64
+    by_din = {}
+    for d in mats:
+        by_din[d["d_in"]] = by_din.get(d["d_in"], 0) + 1
+    gemv_runs = sum((k + 63) // 64 for k in by_din.values())
+    return n + 5 * runs + 2 * gemv_runs
 
 
 def run_gemv_lines(args, wl, dev, stream, hbm) -> dict:
@@ -905,12 +923,25 @@ def run_single_stage(args) -> dict:
                         dtype=torch.uint8, device=dev)
     W_hat = torch.empty((rows, d_in), dtype=torch.bfloat16, device=dev)
     y = torch.empty((args.batch, rows), dtype=torch.bfloat16, device=dev)
+    count = args.count if args.only == "gemv_many" else 1
+    if args.only == "gemv_many":
+        # `count` distinct encodings of W (own index buffers: more than L2 holds)
+        mlist = [m]
+        for i in range(1, count):
+            mi = qamw.EncodedMatrix.empty(rows, d_in, BLOCK, bits, codebook, i, prefilter)
+            qamw.qamw_encode(W, mi, act, ALPHA)
+            mlist.append(mi)
+        xl = [x[:1].clone() for _ in range(count)]
+        yl = [torch.empty((1, rows), dtype=torch.bfloat16, device=dev) for _ in range(count)]
+        ws_many = torch.empty(max(16, qamw.qamw_decode_gemv_many_workspace_bytes(mlist)),
+                              dtype=torch.uint8, device=dev)
     fns = {
         "encode": lambda: qamw.qamw_encode_rows(W, m),
         "calibrate": lambda: qamw.qamw_calibrate_sigma(W, m, workspace=ws_cal),
         "decode": lambda: qamw.qamw_decode(m, W_hat),
         "gemv": lambda: qamw.qamw_decode_gemv(m, x, y, workspace=ws_g),
         "gemm": lambda: qamw.qamw_decode_gemm(m, x, y, workspace=ws_gm),
+        "gemv_many": lambda: qamw.qamw_decode_gemv_many(mlist, xl, yl, workspace=ws_many),
         "train": lambda: qamw.qamw_train_codebook(samples, bits, 1, codebook),
     }
     fn = fns[args.only]
@@ -939,12 +970,14 @@ def run_single_stage(args) -> dict:
     ms = e0.elapsed_time(e1) / args.steps
     ab = algorithmic_bytes(rows, d_in, bits, args.batch)
     key = {"encode": "encode", "calibrate": "encode", "decode": "decode", "gemv": "gemv",
-           "gemm": "gemv"}.get(args.only)
+           "gemm": "gemv", "gemv_many": "gemv"}.get(args.only)
     out = dict(stage=args.only, rows=rows, d_in=d_in, bits=bits, batch=args.batch, ms=ms,
                timing="eager" if args.eager else "cuda graph of back-to-back calls",
-               Mweights_per_s=rows * d_in / (ms * 1e-3) / 1e6)
+               Mweights_per_s=count * rows * d_in / (ms * 1e-3) / 1e6)
+    if args.only == "gemv_many":
+        out["matrices"] = count
     if key:
-        out["GB_per_s"] = ab[key] / (ms * 1e-3) / 1e9
+        out["GB_per_s"] = count * ab[key] / (ms * 1e-3) / 1e9
     return out
 
 
@@ -963,12 +996,14 @@ def main(argv=None) -> int:
     ap.add_argument("--ref-rows", type=int, default=ORACLE_SAMPLE_ROWS,
                     help="--impl reference: rows of each sample step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["encode", "calibrate", "decode", "gemv", "gemm", "train"],
+    ap.add_argument("--only", choices=["encode", "calibrate", "decode", "gemv", "gemv_many", "gemm",
+                                       "train"],
                     help="profiling mode: time one stage alone (no step, no JSON contract)")
     ap.add_argument("--rows", type=int, default=16384, help="--only: rows of the matrix")
     ap.add_argument("--din", type=int, default=4096, help="--only: columns of the matrix")
     ap.add_argument("--bits", type=int, default=BITS, help="--only: bits per pair")
     ap.add_argument("--batch", type=int, default=1, help="--only gemv / gemm: batch columns / tokens")
+    ap.add_argument("--count", type=int, default=16, help="--only gemv_many: matrices in the list")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--eager", action="store_true", help="--only: time eager calls, not a graph")
     args = ap.parse_args(argv)

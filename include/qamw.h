@@ -339,6 +339,22 @@ QAMW_API int qamw_decode_many(const qamw_matrix *ms, int n, uint16_t *const *d_W
 QAMW_API int qamw_decode_gemv(const qamw_matrix *m, const uint16_t *d_x, int batch, uint16_t *d_y,
                      void *d_workspace, size_t ws_bytes, int32_t *d_status, void *stream);
 
+/* qamw_decode_gemv at batch 1 for n matrices in one call: y_i = x_i * W_hat_i^T
+ * (ms: host array of n descriptors; d_x, d_y: host arrays of n device
+ * pointers, d_x[i] [d_in_i] bf16 16B-aligned, d_y[i] [d_out_i] bf16).  The
+ * rotated activations x_bar_i are formed once each, into the workspace, and the
+ * products of consecutive matrices with the same d_in, block, bits and codebook
+ * share one launch (up to 64 at a time): the per-launch set-up (the replicated
+ * codeword table) is paid once for the run.  Each y_i equals the
+ * qamw_decode_gemv result for (ms[i], d_x[i]) bit for bit.
+ *   d_workspace qamw_decode_gemv_many_workspace_bytes(ms, n) bytes, 16B-aligned.
+ * Errors: those of qamw_decode_gemv for any matrix (nothing is enqueued then);
+ * QAMW_ERR_INVALID for n < 0 or null arrays.  Flags: NONFINITE (non-finite x). */
+QAMW_API size_t qamw_decode_gemv_many_workspace_bytes(const qamw_matrix *ms, int n);
+QAMW_API int qamw_decode_gemv_many(const qamw_matrix *ms, int n, const uint16_t *const *d_x,
+                                   uint16_t *const *d_y, void *d_workspace, size_t ws_bytes,
+                                   int32_t *d_status, void *stream);
+
 /* Prefill-size product Y = X * W_hat^T for many tokens, on the tensor cores,
  * without forming W_hat (the form the paper's section 1 leaves to future work:
  * fused kernels for latency).  The same identity as qamw_decode_gemv:

@@ -408,6 +408,31 @@ int qamw_decode_gemv(const qamw_matrix* m, const uint16_t* d_x, int batch, uint1
                                     static_cast<cudaStream_t>(stream)));
 }
 
+size_t qamw_decode_gemv_many_workspace_bytes(const qamw_matrix* ms, int n) {
+  if (n <= 0 || !ms) return 0;
+  return gemv_many_workspace_bytes(ms, n);
+}
+
+int qamw_decode_gemv_many(const qamw_matrix* ms, int n, const uint16_t* const* d_x,
+                          uint16_t* const* d_y, void* d_workspace, size_t ws_bytes,
+                          int32_t* d_status, void* stream) {
+  if (n < 0 || (n > 0 && (!ms || !d_x || !d_y))) return QAMW_ERR_INVALID;
+  for (int i = 0; i < n; ++i) {
+    const int rc = check_matrix(&ms[i], false);
+    if (rc != QAMW_OK) return rc;
+    if (ms[i].d_out == 0) continue;
+    if (!d_x[i] || !d_y[i]) return QAMW_ERR_INVALID;
+    if (!aligned16(d_x[i])) return QAMW_ERR_ALIGN;
+  }
+  if (n == 0) return QAMW_OK;
+  const size_t need = gemv_many_workspace_bytes(ms, n);
+  if (need == 0) return QAMW_OK;
+  if (!d_workspace || ws_bytes < need) return QAMW_ERR_WORKSPACE;
+  if (!aligned16(d_workspace)) return QAMW_ERR_ALIGN;
+  return cuda_rc(launch_decode_gemv_many(ms, n, d_x, d_y, d_workspace, d_status,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
 int qamw_decode_gemm(const qamw_matrix* m, const uint16_t* d_x, int ntok, uint16_t* d_y,
                      void* d_workspace, size_t ws_bytes, int32_t* d_status, void* stream) {
   int rc = check_matrix(m, false);

@@ -19,6 +19,7 @@
 //   MMAs (binary16 high/low parts, fp32 accumulation), the packed indices
 //   streaming into shared memory through per-warp bulk-copy rings.
 #include <utility>
+#include <vector>
 
 #include "common.cuh"
 #include "launch.cuh"
@@ -314,6 +315,340 @@ cudaError_t run_gemv1(const qamw_matrix& m, const uint16_t* d_x, uint16_t* d_y,
   if (threads <= 256)
     return launch_pdl(k_gemv1<BITS, 256>, dim3(grid), dim3(threads), smem, stream, a);
   return launch_pdl(k_gemv1<BITS, 512>, dim3(grid), dim3(threads), smem, stream, a);
+}
+
+// ------------------------------------------------ batch 1, many matrices
+//
+// qamw_decode_gemv_many: x_bar of every matrix is formed once, by
+// k_xbar1_many, into the workspace as [chunk][64] floats -- the arithmetic of
+// k_gemv1's own preparation, so the products are bitwise those of single calls
+// -- and one persistent launch per run of matrices with the same d_in, block,
+// bits and codebook (k_gemv1_many) builds the replicated codebook table once
+// and streams the tiles of all of them.  Each CTA takes a contiguous range of
+// the run's (matrix, tile) sequence and reloads its lanes' x_bar only where the
+// matrix changes.
+
+constexpr int kGemvManyMax = 64;
+constexpr int kXb1Threads = 128;
+
+struct Xbar1Mat {
+  const __nv_bfloat16* x;
+  const __half* sigma;
+  const __half* scale;
+  float* xbar;  // [C][64]
+  uint64_t seed;
+};
+
+template <int MAXM>
+struct Xbar1Args {
+  Xbar1Mat m[MAXM];
+  int32_t* status;
+  int n, d_in, block;
+};
+
+// One lane per (matrix, chunk), matrices consecutive, chunks of a matrix in
+// consecutive lanes (a block > 64 spans lanes of one matrix: C is a multiple of
+// block / 64).
+template <int MAXM>
+__global__ void __launch_bounds__(kXb1Threads) k_xbar1_many(const __grid_constant__ Xbar1Args<MAXM> a) {
+  const int C = a.d_in / kE;
+  const int64_t V = (int64_t)a.n * C;
+  const int64_t v = (int64_t)blockIdx.x * kXb1Threads + threadIdx.x;
+  const bool active = v < V;
+  const int mi = active ? (int)(v / C) : 0;
+  const int c = active ? (int)(v - (int64_t)mi * C) : 0;
+  const Xbar1Mat& M = a.m[mi];
+  int flags = 0;
+  pdl_wait();
+  pdl_trigger();
+  float xr[kE];
+  if (active) {
+    const uint4* xp = reinterpret_cast<const uint4*>(M.x + (int64_t)c * kE);
+    const uint4* sp = reinterpret_cast<const uint4*>(M.scale + (int64_t)c * kE);
+#pragma unroll
+    for (int t = 0; t < kE / 8; ++t) {
+      const uint4 xv = __ldg(xp + t);
+      const uint4 sv = __ldg(sp + t);
+      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+      const __half2* sh = reinterpret_cast<const __half2*>(&sv);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 s2 = __half22float2(sh[e]);
+        const float x0 = __uint_as_float(xw[e] << 16), x1 = __uint_as_float(xw[e] & 0xffff0000u);
+        if (!isfinite(x0) || !isfinite(x1)) flags = QAMW_STATUS_NONFINITE;
+        const int j = 8 * t + 2 * e, col = c * kE + j;
+        const float q0 = __fdiv_rn(x0, s2.x), q1 = __fdiv_rn(x1, s2.y);
+        xr[j] = mask_negative(M.seed, (uint32_t)col) ? -q0 : q0;
+        xr[j + 1] = mask_negative(M.seed, (uint32_t)(col + 1)) ? -q1 : q1;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < kE; ++j) xr[j] = 0.f;
+  }
+  fwht_reg<kE>(xr, min(a.block, kE));
+  fwht_lanes<kE>(xr, max(a.block / kE, 1));
+  if (active) {
+    const float inv_sqrt_b = 1.0f / sqrtf((float)a.block);
+    const uint4* sg8 = reinterpret_cast<const uint4*>(M.sigma + (int64_t)c * kQ);
+    float4* dst = reinterpret_cast<float4*>(M.xbar + (int64_t)c * kE);
+#pragma unroll
+    for (int t = 0; t < kQ / 8; ++t) {  // sigma of pairs 8t .. 8t + 7
+      const uint4 u = __ldg(sg8 + t);
+      const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f2 = __half22float2(h[e]);
+        const int q = 8 * t + 2 * e;
+        dst[q / 2] = make_float4(xr[2 * q] * (f2.x * inv_sqrt_b), xr[2 * q + 1] * (f2.x * inv_sqrt_b),
+                                 xr[2 * q + 2] * (f2.y * inv_sqrt_b),
+                                 xr[2 * q + 3] * (f2.y * inv_sqrt_b));
+      }
+    }
+  }
+  raise_flag(a.status, flags);
+}
+
+struct Gemv1ManyMat {
+  const uint8_t* packed;
+  const __half* rnorm;
+  const float* xbar;  // [C][64]
+  __nv_bfloat16* y;
+  int64_t tile0;  // first tile of this matrix in the run
+  int d_out;
+};
+
+template <int MAXM>
+struct Gemv1ManyArgs {
+  Gemv1ManyMat m[MAXM];
+  const float2* codebook;
+  int32_t* status;
+  int64_t row_bytes;
+  int64_t ntiles;
+  int n, d_in, K, S, k, R, copies_log2;
+  unsigned stage_bytes;
+};
+
+// Shared memory of k_gemv1_many: the table, the ring, the partial sums, bars.
+size_t gemv1_many_smem(int K, int copies_log2, unsigned stage_bytes, int R, int S) {
+  return gemv1_table_bytes(K, copies_log2) + (size_t)kGemvStages * stage_bytes +
+         align16((size_t)kGemvStages * R * S * 4) + kGemvStages * sizeof(uint64_t) +
+         2 * kGemvStages * sizeof(int);
+}
+
+template <int BITS, int MAXT, int MAXM>
+__global__ void __launch_bounds__(MAXT, 1) k_gemv1_many(const __grid_constant__ Gemv1ManyArgs<MAXM> a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int copies = 1 << a.copies_log2;
+  uint32_t* tab = reinterpret_cast<uint32_t*>(smem);
+  unsigned char* stage = smem + gemv1_table_bytes(a.K, a.copies_log2);
+  float* partial = reinterpret_cast<float*>(stage + (size_t)kGemvStages * a.stage_bytes);
+  const size_t part_floats = (size_t)a.R * a.S;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(partial) +
+                                              align16(kGemvStages * part_floats * 4));
+  int* done = reinterpret_cast<int*>(bar + kGemvStages);
+  int* issued = done + kGemvStages;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int C = a.d_in / kE;
+  const int nwarps = a.S * a.k;
+
+  if (tid == 0) {
+    for (int s = 0; s < kGemvStages; ++s) {
+      mbar_init(&bar[s], 1);
+      done[s] = 0;
+      issued[s] = 0;
+    }
+    fence_mbar_init();
+  }
+  // the fp16x2 codebook table (as k_gemv1's) needs nothing from the kernels ahead
+#pragma unroll 4
+  for (int j = tid; j < a.K; j += blockDim.x) {
+    const float2 cw = __ldg(a.codebook + j);
+    const __half2 h = __floats2half2_rn(cw.x, cw.y);
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(&h);
+    for (int r = 0; r < copies; ++r)
+      tab[(j << a.copies_log2) + ((r + lane) & (copies - 1))] = u;
+  }
+  __syncthreads();
+  // the indices, r_hat and x_bar come from the kernels ahead
+  pdl_wait();
+  pdl_trigger();
+  const int64_t t_lo = (int64_t)blockIdx.x * a.ntiles / gridDim.x;
+  const int64_t t_hi = ((int64_t)blockIdx.x + 1) * a.ntiles / gridDim.x;
+  // the matrix whose tiles hold tile t (tile0 ascending)
+  auto mat_of = [&](int64_t t) {
+    int lo = 0, hi = a.n - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.m[mid].tile0 <= t) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  };
+  auto issue = [&](int64_t t, int s) {
+    const Gemv1ManyMat& M = a.m[mat_of(t)];
+    const int r0 = (int)(t - M.tile0) * a.R, nr = min(a.R, M.d_out - r0);
+    const unsigned bytes = (unsigned)(nr * a.row_bytes);
+    mbar_expect_tx(&bar[s], bytes);
+    bulk_g2s(stage + (size_t)s * a.stage_bytes, M.packed + (int64_t)r0 * a.row_bytes, bytes, &bar[s]);
+  };
+  if (tid == 0) {
+    for (int s = 0; s < kGemvStages && t_lo + s < t_hi; ++s) {
+      issue(t_lo + s, s);
+      issued[s] = 1;
+    }
+  }
+  const int sl = warp % a.S, kk = warp / a.S;
+  const int c = sl * 32 + lane;
+  const bool active = c < C;
+  const uint32_t copy = (uint32_t)lane & (uint32_t)(copies - 1);
+  float xr[kE];
+  int cur = -1;
+  int flags = 0;
+  int it = 0;
+  for (int64_t t = t_lo; t < t_hi; ++t, ++it) {
+    const int st = it % kGemvStages;
+    if (!mbar_wait_bounded(&bar[st], (unsigned)(it / kGemvStages) & 1u)) {
+      flags |= QAMW_STATUS_TIMEOUT;
+      break;
+    }
+    const int mi = mat_of(t);
+    const Gemv1ManyMat& M = a.m[mi];
+    if (mi != cur) {  // this lane's chunk of the matrix's x_bar
+      cur = mi;
+      if (active) {
+        const float4* xp = reinterpret_cast<const float4*>(M.xbar + (int64_t)c * kE);
+#pragma unroll
+        for (int q = 0; q < kE / 4; ++q) {
+          const float4 f = __ldg(xp + q);
+          xr[4 * q] = f.x;
+          xr[4 * q + 1] = f.y;
+          xr[4 * q + 2] = f.z;
+          xr[4 * q + 3] = f.w;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < kE; ++j) xr[j] = 0.f;
+      }
+    }
+    const int r0 = (int)(t - M.tile0) * a.R, nr = min(a.R, M.d_out - r0);
+    const unsigned char* buf = stage + (size_t)st * a.stage_bytes;
+    float* part = partial + st * part_floats;
+    for (int rl = kk; rl < nr; rl += a.k) {
+      float acc0 = 0.f, acc1 = 0.f;
+      if (active) {
+        const uint32_t* src =
+            reinterpret_cast<const uint32_t*>(buf + (size_t)rl * a.row_bytes) + (size_t)c * BITS;
+        uint32_t w[BITS];
+#pragma unroll
+        for (int q = 0; q < BITS; ++q) w[q] = src[q];
+        dot_pairs<BITS>(w, tab, a.copies_log2, copy, xr, acc0, acc1,
+                        std::make_integer_sequence<int, kQ>{});
+      }
+      float acc = acc0 + acc1;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) part[rl * a.S + sl] = acc;
+    }
+    int last = 0;
+    if (lane == 0) {
+      __threadfence_block();
+      last = atomicAdd(&done[st], 1) == nwarps - 1;
+    }
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) {
+      __threadfence_block();
+      for (int r = lane; r < nr; r += 32) {
+        float sum = 0.f;
+        for (int s = 0; s < a.S; ++s) sum += part[r * a.S + s];
+        M.y[r0 + r] = __float2bfloat16_rn(sum * __half2float(M.rnorm[r0 + r]));
+      }
+      __syncwarp();
+      if (lane == 0) {
+        done[st] = 0;
+        if (t + kGemvStages < t_hi) {
+          issue(t + kGemvStages, st);
+          issued[st] += 1;
+        }
+      }
+    }
+  }
+  // after a timeout: let the copies still in flight land before this CTA's
+  // shared memory goes away
+  __syncthreads();
+  if (tid == 0) {
+    for (int s = 0; s < kGemvStages; ++s)
+      if (issued[s] > 0) mbar_wait_bounded(&bar[s], (unsigned)(issued[s] - 1) & 1u);
+  }
+  raise_flag(a.status, flags);
+}
+
+// One run: x_bar of its matrices, then their products.
+template <int BITS>
+cudaError_t run_gemv1_many(const qamw_matrix* const* ms, int n, const uint16_t* const* xs,
+                           uint16_t* const* ys, float* const* xbars, int32_t* d_status,
+                           cudaStream_t stream) {
+  const qamw_matrix& f = *ms[0];
+  {
+    Xbar1Args<kGemvManyMax> xa;
+    for (int i = 0; i < n; ++i) {
+      xa.m[i].x = reinterpret_cast<const __nv_bfloat16*>(xs[i]);
+      xa.m[i].sigma = reinterpret_cast<const __half*>(ms[i]->sigma);
+      xa.m[i].scale = reinterpret_cast<const __half*>(ms[i]->chan_scale);
+      xa.m[i].xbar = xbars[i];
+      xa.m[i].seed = ms[i]->mask_seed;
+    }
+    xa.status = d_status;
+    xa.n = n;
+    xa.d_in = f.d_in;
+    xa.block = f.block;
+    const int64_t V = (int64_t)n * (f.d_in / kE);
+    cudaError_t err = launch_pdl(k_xbar1_many<kGemvManyMax>,
+                                 dim3((unsigned)((V + kXb1Threads - 1) / kXb1Threads)),
+                                 dim3(kXb1Threads), 0, stream, xa);
+    if (err != cudaSuccess) return err;
+  }
+  Gemv1ManyArgs<kGemvManyMax> a;
+  a.codebook = reinterpret_cast<const float2*>(f.codebook);
+  a.status = d_status;
+  a.row_bytes = f.row_bytes;
+  a.n = n;
+  a.d_in = f.d_in;
+  a.K = 1 << f.bits;
+  const int C = f.d_in / kE;
+  a.S = (C + 31) / 32;
+  a.k = a.S <= 16 ? 16 / a.S : 1;  // 16 warps (512 threads) per SM
+  int R = (int)(20480 / f.row_bytes);
+  R = R < a.k ? a.k : (R / a.k) * a.k;
+  a.R = R;
+  a.stage_bytes = (unsigned)(R * f.row_bytes);
+  int64_t tiles = 0;
+  for (int i = 0; i < n; ++i) {
+    a.m[i].packed = ms[i]->packed;
+    a.m[i].rnorm = reinterpret_cast<const __half*>(ms[i]->row_norm);
+    a.m[i].xbar = xbars[i];
+    a.m[i].y = reinterpret_cast<__nv_bfloat16*>(ys[i]);
+    a.m[i].tile0 = tiles;
+    a.m[i].d_out = ms[i]->d_out;
+    tiles += (ms[i]->d_out + R - 1) / R;
+  }
+  a.ntiles = tiles;
+  int cl = a.K <= 1024 ? 5 : 4;
+  while (cl > 0 && gemv1_many_smem(a.K, cl, a.stage_bytes, R, a.S) > 227 * 1024) --cl;
+  a.copies_log2 = cl;
+  const size_t smem = gemv1_many_smem(a.K, cl, a.stage_bytes, R, a.S);
+  if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
+  const int threads = 32 * a.S * a.k;
+  const void* fn = threads <= 256
+                       ? reinterpret_cast<const void*>(&k_gemv1_many<BITS, 256, kGemvManyMax>)
+                       : reinterpret_cast<const void*>(&k_gemv1_many<BITS, 512, kGemvManyMax>);
+  cudaError_t err = allow_smem(fn, smem);
+  if (err != cudaSuccess) return err;
+  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  if (threads <= 256)
+    return launch_pdl(k_gemv1_many<BITS, 256, kGemvManyMax>, dim3(grid), dim3(threads), smem,
+                      stream, a);
+  return launch_pdl(k_gemv1_many<BITS, 512, kGemvManyMax>, dim3(grid), dim3(threads), smem, stream,
+                    a);
 }
 
 // ------------------------------------------------------------- batch 2..16
@@ -693,6 +1028,63 @@ cudaError_t launch_decode_gemv(const qamw_matrix& m, const uint16_t* d_x, int ba
     case 11: return gemv_bits<11>(m, d_x, batch, xbar, d_y, d_status, stream);
     default: return cudaErrorInvalidValue;
   }
+}
+
+size_t gemv_many_workspace_bytes(const qamw_matrix* ms, int n) {
+  size_t b = 0;
+  for (int i = 0; i < n; ++i)
+    if (ms[i].d_out > 0) b += ((size_t)ms[i].d_in * sizeof(float) + 255) & ~(size_t)255;
+  return b;
+}
+
+cudaError_t launch_decode_gemv_many(const qamw_matrix* ms, int n, const uint16_t* const* d_x,
+                                    uint16_t* const* d_y, void* d_ws, int32_t* d_status,
+                                    cudaStream_t stream) {
+  // runs of up to kGemvManyMax consecutive matrices with the same d_in, block,
+  // bits and codebook; x_bar of matrix i at its offset in the workspace
+  std::vector<const qamw_matrix*> g;
+  std::vector<const uint16_t*> gx;
+  std::vector<uint16_t*> gy;
+  std::vector<float*> gb;
+  auto flush = [&]() -> cudaError_t {
+    if (g.empty()) return cudaSuccess;
+    cudaError_t e;
+    switch (g[0]->bits) {
+#define QAMW_GEMV_MANY_CASE(B)                                                                 \
+  case B:                                                                                     \
+    e = run_gemv1_many<B>(g.data(), (int)g.size(), gx.data(), gy.data(), gb.data(), d_status, \
+                          stream);                                                            \
+    break;
+      QAMW_GEMV_MANY_CASE(1) QAMW_GEMV_MANY_CASE(2) QAMW_GEMV_MANY_CASE(3) QAMW_GEMV_MANY_CASE(4)
+      QAMW_GEMV_MANY_CASE(5) QAMW_GEMV_MANY_CASE(6) QAMW_GEMV_MANY_CASE(7) QAMW_GEMV_MANY_CASE(8)
+      QAMW_GEMV_MANY_CASE(9) QAMW_GEMV_MANY_CASE(10) QAMW_GEMV_MANY_CASE(11)
+#undef QAMW_GEMV_MANY_CASE
+      default: e = cudaErrorInvalidValue;
+    }
+    g.clear();
+    gx.clear();
+    gy.clear();
+    gb.clear();
+    return e;
+  };
+  unsigned char* ws = static_cast<unsigned char*>(d_ws);
+  for (int i = 0; i < n; ++i) {
+    if (ms[i].d_out == 0) continue;
+    if (!g.empty()) {
+      const qamw_matrix& f = *g[0];
+      if (f.d_in != ms[i].d_in || f.block != ms[i].block || f.bits != ms[i].bits ||
+          f.codebook != ms[i].codebook || (int)g.size() == kGemvManyMax) {
+        const cudaError_t e = flush();
+        if (e != cudaSuccess) return e;
+      }
+    }
+    g.push_back(&ms[i]);
+    gx.push_back(d_x[i]);
+    gy.push_back(d_y[i]);
+    gb.push_back(reinterpret_cast<float*>(ws));
+    ws += ((size_t)ms[i].d_in * sizeof(float) + 255) & ~(size_t)255;
+  }
+  return flush();
 }
 
 }  // namespace qamw

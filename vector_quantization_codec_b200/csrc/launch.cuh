@@ -109,5 +109,10 @@ cudaError_t launch_decode_gemm(const qamw_matrix& m, const uint16_t* d_x, int nt
 cudaError_t launch_decode_gemv(const qamw_matrix& m, const uint16_t* d_x, int batch,
                                uint16_t* d_y, void* d_ws, int32_t* d_status,
                                cudaStream_t stream);
+// Batch-1 products of n matrices (workspace: gemv_many_workspace_bytes).
+size_t gemv_many_workspace_bytes(const qamw_matrix* ms, int n);
+cudaError_t launch_decode_gemv_many(const qamw_matrix* ms, int n, const uint16_t* const* d_x,
+                                    uint16_t* const* d_y, void* d_ws, int32_t* d_status,
+                                    cudaStream_t stream);
 
 }  // namespace qamw

@@ -48,7 +48,8 @@ EXPORTS = ("qamw_row_bytes", "qamw_default_block", "qamw_bits_per_weight",
            "qamw_train_codebook", "qamw_build_prefilter", "qamw_encode", "qamw_channel_scales",
            "qamw_calibrate_sigma", "qamw_calibrate_many", "qamw_calibrate_many_workspace_bytes",
            "qamw_encode_rows", "qamw_decode", "qamw_decode_many",
-           "qamw_decode_gemv", "qamw_decode_gemm",
+           "qamw_decode_gemv", "qamw_decode_gemv_many", "qamw_decode_gemv_many_workspace_bytes",
+           "qamw_decode_gemm",
            "qamw_decode_gemv_noalloc", "qamw_polar_codebook", "qamw_encode_rows_polar",
            "qamw_scalar_codebook", "qamw_encode_rows_scalar",
            "qamw_normalised_pairs", "qamw_selftest_wait_timeout")
@@ -92,6 +93,9 @@ def _load() -> C.CDLL:
         "qamw_decode": (I, [C.POINTER(qamw_matrix), V, V, V]),
         "qamw_decode_many": (I, [C.POINTER(qamw_matrix), I, C.POINTER(C.c_void_p), V, V]),
         "qamw_decode_gemv": (I, [C.POINTER(qamw_matrix), V, I, V, V, SZ, V, V]),
+        "qamw_decode_gemv_many": (I, [C.POINTER(qamw_matrix), I, C.POINTER(C.c_void_p),
+                                      C.POINTER(C.c_void_p), V, SZ, V, V]),
+        "qamw_decode_gemv_many_workspace_bytes": (SZ, [C.POINTER(qamw_matrix), I]),
         "qamw_decode_gemm": (I, [C.POINTER(qamw_matrix), V, I, V, V, SZ, V, V]),
         "qamw_decode_gemv_noalloc": (I, [C.POINTER(qamw_matrix), V, I, V, V, V]),
         "qamw_polar_codebook": (I, [I, V, V]),
@@ -414,6 +418,32 @@ def qamw_decode_gemv(m: EncodedMatrix, x: torch.Tensor, y: torch.Tensor | None =
                                _p(status), _s(stream))
     _check("qamw_decode_gemv", rc)
     return y
+
+
+def qamw_decode_gemv_many_workspace_bytes(ms: list) -> int:
+    return int(_lib.qamw_decode_gemv_many_workspace_bytes(_matrix_array(ms), len(ms)))
+
+
+def qamw_decode_gemv_many(ms: list, xs: list, ys: list | None = None,
+                          workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                          stream=None) -> list:
+    """Batch-1 y_i = x_i W_hat_i^T of every matrix of `ms` in one call (x_i: bf16
+    [d_in] or [1, d_in]; y_i: bf16 [1, d_out])."""
+    n = len(ms)
+    if len(xs) != n or (ys is not None and len(ys) != n):
+        raise ValueError("one activation (and output) per matrix")
+    if ys is None:
+        ys = [torch.empty((1, m.d_out), dtype=torch.bfloat16, device=x.device) for m, x in zip(ms, xs)]
+    arr = _matrix_array(ms)
+    if workspace is None:
+        workspace = _workspace(int(_lib.qamw_decode_gemv_many_workspace_bytes(arr, n)),
+                               xs[0].device if n else torch.device("cuda"))
+    xp = (C.c_void_p * max(n, 1))(*[x.data_ptr() for x in xs])
+    yp = (C.c_void_p * max(n, 1))(*[y.data_ptr() for y in ys])
+    rc = _lib.qamw_decode_gemv_many(arr, n, xp, yp, _p(workspace), workspace.numel(), _p(status),
+                                    _s(stream))
+    _check("qamw_decode_gemv_many", rc)
+    return ys
 
 
 def qamw_decode_gemm(m: EncodedMatrix, x: torch.Tensor, y: torch.Tensor | None = None,
