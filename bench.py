@@ -923,7 +923,7 @@ def run_single_stage(args) -> dict:
                         dtype=torch.uint8, device=dev)
     W_hat = torch.empty((rows, d_in), dtype=torch.bfloat16, device=dev)
     y = torch.empty((args.batch, rows), dtype=torch.bfloat16, device=dev)
-    count = args.count if args.only == "gemv_many" else 1
+    count = args.count if args.only in ("gemv_many", "calibrate_many") else 1
     if args.only == "gemv_many":
         # `count` distinct encodings of W (own index buffers: more than L2 holds)
         mlist = [m]
@@ -935,6 +935,12 @@ def run_single_stage(args) -> dict:
         yl = [torch.empty((1, rows), dtype=torch.bfloat16, device=dev) for _ in range(count)]
         ws_many = torch.empty(max(16, qamw.qamw_decode_gemv_many_workspace_bytes(mlist)),
                               dtype=torch.uint8, device=dev)
+    if args.only == "calibrate_many":
+        # `count` matrices calibrated from the same W (own s and sigma)
+        clist = [m] + [qamw.EncodedMatrix.empty(rows, d_in, BLOCK, bits, codebook, i, prefilter)
+                       for i in range(1, count)]
+        ws_cm = torch.empty(max(16, qamw.qamw_calibrate_many_workspace_bytes(clist)),
+                            dtype=torch.uint8, device=dev)
     fns = {
         "encode": lambda: qamw.qamw_encode_rows(W, m),
         "calibrate": lambda: qamw.qamw_calibrate_sigma(W, m, workspace=ws_cal),
@@ -942,6 +948,8 @@ def run_single_stage(args) -> dict:
         "gemv": lambda: qamw.qamw_decode_gemv(m, x, y, workspace=ws_g),
         "gemm": lambda: qamw.qamw_decode_gemm(m, x, y, workspace=ws_gm),
         "gemv_many": lambda: qamw.qamw_decode_gemv_many(mlist, xl, yl, workspace=ws_many),
+        "calibrate_many": lambda: qamw.qamw_calibrate_many([W] * count, clist, [act] * count, ALPHA,
+                                                           workspace=ws_cm),
         "train": lambda: qamw.qamw_train_codebook(samples, bits, 1, codebook),
     }
     fn = fns[args.only]
@@ -974,7 +982,7 @@ def run_single_stage(args) -> dict:
     out = dict(stage=args.only, rows=rows, d_in=d_in, bits=bits, batch=args.batch, ms=ms,
                timing="eager" if args.eager else "cuda graph of back-to-back calls",
                Mweights_per_s=count * rows * d_in / (ms * 1e-3) / 1e6)
-    if args.only == "gemv_many":
+    if count > 1:
         out["matrices"] = count
     if key:
         out["GB_per_s"] = count * ab[key] / (ms * 1e-3) / 1e9
@@ -996,14 +1004,15 @@ def main(argv=None) -> int:
     ap.add_argument("--ref-rows", type=int, default=ORACLE_SAMPLE_ROWS,
                     help="--impl reference: rows of each sample step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["encode", "calibrate", "decode", "gemv", "gemv_many", "gemm",
-                                       "train"],
+    ap.add_argument("--only", choices=["encode", "calibrate", "calibrate_many", "decode", "gemv",
+                                       "gemv_many", "gemm", "train"],
                     help="profiling mode: time one stage alone (no step, no JSON contract)")
     ap.add_argument("--rows", type=int, default=16384, help="--only: rows of the matrix")
     ap.add_argument("--din", type=int, default=4096, help="--only: columns of the matrix")
     ap.add_argument("--bits", type=int, default=BITS, help="--only: bits per pair")
     ap.add_argument("--batch", type=int, default=1, help="--only gemv / gemm: batch columns / tokens")
-    ap.add_argument("--count", type=int, default=16, help="--only gemv_many: matrices in the list")
+    ap.add_argument("--count", type=int, default=16,
+                    help="--only gemv_many / calibrate_many: matrices in the list")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--eager", action="store_true", help="--only: time eager calls, not a graph")
     args = ap.parse_args(argv)
