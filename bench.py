@@ -482,6 +482,7 @@ def run_gpu(args) -> dict | None:
     # ---- decode-GEMV on the MLP shapes at batch 1 / 4 / 16 (cycling 32 layers)
     gemv_lines = run_gemv_lines(args, wl, dev, stream, hbm)
     gemm_lines = run_gemm_lines(args, wl, dev, stream, hbm, peaks["bf16_tflops"])
+    dense_context = run_dense_context(args, wl, dev, stream, hbm)
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(args, wl, stream, world, dev)
     del wl
@@ -518,6 +519,7 @@ def run_gpu(args) -> dict | None:
                                    frac_hbm=ab["gemv"] / (gemv_ms * 1e-3) / 1e9 / hbm),
         "decode_gemv_mlp": gemv_lines,
         "decode_gemm_prefill": gemm_lines,
+        "gpu_context_dense_bf16": dense_context,
         "train": dict(ms=train_ms, samples=TRAIN_N, iters=TRAIN_ITERS, K=1 << BITS,
                       note="per-codec constant, outside the step"),
     }
@@ -617,6 +619,61 @@ def run_gemv_lines(args, wl, dev, stream, hbm) -> dict:
                 gflops=2.0 * b * d0["d_out"] * d0["d_in"] / (ms * 1e-3) / 1e9,
                 matrices_cycled=len(sel))
     wl.check_status("decode-GEMV lines")
+    return lines
+
+
+def run_dense_context(args, wl, dev, stream, hbm) -> dict:
+    """Context on the GPU, not the target: torch's dense BF16 product x @ W^T on
+    the same 11008x4096 and 4096x11008 weights (BF16, 90 MB each) at the batches
+    of the decode-GEMV lines and the token counts of the decode-GEMM lines, and
+    a BF16 copy of the same bytes (W into a scratch buffer).  Each line is one
+    CUDA graph over the 32 layers' matrices of that shape."""
+    import torch
+
+    from vector_quantization_codec_b200 import synth
+    lines = {}
+    for name in ("gate", "down"):
+        sel = [i for i, d in enumerate(wl.mats) if d["name"] == name]
+        d0 = wl.mats[sel[0]]
+        wbytes = 2 * d0["d_out"] * d0["d_in"]
+        for b in tuple(GEMV_BATCHES) + tuple(GEMM_TOKENS):
+            xs = [torch.from_numpy(synth.gemv_x(b, d0["d_in"], seed=7000 + i)).to(torch.bfloat16).to(dev)
+                  for i in sel]
+            ys = [torch.empty((b, d0["d_out"]), dtype=torch.bfloat16, device=dev) for _ in sel]
+
+            def calls():
+                for i, x, y in zip(sel, xs, ys):
+                    torch.matmul(x, wl.W[i].t(), out=y)
+
+            calls()
+            torch.cuda.synchronize()
+            g = capture(calls)
+            g.replay()
+            ms = time_graph(g, max(3, args.steps // 2), stream) / len(sel)
+            del g
+            byts = wbytes + 2 * b * (d0["d_in"] + d0["d_out"])
+            lines[f"{d0['d_out']}x{d0['d_in']}_dense_bf16_m{b}"] = dict(
+                us_per_call=ms * 1e3, GB_per_s=byts / (ms * 1e-3) / 1e9,
+                tflops=2.0 * b * d0["d_out"] * d0["d_in"] / (ms * 1e-3) / 1e12)
+        scratch = torch.empty_like(wl.W[sel[0]])
+
+        def copies():
+            for i in sel:
+                scratch.copy_(wl.W[i])
+
+        copies()
+        torch.cuda.synchronize()
+        g = capture(copies)
+        g.replay()
+        ms = time_graph(g, max(3, args.steps // 2), stream) / len(sel)
+        del g
+        lines[f"{d0['d_out']}x{d0['d_in']}_bf16_copy"] = dict(
+            us_per_call=ms * 1e3, GB_per_s=2 * wbytes / (ms * 1e-3) / 1e9,
+            frac_hbm=2 * wbytes / (ms * 1e-3) / 1e9 / hbm)
+        del scratch
+    lines["note"] = ("torch.matmul (cuBLAS) on the uncompressed BF16 weights, and torch copy_ of "
+                     "them: context for the decode-GEMV and decode-GEMM lines, not their target; "
+                     "the dense path reads 2 B/weight, the codec 11/16 B/weight")
     return lines
 
 

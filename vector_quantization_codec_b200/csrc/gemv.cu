@@ -8,7 +8,7 @@
 //
 // batch 1 (k_gemv1): one persistent CTA per SM.  Each warp owns a fixed slice of
 //   32 chunks (1024 pairs) and computes xbar for it straight into registers.
-//   Tiles of R whole rows of packed indices stream into a 3-stage shared ring
+//   Tiles of R whole rows of packed indices (~45 KB) stream into a 2-stage shared ring
 //   through cp.async.bulk (TMA, mbarrier completion, bounded waits); codewords
 //   come from an fp16x2 copy of the codebook replicated so that a warp's 32
 //   random lookups hit at most 2 lanes per bank.  Per-slice partial dot
@@ -29,7 +29,11 @@ namespace {
 
 // ------------------------------------------------------------------ batch 1
 
-constexpr int kGemvStages = 3;
+constexpr int kGemvStages = 2;
+// Index bytes per tile of whole rows: two or more rows per warp at the common
+// widths, so a warp's per-tile cost (its wait, its share of the row sums)
+// spreads over more pairs.
+constexpr int kGemvTileBytes = 46080;
 
 struct Gemv1Args {
   const uint8_t* packed;
@@ -294,8 +298,8 @@ cudaError_t run_gemv1(const qamw_matrix& m, const uint16_t* d_x, uint16_t* d_y,
   const int C = m.d_in / kE;
   a.S = (C + 31) / 32;
   a.k = a.S <= 16 ? 16 / a.S : 1;  // 16 warps (512 threads) per SM
-  // ~20 KB of indices per stage, whole rows, a multiple of k rows
-  int R = (int)(20480 / m.row_bytes);
+  // ~45 KB of indices per stage, whole rows, a multiple of k rows
+  int R = (int)(kGemvTileBytes / m.row_bytes);
   R = R < a.k ? a.k : (R / a.k) * a.k;
   a.R = R;
   a.stage_bytes = (unsigned)(R * m.row_bytes);
@@ -329,6 +333,8 @@ cudaError_t run_gemv1(const qamw_matrix& m, const uint16_t* d_x, uint16_t* d_y,
 // matrix changes.
 
 constexpr int kGemvManyMax = 64;
+constexpr int kGemvManyStages = kGemvStages;       // ring depth of k_gemv1_many
+constexpr int kGemvManyTileBytes = kGemvTileBytes;  // index bytes per tile (whole rows)
 constexpr int kXb1Threads = 128;
 
 struct Xbar1Mat {
@@ -431,9 +437,9 @@ struct Gemv1ManyArgs {
 
 // Shared memory of k_gemv1_many: the table, the ring, the partial sums, bars.
 size_t gemv1_many_smem(int K, int copies_log2, unsigned stage_bytes, int R, int S) {
-  return gemv1_table_bytes(K, copies_log2) + (size_t)kGemvStages * stage_bytes +
-         align16((size_t)kGemvStages * R * S * 4) + kGemvStages * sizeof(uint64_t) +
-         2 * kGemvStages * sizeof(int);
+  return gemv1_table_bytes(K, copies_log2) + (size_t)kGemvManyStages * stage_bytes +
+         align16((size_t)kGemvManyStages * R * S * 4) + kGemvManyStages * sizeof(uint64_t) +
+         2 * kGemvManyStages * sizeof(int);
 }
 
 template <int BITS, int MAXT, int MAXM>
@@ -442,18 +448,18 @@ __global__ void __launch_bounds__(MAXT, 1) k_gemv1_many(const __grid_constant__ 
   const int copies = 1 << a.copies_log2;
   uint32_t* tab = reinterpret_cast<uint32_t*>(smem);
   unsigned char* stage = smem + gemv1_table_bytes(a.K, a.copies_log2);
-  float* partial = reinterpret_cast<float*>(stage + (size_t)kGemvStages * a.stage_bytes);
+  float* partial = reinterpret_cast<float*>(stage + (size_t)kGemvManyStages * a.stage_bytes);
   const size_t part_floats = (size_t)a.R * a.S;
   uint64_t* bar = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(partial) +
-                                              align16(kGemvStages * part_floats * 4));
-  int* done = reinterpret_cast<int*>(bar + kGemvStages);
-  int* issued = done + kGemvStages;
+                                              align16(kGemvManyStages * part_floats * 4));
+  int* done = reinterpret_cast<int*>(bar + kGemvManyStages);
+  int* issued = done + kGemvManyStages;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int C = a.d_in / kE;
   const int nwarps = a.S * a.k;
 
   if (tid == 0) {
-    for (int s = 0; s < kGemvStages; ++s) {
+    for (int s = 0; s < kGemvManyStages; ++s) {
       mbar_init(&bar[s], 1);
       done[s] = 0;
       issued[s] = 0;
@@ -492,7 +498,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_gemv1_many(const __grid_constant__ 
     bulk_g2s(stage + (size_t)s * a.stage_bytes, M.packed + (int64_t)r0 * a.row_bytes, bytes, &bar[s]);
   };
   if (tid == 0) {
-    for (int s = 0; s < kGemvStages && t_lo + s < t_hi; ++s) {
+    for (int s = 0; s < kGemvManyStages && t_lo + s < t_hi; ++s) {
       issue(t_lo + s, s);
       issued[s] = 1;
     }
@@ -506,8 +512,8 @@ __global__ void __launch_bounds__(MAXT, 1) k_gemv1_many(const __grid_constant__ 
   int flags = 0;
   int it = 0;
   for (int64_t t = t_lo; t < t_hi; ++t, ++it) {
-    const int st = it % kGemvStages;
-    if (!mbar_wait_bounded(&bar[st], (unsigned)(it / kGemvStages) & 1u)) {
+    const int st = it % kGemvManyStages;
+    if (!mbar_wait_bounded(&bar[st], (unsigned)(it / kGemvManyStages) & 1u)) {
       flags |= QAMW_STATUS_TIMEOUT;
       break;
     }
@@ -565,8 +571,8 @@ __global__ void __launch_bounds__(MAXT, 1) k_gemv1_many(const __grid_constant__ 
       __syncwarp();
       if (lane == 0) {
         done[st] = 0;
-        if (t + kGemvStages < t_hi) {
-          issue(t + kGemvStages, st);
+        if (t + kGemvManyStages < t_hi) {
+          issue(t + kGemvManyStages, st);
           issued[st] += 1;
         }
       }
@@ -576,7 +582,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_gemv1_many(const __grid_constant__ 
   // shared memory goes away
   __syncthreads();
   if (tid == 0) {
-    for (int s = 0; s < kGemvStages; ++s)
+    for (int s = 0; s < kGemvManyStages; ++s)
       if (issued[s] > 0) mbar_wait_bounded(&bar[s], (unsigned)(issued[s] - 1) & 1u);
   }
   raise_flag(a.status, flags);
@@ -617,7 +623,7 @@ cudaError_t run_gemv1_many(const qamw_matrix* const* ms, int n, const uint16_t* 
   const int C = f.d_in / kE;
   a.S = (C + 31) / 32;
   a.k = a.S <= 16 ? 16 / a.S : 1;  // 16 warps (512 threads) per SM
-  int R = (int)(20480 / f.row_bytes);
+  int R = (int)(kGemvManyTileBytes / f.row_bytes);
   R = R < a.k ? a.k : (R / a.k) * a.k;
   a.R = R;
   a.stage_bytes = (unsigned)(R * f.row_bytes);
