@@ -151,7 +151,7 @@ __host__ __device__ inline int calib_rpc(int d_in) {
   return r < 1 ? 1 : (r > kCalPer ? kCalPer : r);
 }
 
-// Shared memory of k_calib_rows for a matrix: fT [d_in] | red [RPC][P] |
+// Shared memory of k_calib_rows for a matrix: fT4 [d_in / 4] (quads) | red [RPC][P] |
 // part [512] | rsum [32].
 __host__ __device__ inline size_t calib_rows_smem(int d_in) {
   return ((size_t)d_in + (size_t)calib_rpc(d_in) * (d_in / 2) + kCalThreads + kCalPer) * sizeof(float);
@@ -164,14 +164,14 @@ __global__ void __launch_bounds__(kCalThreads) k_calib_rows(const __grid_constan
   const T* __restrict__ W = static_cast<const T*>(M.W);
   const int d_in = M.d_in, C = d_in / kE, P = d_in / 2;
   const int RPC = calib_rpc(d_in);
-  float* fT = sm;                       // [j][c]: D * s of column 64c + j
+  float4* fT4 = reinterpret_cast<float4*>(sm);  // [j/4][c]: D * s of columns 64c + j .. + 3
   float* red = sm + d_in;               // [g][q][c]
   float* part = red + (size_t)RPC * P;  // [blockDim] partial sums of squares
   float* rsum = part + kCalThreads;     // [RPC]
   pdl_wait();  // s comes from the kernel ahead
   pdl_trigger();
   const uint64_t seed = M.seed;
-  fill_interleaved<kE>(fT, M.s, d_in, C, [=](int j, float v) {
+  fill_quads<kE>(fT4, M.s, d_in, C, [=](int j, float v) {
     return mask_negative(seed, (uint32_t)j) ? -v : v;
   });
   __syncthreads();
@@ -194,9 +194,16 @@ __global__ void __launch_bounds__(kCalThreads) k_calib_rows(const __grid_constan
     if (active) {
       load64(W + (int64_t)row * d_in + (int64_t)c * kE, x);
 #pragma unroll
-      for (int j = 0; j < kE; ++j) {
-        x[j] *= fT[j * C + c];
-        ss = fmaf(x[j], x[j], ss);
+      for (int i = 0; i < kE / 4; ++i) {  // four factors per 16-byte load, element order kept
+        const float4 f = fT4[i * C + c];
+        x[4 * i] *= f.x;
+        ss = fmaf(x[4 * i], x[4 * i], ss);
+        x[4 * i + 1] *= f.y;
+        ss = fmaf(x[4 * i + 1], x[4 * i + 1], ss);
+        x[4 * i + 2] *= f.z;
+        ss = fmaf(x[4 * i + 2], x[4 * i + 2], ss);
+        x[4 * i + 3] *= f.w;
+        ss = fmaf(x[4 * i + 3], x[4 * i + 3], ss);
       }
     } else {
 #pragma unroll
@@ -252,7 +259,7 @@ __global__ void __launch_bounds__(kCalThreads) k_calib_rows(const __grid_constan
 // the current row.
 template <typename T, int MAXM>
 __global__ void __launch_bounds__(kCalThreads) k_calib_ext(const __grid_constant__ CalibLaunch<MAXM> L) {
-  extern __shared__ __align__(16) float fT[];  // [j][c]
+  extern __shared__ __align__(16) float4 fT4[];  // [j/4][c]
   __shared__ float part[kCalThreads];
   __shared__ float rtot;
   __shared__ int total;
@@ -276,7 +283,7 @@ __global__ void __launch_bounds__(kCalThreads) k_calib_ext(const __grid_constant
   __syncthreads();
   if (total < kCalRows && d_out > kCalRows) {
     const uint64_t seed = M.seed;
-    fill_interleaved<kE>(fT, M.s, d_in, C, [=](int j, float v) {
+    fill_quads<kE>(fT4, M.s, d_in, C, [=](int j, float v) {
       return mask_negative(seed, (uint32_t)j) ? -v : v;
     });
     __syncthreads();
@@ -288,9 +295,16 @@ __global__ void __launch_bounds__(kCalThreads) k_calib_ext(const __grid_constant
       if (active_c) {
         load64(W + (int64_t)row * d_in + (int64_t)c * kE, x);
 #pragma unroll
-        for (int j = 0; j < kE; ++j) {
-          x[j] *= fT[j * C + c];
-          ss = fmaf(x[j], x[j], ss);
+        for (int i = 0; i < kE / 4; ++i) {
+          const float4 f = fT4[i * C + c];
+          x[4 * i] *= f.x;
+          ss = fmaf(x[4 * i], x[4 * i], ss);
+          x[4 * i + 1] *= f.y;
+          ss = fmaf(x[4 * i + 1], x[4 * i + 1], ss);
+          x[4 * i + 2] *= f.z;
+          ss = fmaf(x[4 * i + 2], x[4 * i + 2], ss);
+          x[4 * i + 3] *= f.w;
+          ss = fmaf(x[4 * i + 3], x[4 * i + 3], ss);
         }
       } else {
 #pragma unroll
