@@ -145,56 +145,93 @@ __global__ void __launch_bounds__(kScaleThreads) k_scales(const __grid_constant_
 //                  (n sqrt(pi/2))), 1 when that rounds to 0.
 constexpr int kCalThreads = 512;
 constexpr int kCalPer = kCalRows / kCalCtas;  // rows per CTA: 32
+// k_calib_rows gives each thread CE consecutive columns of a row: 32 (16 pairs)
+// when every matrix of the launch has d_in <= 32 x 512, so that a thread's
+// values and sums fit its registers with two CTAs per SM, else 64.  The
+// butterflies give bitwise the same rotation for either width.
+constexpr int kCalNarrow = 32;
+constexpr int kCalNarrowMaxDin = kCalNarrow * kCalThreads;
 
-__host__ __device__ inline int calib_rpc(int d_in) {
-  const int r = kCalThreads / (d_in / kE);
+__host__ __device__ inline int calib_rpc(int d_in, int ce) {
+  const int r = kCalThreads / (d_in / ce);
   return r < 1 ? 1 : (r > kCalPer ? kCalPer : r);
 }
 
-// Shared memory of k_calib_rows for a matrix: fT4 [d_in / 4] (quads) | red [RPC][P] |
-// part [512] | rsum [32].
-__host__ __device__ inline size_t calib_rows_smem(int d_in) {
-  return ((size_t)d_in + (size_t)calib_rpc(d_in) * (d_in / 2) + kCalThreads + kCalPer) * sizeof(float);
+// Shared memory of k_calib_rows for a matrix: fT4 [d_in / 4] (quads of a
+// CE-column chunk) | red [RPC][P] | part [512] | rsum [32].
+__host__ __device__ inline size_t calib_rows_smem(int d_in, int ce) {
+  return ((size_t)d_in + (size_t)calib_rpc(d_in, ce) * (d_in / 2) + kCalThreads + kCalPer) *
+         sizeof(float);
 }
 
-template <typename T, int MAXM>
-__global__ void __launch_bounds__(kCalThreads) k_calib_rows(const __grid_constant__ CalibLaunch<MAXM> L) {
+// N consecutive values of a row as fp32.
+template <int N>
+__device__ __forceinline__ void load_cols(const float* p, float (&x)[N]) {
+  const float4* s4 = reinterpret_cast<const float4*>(p);
+#pragma unroll
+  for (int t = 0; t < N / 4; ++t) {
+    const float4 v = __ldg(s4 + t);
+    x[4 * t] = v.x;
+    x[4 * t + 1] = v.y;
+    x[4 * t + 2] = v.z;
+    x[4 * t + 3] = v.w;
+  }
+}
+template <int N>
+__device__ __forceinline__ void load_cols(const __nv_bfloat16* p, float (&x)[N]) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int t = 0; t < N / 8; ++t) {
+    const uint4 v = __ldg(s4 + t);
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      x[8 * t + 2 * e] = __uint_as_float(u[e] << 16);
+      x[8 * t + 2 * e + 1] = __uint_as_float(u[e] & 0xffff0000u);
+    }
+  }
+}
+
+template <typename T, int MAXM, int kCE>
+__global__ void __launch_bounds__(kCalThreads, kCE == kCalNarrow ? 2 : 1)
+    k_calib_rows(const __grid_constant__ CalibLaunch<MAXM> L) {
   extern __shared__ __align__(16) float sm[];
+  constexpr int kQh = kCE / 2;  // pairs per thread
   const CalibMat& M = L.m[blockIdx.y];
   const T* __restrict__ W = static_cast<const T*>(M.W);
-  const int d_in = M.d_in, C = d_in / kE, P = d_in / 2;
-  const int RPC = calib_rpc(d_in);
-  float4* fT4 = reinterpret_cast<float4*>(sm);  // [j/4][c]: D * s of columns 64c + j .. + 3
+  const int d_in = M.d_in, C = d_in / kCE, P = d_in / 2;
+  const int RPC = calib_rpc(d_in, kCE);
+  float4* fT4 = reinterpret_cast<float4*>(sm);  // [j/4][c]: D * s of columns kCE c + j .. + 3
   float* red = sm + d_in;               // [g][q][c]
   float* part = red + (size_t)RPC * P;  // [blockDim] partial sums of squares
   float* rsum = part + kCalThreads;     // [RPC]
   pdl_wait();  // s comes from the kernel ahead
   pdl_trigger();
   const uint64_t seed = M.seed;
-  fill_quads<kE>(fT4, M.s, d_in, C, [=](int j, float v) {
+  fill_quads<kCE>(fT4, M.s, d_in, C, [=](int j, float v) {
     return mask_negative(seed, (uint32_t)j) ? -v : v;
   });
   __syncthreads();
   const int g = threadIdx.x / C, c = threadIdx.x - g * C;
   const bool lane_ok = g < RPC;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = kCalThreads >> 5;
-  const int nb = min(M.block, kE), lanes = max(M.block / kE, 1);
+  const int nb = min(M.block, kCE), lanes = max(M.block / kCE, 1);
   const float inv_sqrt_b = 1.0f / sqrtf((float)M.block);
   const int rows = min(M.d_out, kCalRows);
   const int t0 = blockIdx.x * kCalPer, t1 = min(t0 + kCalPer, rows);
-  float acc[kQ];
+  float acc[kQh];
 #pragma unroll
-  for (int q = 0; q < kQ; ++q) acc[q] = 0.f;
+  for (int q = 0; q < kQh; ++q) acc[q] = 0.f;
   int nz = 0, flags = 0;
   for (int base = t0; base < t1; base += RPC) {
     const int row = base + g;
     const bool active = lane_ok && row < t1;
-    float x[kE];
+    float x[kCE];
     float ss = 0.f;
     if (active) {
-      load64(W + (int64_t)row * d_in + (int64_t)c * kE, x);
+      load_cols<kCE>(W + (int64_t)row * d_in + (int64_t)c * kCE, x);
 #pragma unroll
-      for (int i = 0; i < kE / 4; ++i) {  // four factors per 16-byte load, element order kept
+      for (int i = 0; i < kCE / 4; ++i) {  // four factors per 16-byte load, element order kept
         const float4 f = fT4[i * C + c];
         x[4 * i] *= f.x;
         ss = fmaf(x[4 * i], x[4 * i], ss);
@@ -207,11 +244,11 @@ __global__ void __launch_bounds__(kCalThreads) k_calib_rows(const __grid_constan
       }
     } else {
 #pragma unroll
-      for (int j = 0; j < kE; ++j) x[j] = 0.f;
+      for (int j = 0; j < kCE; ++j) x[j] = 0.f;
     }
     part[threadIdx.x] = ss;
-    fwht_reg<kE>(x, nb);
-    fwht_lanes<kE>(x, lanes);
+    fwht_reg<kCE>(x, nb);
+    fwht_lanes<kCE>(x, lanes);
     __syncthreads();
     for (int q = warp; q < RPC; q += nwarps) {
       float t = 0.f;
@@ -228,7 +265,7 @@ __global__ void __launch_bounds__(kCalThreads) k_calib_rows(const __grid_constan
         if (c == 0) ++nz;
         const float inv = inv_sqrt_b / r;
 #pragma unroll
-        for (int q = 0; q < kQ; ++q) {
+        for (int q = 0; q < kQh; ++q) {
           const float zx = x[2 * q] * inv, zy = x[2 * q + 1] * inv;
           acc[q] += sqrtf(fmaf(zx, zx, zy * zy));
         }
@@ -238,7 +275,7 @@ __global__ void __launch_bounds__(kCalThreads) k_calib_rows(const __grid_constan
   }
   if (lane_ok) {
 #pragma unroll
-    for (int q = 0; q < kQ; ++q) red[(size_t)g * P + q * C + c] = acc[q];
+    for (int q = 0; q < kQh; ++q) red[(size_t)g * P + q * C + c] = acc[q];
   }
   // non-zero rows of this CTA: thread (g, 0) counted those of group g
   __shared__ int cnt_sh;
@@ -247,7 +284,7 @@ __global__ void __launch_bounds__(kCalThreads) k_calib_rows(const __grid_constan
   if (nz) atomicAdd(&cnt_sh, nz);
   for (int k = threadIdx.x; k < P; k += kCalThreads) {
     float v = 0.f;
-    for (int gg = 0; gg < RPC; ++gg) v += red[(size_t)gg * P + (k % kQ) * C + k / kQ];
+    for (int gg = 0; gg < RPC; ++gg) v += red[(size_t)gg * P + (k % kQh) * C + k / kQh];
     M.partial[(size_t)blockIdx.x * P + k] = v;
   }
   __syncthreads();
@@ -379,16 +416,25 @@ cudaError_t calibrate_group(const CalibLaunch<MAXM>& L, bool scales, bool sigma,
     if (err != cudaSuccess) return err;
   }
   if (!sigma) return cudaSuccess;
-  size_t smem = 0, esmem = 0;
-  int pmax = 0;
+  size_t esmem = 0;
+  int pmax = 0, dmax = 0;
   for (int i = 0; i < L.n; ++i) {
-    smem = std::max(smem, calib_rows_smem(L.m[i].d_in));
     esmem = std::max(esmem, (size_t)L.m[i].d_in * sizeof(float));
     pmax = std::max(pmax, L.m[i].d_in / 2);
+    dmax = std::max(dmax, L.m[i].d_in);
   }
-  const void* fn = reinterpret_cast<const void*>(&k_calib_rows<T, MAXM>);
+  const int ce = dmax <= kCalNarrowMaxDin ? kCalNarrow : kE;
+  size_t smem = 0;
+  for (int i = 0; i < L.n; ++i) smem = std::max(smem, calib_rows_smem(L.m[i].d_in, ce));
+  const void* fn = ce == kCalNarrow ? reinterpret_cast<const void*>(&k_calib_rows<T, MAXM, kCalNarrow>)
+                                    : reinterpret_cast<const void*>(&k_calib_rows<T, MAXM, kE>);
   if ((err = allow_smem(fn, smem)) != cudaSuccess) return err;
-  err = launch_pdl(k_calib_rows<T, MAXM>, dim3(kCalCtas, L.n), dim3(kCalThreads), smem, stream, L);
+  if (ce == kCalNarrow)
+    err = launch_pdl(k_calib_rows<T, MAXM, kCalNarrow>, dim3(kCalCtas, L.n), dim3(kCalThreads), smem,
+                     stream, L);
+  else
+    err = launch_pdl(k_calib_rows<T, MAXM, kE>, dim3(kCalCtas, L.n), dim3(kCalThreads), smem, stream,
+                     L);
   if (err != cudaSuccess) return err;
   const void* efn = reinterpret_cast<const void*>(&k_calib_ext<T, MAXM>);
   if ((err = allow_smem(efn, esmem)) != cudaSuccess) return err;
