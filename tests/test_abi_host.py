@@ -111,6 +111,11 @@ def test_matrix_argument_errors(kw, rc):
     assert qamw.lib().qamw_decode(C.byref(m), C.c_void_p(FAKE), None, None) == rc
     assert qamw.lib().qamw_decode_gemv(C.byref(m), C.c_void_p(FAKE), 1, C.c_void_p(FAKE),
                                        C.c_void_p(FAKE), 1 << 40, None, None) == rc
+    assert qamw.lib().qamw_decode_gemm(C.byref(m), C.c_void_p(FAKE), 64, C.c_void_p(FAKE),
+                                       C.c_void_p(FAKE), 1 << 40, None, None) == rc
+    one = (qamw.qamw_matrix * 1)(m)
+    assert qamw.lib().qamw_decode_gemv_many(one, 1, (C.c_void_p * 1)(FAKE), (C.c_void_p * 1)(FAKE),
+                                            C.c_void_p(FAKE), 1 << 40, None, None) == rc
 
 
 def test_encode_argument_errors():
@@ -156,6 +161,74 @@ def test_gemv_and_train_argument_errors():
     P = L.qamw_normalised_pairs
     assert P(C.c_void_p(FAKE), qamw.QAMW_DTYPE_BF16, C.byref(m), 90, 20, C.c_void_p(FAKE), None,
              None) == qamw.QAMW_ERR_SHAPE
+
+
+def _gemm_plan_bytes(d_out, d_in, ntok, sms=148):
+    """Workspace of qamw_decode_gemm re-derived from its stated plan: 64-column
+    chunks, token groups of 64 (<= 64 tokens) or 128, 128-row tiles, the units
+    shared equally over min(SMs, units / 4) CTAs, x_bar images (2 parts x 8 KB
+    per chunk and 64 tokens) and one fp32 partial sum per (CTA share of a row
+    tile and token group)."""
+    C = d_in // 64
+    NT = 128 if ntok > 64 else 64
+    TG = (ntok + NT - 1) // NT
+    ntt = TG * NT // 64
+    U = ((d_out + 127) // 128) * TG * C
+    G = min(sms, max(1, U // 4))
+    per = max(1, U // G)
+    segmax = min(G, (C - 1 + per - 1) // per + 1)
+    return C * 2 * ntt * 8192 + segmax * ntt * 64 * d_out * 4
+
+
+@pytest.mark.parametrize("d_out,d_in,ntok", [(11008, 4096, 128), (4096, 4096, 64), (4096, 11008, 3),
+                                             (300, 1024, 100), (24, 11008, 256), (64, 192, 70)])
+def test_gemm_workspace_follows_the_plan(d_out, d_in, ntok):
+    # without a device the library plans for 148 SMs
+    assert qamw.qamw_workspace_bytes(qamw.QAMW_OP_GEMM, d_out, d_in, 11, ntok) == \
+        _gemm_plan_bytes(d_out, d_in, ntok)
+
+
+def test_gemv_many_workspace_sizes():
+    ms = [_matrix(d_in=4096), _matrix(d_in=11008), _matrix(d_out=0, d_in=4096), _matrix(d_in=192)]
+    arr = (qamw.qamw_matrix * 4)(*ms)
+    # x_bar of every non-empty matrix, fp32, each rounded up to 256 bytes
+    assert qamw.lib().qamw_decode_gemv_many_workspace_bytes(arr, 4) == 4096 * 4 + 11008 * 4 + 768
+    assert qamw.lib().qamw_decode_gemv_many_workspace_bytes(arr, 0) == 0
+
+
+def test_gemm_and_gemv_many_argument_errors():
+    L = qamw.lib()
+    m = _matrix()
+    G = L.qamw_decode_gemm
+    for ntok in (0, 65537):
+        assert G(C.byref(m), C.c_void_p(FAKE), ntok, C.c_void_p(FAKE), C.c_void_p(FAKE), 1 << 40,
+                 None, None) == qamw.QAMW_ERR_INVALID
+    assert G(C.byref(m), None, 64, C.c_void_p(FAKE), C.c_void_p(FAKE), 1 << 40, None, None) == \
+        qamw.QAMW_ERR_INVALID
+    assert G(C.byref(m), C.c_void_p(FAKE + 2), 64, C.c_void_p(FAKE), C.c_void_p(FAKE), 1 << 40,
+             None, None) == qamw.QAMW_ERR_ALIGN
+    assert G(C.byref(m), C.c_void_p(FAKE), 64, C.c_void_p(FAKE), C.c_void_p(FAKE), 100, None,
+             None) == qamw.QAMW_ERR_WORKSPACE
+    assert G(C.byref(m), C.c_void_p(FAKE), 64, C.c_void_p(FAKE), C.c_void_p(FAKE + 8), 1 << 40,
+             None, None) == qamw.QAMW_ERR_ALIGN
+    empty = _matrix(d_out=0)
+    assert G(C.byref(empty), None, 64, None, None, 0, None, None) == qamw.QAMW_OK
+    M = L.qamw_decode_gemv_many
+    arr = (qamw.qamw_matrix * 2)(_matrix(), _matrix(d_in=256))
+    xs = (C.c_void_p * 2)(FAKE, FAKE)
+    ys = (C.c_void_p * 2)(FAKE, FAKE)
+    assert M(arr, -1, xs, ys, C.c_void_p(FAKE), 1 << 40, None, None) == qamw.QAMW_ERR_INVALID
+    assert M(arr, 2, None, ys, C.c_void_p(FAKE), 1 << 40, None, None) == qamw.QAMW_ERR_INVALID
+    assert M(arr, 2, (C.c_void_p * 2)(FAKE, None), ys, C.c_void_p(FAKE), 1 << 40, None, None) == \
+        qamw.QAMW_ERR_INVALID
+    assert M(arr, 2, (C.c_void_p * 2)(FAKE, FAKE + 2), ys, C.c_void_p(FAKE), 1 << 40, None, None) == \
+        qamw.QAMW_ERR_ALIGN
+    assert M(arr, 2, xs, ys, C.c_void_p(FAKE), 100, None, None) == qamw.QAMW_ERR_WORKSPACE
+    assert M(arr, 2, xs, ys, None, 1 << 40, None, None) == qamw.QAMW_ERR_WORKSPACE
+    assert M(arr, 0, None, None, None, 0, None, None) == qamw.QAMW_OK
+    # a bad matrix anywhere in the list is reported before anything is enqueued
+    bad = (qamw.qamw_matrix * 2)(_matrix(), _matrix(bits=12))
+    assert M(bad, 2, xs, ys, C.c_void_p(FAKE), 1 << 40, None, None) == qamw.QAMW_ERR_INVALID
 
 
 def test_status_strings():
