@@ -19,8 +19,9 @@
 //                   of units (tile of 128 weight rows, group of NT tokens,
 //                   K-chunk), chunks fastest; each CTA takes an equal share of
 //                   consecutive units.  Eight decode warps gather the codewords
-//                   of a chunk into swizzled A tiles (hi, lo) in shared memory,
-//                   a copy warp brings the chunk's B tiles in, one thread
+//                   of a chunk and store them (hi, lo) straight into tensor
+//                   memory as the A operand (lane = weight row), a copy warp
+//                   brings the chunk's B tiles into shared memory, one thread
 //                   issues the MMAs into an fp32 accumulator in tensor memory,
 //                   and four epilogue warps write the accumulator out as the
 //                   partial sum of the CTA's part of the (row tile, token group)
@@ -315,7 +316,8 @@ struct HalfWords {
 };
 
 // Decode warps: warp w decodes half H = w / 4 (pairs 16 H .. 16 H + 15) of the
-// 32 rows 32 (w % 4) .. + 31 of every unit into the A tiles of the unit's stage.
+// 32 rows 32 (w % 4) .. + 31 of every unit into the unit's A stage in tensor
+// memory (the warp's lane quarter: lane = row).
 // The packed words are loaded coalesced (lane i of load j takes word j * 32 + i
 // of the 32 rows' half-chunks), two units ahead, and pass through the warp's
 // word buffer to the lane of their row.
