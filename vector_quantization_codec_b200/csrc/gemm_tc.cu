@@ -51,8 +51,6 @@ constexpr int kMaxStages = 4;
 constexpr uint32_t kImg = kImgTok * kTcK * 2;    // 8 KB: one binary16 image of 64 tokens
 constexpr int kWordStride = 7;  // words per row in a decode warp's word buffer (odd)
 
-__host__ __device__ inline int tok_tiles(int ntok) { return (ntok + kImgTok - 1) / kImgTok; }
-
 // binary16 high and low parts of a pair of floats.
 __device__ __forceinline__ uint2 split_h2(float a, float b) {
   const __half2 hi = __floats2half2_rn(a, b);
